@@ -1,0 +1,158 @@
+/*
+ * gdpa.h -- C ABI of libgdpa, Generalized Dot-Product Attention on B200.
+ *
+ * GDPA (Kunlun paper review, §2.3 "GDPA" and Fig. 2; Kunlun Breakdown, "The
+ * Core Architecture and Mechanics") recasts the personalised FFN as
+ * attention: a sample's jagged behaviour sequence is the query, and weights
+ * generated from the sample's context are the keys and values.  Per sample b
+ * and head h it computes
+ *
+ *     O = phi(scale * Q K^T + beta) V
+ *
+ * where phi is an element-wise activation (SiLU, reproducing act(X W1) W2) or
+ * a row softmax (pooling, cross-attention and sliding-window self-attention),
+ * and beta is an optional per-key additive bias, or the gate log sigmoid(G)
+ * of the Kunlun reproduction notes ("Core equations").  The optional band
+ * (window_left, window_right) is the sliding window of the Kunlun paper
+ * review, §2.5: key j is visible to query i iff
+ *     (window_left < 0 || j >= i - window_left) &&
+ *     (window_right < 0 || j <= i + window_right),
+ * with i and j counted from the start of their own sample.
+ *
+ * Layouts (all tensors are DEVICE pointers, row-major, no padding):
+ *   q, o, dout, dq        bf16 [total_q ][H][D]
+ *   k, v, dk, dv          bf16 [total_kv][H][D]
+ *   bias (or gate G), dbias  fp32 [H][total_kv]   (broadcast over queries)
+ *   lse                   fp32 [H][total_q]       natural-log log-sum-exp
+ *   q_offsets, kv_offsets int32 [B+1], offsets[0] = 0, non-decreasing,
+ *                         offsets[B] = total.  Sample b owns rows
+ *                         [offsets[b], offsets[b+1]).
+ * q, k, v, o, dout, dq, dk, dv and the workspace must be 16-byte aligned.
+ * D must be 32, 64 or 128.  B <= 16384.
+ *
+ * Ownership: the caller allocates and frees everything (inputs, outputs and
+ * the workspace).  The library never allocates, frees or synchronises,
+ * except gdpa_get_device_status, which synchronises the stream it is given.
+ * All launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream).  Calls that share one workspace must not overlap.
+ *
+ * Errors: argument errors are reported at the call (GDPA_ERR_*), before
+ * anything is launched.  Launch failures return GDPA_ERR_CUDA.  Errors found
+ * by the device (a bounded wait that ran out, an offset beyond the declared
+ * maximum length) are recorded in the workspace and read back with
+ * gdpa_get_device_status.  Offsets contents are trusted beyond those checks.
+ */
+#ifndef GDPA_H_
+#define GDPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDPA_API __attribute__((visibility("default")))
+#else
+#define GDPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gdpa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  GDPA_OK = 0,
+  GDPA_ERR_INVALID_ARG = 1,  /* null/unaligned pointer, bad size or offset shape */
+  GDPA_ERR_UNSUPPORTED = 2,  /* D, phi, bias kind, batch size or device not supported */
+  GDPA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdpa_workspace_size */
+  GDPA_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed */
+  GDPA_ERR_TIMEOUT = 5,      /* device: a bounded wait inside a kernel ran out */
+  GDPA_ERR_DEVICE_CHECK = 6  /* device: a sample is longer than max_seqlen_q / _kv */
+} gdpa_status_t;
+
+enum { GDPA_PHI_SILU = 0, GDPA_PHI_SOFTMAX = 1, GDPA_PHI_IDENTITY = 2 };
+enum { GDPA_BIAS_NONE = 0, GDPA_BIAS_ADD = 1, GDPA_BIAS_GATE = 2 };
+
+typedef struct {
+  int B;              /* samples */
+  int H;              /* heads */
+  int D;              /* head dim: 32, 64 or 128 */
+  int64_t total_q;    /* q_offsets[B]  (host-known: sizes the TMA descriptors) */
+  int64_t total_kv;   /* kv_offsets[B] */
+  int max_seqlen_q;   /* upper bound on any sample's query length; 0 = total_q */
+  int max_seqlen_kv;  /* upper bound on any sample's key length;   0 = total_kv */
+  int phi;            /* GDPA_PHI_* : SiLU x*sigmoid(x), row softmax, or identity */
+  float scale;        /* multiplies QK^T before beta is added (= 1/tau) */
+  int window_left;    /* -1 = unbounded */
+  int window_right;   /* -1 = unbounded */
+  int bias_kind;      /* GDPA_BIAS_*: none, beta = bias, or beta = log sigmoid(bias) */
+  int debug_flags;    /* 0 in normal use; bit 0 drops one producer arrival so that
+                         the bounded-wait path can be tested (returns TIMEOUT) */
+  int wait_timeout_us;/* bound on any single in-kernel wait; 0 = 2000000 (2 s) */
+} gdpa_params_t;
+
+/* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward
+ * (backward = 1) needs for these parameters.  0 on invalid parameters. */
+GDPA_API size_t gdpa_workspace_size(const gdpa_params_t* p, int backward);
+
+/* Forward: o (and lse when phi = softmax; lse may be NULL otherwise or when not
+ * wanted) from q, k, v.  bias must be non-NULL iff bias_kind != NONE.
+ * Rows with no visible key get O = 0 and LSE = -inf.
+ * Defined by: Kunlun paper review §2.3 (GDPA, Fig. 2) and §2.5 (window);
+ * Kunlun reproduction notes, "Core equations" (softmax with log-sigmoid gate). */
+GDPA_API gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
+                           const void* v, const int32_t* q_offsets,
+                           const int32_t* kv_offsets, const float* bias, void* o,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           gdpa_stream_t stream);
+
+/* Backward: dq, dk, dv (bf16) from the forward's inputs, its output o, the
+ * upstream gradient dout, and lse (softmax only; o and lse are unused for the
+ * element-wise activations and may be NULL there).  Every row of dq, dk, dv is
+ * written (zeros where nothing flows).  dbias must be NULL (the bias/gate
+ * gradient is not produced).  The gradient of the definition above:
+ *   dV_j = sum_i p_ij dO_i,  dP_ij = dO_i . V_j,
+ *   dS_ij = p_ij (dP_ij - dO_i . O_i) (softmax)  or  dP_ij * phi'(s_ij),
+ *   dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i.
+ * The pages ask that the fused backward avoid materialising large
+ * intermediates (Kunlun paper review §2.3, Fig. 2 discussion). */
+GDPA_API gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k,
+                            const void* v, const void* o, const void* dout,
+                            const float* lse, const int32_t* q_offsets,
+                            const int32_t* kv_offsets, const float* bias, void* dq,
+                            void* dk, void* dv, float* dbias, void* workspace,
+                            size_t workspace_bytes, gdpa_stream_t stream);
+
+/* The jagged tile schedule the kernels use, exported so it can be checked:
+ * query tiles of block_m rows, key blocks of block_n keys (both multiples of
+ * 16 in [16, 256]); per sample the cost sum over its tiles of (1 + key blocks
+ * the tile may touch under the window); order = samples by descending cost,
+ * ties by ascending index; tile_start[p] = query tiles of order[0..p),
+ * tile_start[B] = all tiles.  Outputs are device int32 arrays of B+1 and B.
+ * ("tile scheduling" over "jagged sequences": Kunlun paper review §2.3.)
+ * Costs are clamped to 2^32-1. */
+GDPA_API gdpa_status_t gdpa_tile_schedule(const gdpa_params_t* p, int block_m, int block_n,
+                                 const int32_t* q_offsets, const int32_t* kv_offsets,
+                                 int32_t* tile_start, int32_t* order,
+                                 gdpa_stream_t stream);
+
+/* Tile shape (block_m, block_n) the forward kernel uses for these parameters. */
+GDPA_API gdpa_status_t gdpa_forward_tile_shape(const gdpa_params_t* p, int* block_m,
+                                      int* block_n);
+
+/* Synchronises `stream`, then returns the status the last gdpa_forward /
+ * gdpa_backward call on this workspace recorded on the device (GDPA_OK,
+ * GDPA_ERR_TIMEOUT or GDPA_ERR_DEVICE_CHECK), or GDPA_ERR_CUDA. */
+GDPA_API gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream);
+
+/* Static English text for a status code. */
+GDPA_API const char* gdpa_status_string(gdpa_status_t s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDPA_API int gdpa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDPA_H_ */

@@ -1,0 +1,266 @@
+// gdpa_api.cu -- the C ABI (include/gdpa.h): argument checks, workspace layout,
+// TMA descriptor encoding, and the launch sequence.  No allocation, no sync
+// (except gdpa_get_device_status).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "gdpa.h"
+#include "gdpa_internal.h"
+
+using namespace gdpa;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Number of SMs of the current device, and whether it is an sm_100 part.
+bool device_info(int* sms) {
+  static int cache[kMaxDevices];
+  static int major_cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (cache[dev] == 0) {
+    int n = 0, major = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return false;
+    major_cache[dev] = major;
+    cache[dev] = n;
+  }
+  *sms = cache[dev];
+  return major_cache[dev] == 10;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdpa_status_t check_params(const gdpa_params_t* p) {
+  if (!p) return GDPA_ERR_INVALID_ARG;
+  if (p->B < 0 || p->H <= 0 || p->total_q < 0 || p->total_kv < 0) return GDPA_ERR_INVALID_ARG;
+  if (p->total_q >= (int64_t(1) << 31) || p->total_kv >= (int64_t(1) << 31))
+    return GDPA_ERR_INVALID_ARG;
+  if (p->max_seqlen_q < 0 || p->max_seqlen_kv < 0) return GDPA_ERR_INVALID_ARG;
+  if (p->window_left < -1 || p->window_right < -1) return GDPA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return GDPA_ERR_INVALID_ARG;
+  if (p->wait_timeout_us < 0) return GDPA_ERR_INVALID_ARG;
+  if (p->D != 32 && p->D != 64 && p->D != 128) return GDPA_ERR_UNSUPPORTED;
+  if (p->phi < 0 || p->phi > 2) return GDPA_ERR_UNSUPPORTED;
+  if (p->bias_kind < 0 || p->bias_kind > 2) return GDPA_ERR_UNSUPPORTED;
+  if (p->B > kMaxSortBatch) return GDPA_ERR_UNSUPPORTED;
+  if ((int64_t)p->H * p->B >= (int64_t(1) << 31)) return GDPA_ERR_UNSUPPORTED;
+  return GDPA_OK;
+}
+
+int eff_max_q(const gdpa_params_t* p) {
+  return p->max_seqlen_q > 0 ? p->max_seqlen_q : (int)p->total_q;
+}
+int eff_max_kv(const gdpa_params_t* p) {
+  return p->max_seqlen_kv > 0 ? p->max_seqlen_kv : (int)p->total_kv;
+}
+
+int backward_grid(const gdpa_params_t* p, int sms) {
+  const int64_t units = (int64_t)p->B * p->H;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(units, sms));
+}
+
+WorkspaceLayout make_layout(const gdpa_params_t* p, int backward, int sms) {
+  WorkspaceLayout L{};
+  size_t off = sizeof(DeviceStatus);
+  L.order = off;
+  off += align256((size_t)std::max(p->B, 1) * 4);
+  L.tile_start = off;
+  off += align256((size_t)(p->B + 1) * 4);
+  if (backward) {
+    L.delta = off;
+    if (p->phi == GDPA_PHI_SOFTMAX) off += align256((size_t)p->H * (size_t)p->total_q * 4);
+    L.grid = backward_grid(p, sms);
+    L.dq_slot_rows = (std::min(eff_max_q(p), (int)p->total_q) + kBlockM - 1) / kBlockM * kBlockM;
+    L.dq_scratch = off;
+    off += align256((size_t)L.grid * (size_t)L.dq_slot_rows * (size_t)p->D * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+// [rows][H][D] bf16 tensor, boxes of box_rows rows x one head x panel columns.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H, int D, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const int panel = D >= 64 ? 64 : 32;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)panel, 1u, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw =
+      panel == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+uint64_t timeout_ns(const gdpa_params_t* p) {
+  const int us = p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000;
+  return (uint64_t)us * 1000ull;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdpa_version(void) { return 100; }
+
+const char* gdpa_status_string(gdpa_status_t s) {
+  switch (s) {
+    case GDPA_OK: return "ok";
+    case GDPA_ERR_INVALID_ARG: return "invalid argument";
+    case GDPA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case GDPA_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDPA_ERR_CUDA: return "CUDA error";
+    case GDPA_ERR_TIMEOUT: return "device wait timed out";
+    case GDPA_ERR_DEVICE_CHECK: return "sample longer than the declared maximum length";
+  }
+  return "unknown status";
+}
+
+size_t gdpa_workspace_size(const gdpa_params_t* p, int backward) {
+  if (check_params(p) != GDPA_OK) return 0;
+  int sms = 0;
+  if (!device_info(&sms)) sms = 148;
+  return make_layout(p, backward, sms).total;
+}
+
+gdpa_status_t gdpa_forward_tile_shape(const gdpa_params_t* p, int* block_m, int* block_n) {
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  if (!block_m || !block_n) return GDPA_ERR_INVALID_ARG;
+  *block_m = kBlockM;
+  *block_n = forward_block_n(p->D, p->phi, eff_max_kv(p));
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_tile_schedule(const gdpa_params_t* p, int block_m, int block_n,
+                                 const int32_t* q_offsets, const int32_t* kv_offsets,
+                                 int32_t* tile_start, int32_t* order, gdpa_stream_t stream) {
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  if (!q_offsets || !kv_offsets || !tile_start || (!order && p->B > 0)) return GDPA_ERR_INVALID_ARG;
+  if (block_m < 16 || block_m > 256 || block_m % 16 || block_n < 16 || block_n > 256 ||
+      block_n % 16)
+    return GDPA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, block_m, block_n, p->window_left,
+                                  p->window_right, tile_start, order, nullptr,
+                                  (cudaStream_t)stream);
+  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}
+
+gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k, const void* v,
+                           const int32_t* q_offsets, const int32_t* kv_offsets,
+                           const float* bias, void* o, float* lse, void* workspace,
+                           size_t workspace_bytes, gdpa_stream_t stream) {
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
+  if (p->total_q > 0 && (!q || !o)) return GDPA_ERR_INVALID_ARG;
+  if (p->total_kv > 0 && (!k || !v)) return GDPA_ERR_INVALID_ARG;
+  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(workspace))
+    return GDPA_ERR_INVALID_ARG;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  const WorkspaceLayout L = make_layout(p, 0, sms);
+  if (!workspace || workspace_bytes < L.total) return GDPA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(ws + L.tile_start);
+  const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p));
+  cudaStream_t s = (cudaStream_t)stream;
+
+  cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, block_n,
+                                  p->window_left, p->window_right, tile_start, order, status, s);
+  if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  if (p->B == 0 || p->total_q == 0) return GDPA_OK;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+  if (p->total_kv > 0) {
+    if (!make_map(&tk, k, p->total_kv, p->H, p->D, block_n)) return GDPA_ERR_CUDA;
+    if (!make_map(&tv, v, p->total_kv, p->H, p->D, block_n)) return GDPA_ERR_CUDA;
+  } else {
+    tk = tq;  // never dereferenced: no sample has a key
+    tv = tq;
+  }
+  FwdArgs a{};
+  a.q_offsets = q_offsets;
+  a.kv_offsets = kv_offsets;
+  a.order = order;
+  a.bias = bias;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = p->phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
+  a.status = status;
+  a.total_q = p->total_q;
+  a.total_kv = p->total_kv;
+  a.B = p->B;
+  a.H = p->H;
+  a.n_units = p->B * p->H;
+  a.max_q = eff_max_q(p);
+  a.max_kv = eff_max_kv(p);
+  a.scale = p->scale;
+  a.phi = p->phi;
+  a.bias_kind = p->bias_kind;
+  a.wl = p->window_left;
+  a.wr = p->window_right;
+  a.debug_flags = p->debug_flags;
+  a.timeout_ns = timeout_ns(p);
+  const int grid = std::max(1, std::min(a.n_units, sms));
+  e = launch_forward(a, p->D, block_n, tq, tk, tv, grid, s);
+  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}
+
+gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k, const void* v,
+                            const void* o, const void* dout, const float* lse,
+                            const int32_t* q_offsets, const int32_t* kv_offsets,
+                            const float* bias, void* dq, void* dk, void* dv, float* dbias,
+                            void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
+  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)q_offsets;
+  (void)kv_offsets; (void)bias; (void)dq; (void)dk; (void)dv; (void)dbias; (void)workspace;
+  (void)workspace_bytes; (void)stream;
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  return GDPA_ERR_UNSUPPORTED;
+}
+
+gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {
+  if (!workspace || !aligned16(workspace)) return GDPA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDPA_ERR_CUDA;
+  DeviceStatus st;
+  if (cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDPA_ERR_CUDA;
+  return (gdpa_status_t)st.code;
+}
+
+}  // extern "C"

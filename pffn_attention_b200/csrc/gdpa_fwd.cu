@@ -1,0 +1,621 @@
+// gdpa_fwd.cu -- fused GDPA forward for sm_100a.
+//
+// Computes, per sample b and head h, O = phi(scale * Q K^T + beta) V with S and
+// phi(S) kept on chip (Kunlun paper review §2.3 "GDPA", Fig. 2: QK^T / tau, then
+// the activation, then Attn x V, fused block-wise; Kunlun Breakdown, "The Core
+// Architecture and Mechanics": one FlashAttention-style kernel).  phi is SiLU or
+// identity (element-wise) or a row softmax with running max and sum (Kunlun
+// reproduction notes, "Core equations": softmax(QK^T/sqrt(d) + log sigma(G))).
+//
+// One persistent CTA per SM walks (sample, head) units in longest-first order.
+// For each 128-row query tile of the unit it walks the key blocks the tile can
+// see (all of them, or the band of the sliding window, Kunlun paper review
+// §2.5), so padding rows and invisible key blocks are never loaded.
+//
+// Warp roles (256 threads):
+//   warp 0     TMA producer: Q tile (2 buffers), K and V blocks (ring of stages)
+//   warp 1     MMA issuer (one thread): S = Q K^T into TMEM (2 buffers),
+//              O += P V into TMEM
+//   warp 2     TMEM allocator
+//   warp 3     bias warp: beta for each key block (log sigma(G) for the gate)
+//   warps 4-7  phi / epilogue warpgroup: one thread per query row; reads S
+//              from TMEM, applies the mask and phi, writes P (bf16) to shared
+//              memory for the PV MMA, rescales O when the running max moves,
+//              and writes O (bf16) and LSE at the end of the tile.
+// Every wait is bounded; on expiry the kernel records GDPA_ERR_TIMEOUT in the
+// workspace status, all roles leave their loops, TMEM is freed and the kernel
+// returns.
+#include <cfloat>
+#include <climits>
+
+#include "gdpa_internal.h"
+
+namespace gdpa {
+namespace {
+
+template <int D_, int BN_>
+struct FwdCfg {
+  static constexpr int D = D_;
+  static constexpr int BN = BN_;
+  static constexpr int BM = kBlockM;
+  // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
+  // (64 B, 64-byte swizzle) when D = 32.  P panels are always 64 keys wide.
+  static constexpr int PANEL_ELEMS = D >= 64 ? 64 : 32;
+  static constexpr int PANEL_BYTES = PANEL_ELEMS * 2;
+  static constexpr int NPANEL = D / PANEL_ELEMS;
+  static constexpr uint32_t LAYOUT = D >= 64 ? LAYOUT_SW128 : LAYOUT_SW64;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int NQ = 2;
+  static constexpr int NKV = (D == 128 && BN == 128) ? 2 : 3;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NKV * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NKV * KV_BYTES;
+  static constexpr int OFF_BIAS = OFF_P + P_BYTES;          // float [2][BN]
+  static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;     // uint64 barriers
+  // barrier indices
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_QEMPTY = B_QFULL + NQ;
+  static constexpr int B_KVFULL = B_QEMPTY + NQ;
+  static constexpr int B_KVEMPTY = B_KVFULL + NKV;
+  static constexpr int B_SFULL = B_KVEMPTY + NKV;
+  static constexpr int B_SEMPTY = B_SFULL + 2;
+  static constexpr int B_PFULL = B_SEMPTY + 2;
+  static constexpr int B_PVDONE = B_PFULL + 1;
+  static constexpr int B_OFULL = B_PVDONE + 1;
+  static constexpr int B_OEMPTY = B_OFULL + 1;
+  static constexpr int B_BFULL = B_OEMPTY + 1;   // 2 bias buffers
+  static constexpr int B_BEMPTY = B_BFULL + 2;
+  static constexpr int NBARS = B_BEMPTY + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;      // tmem addr, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // + alignment slack
+  // TMEM: S buffers at columns [0, BN) and [BN, 2BN); O at [2BN, 2BN + D).
+  static constexpr int TMEM_S0 = 0;
+  static constexpr int TMEM_O = 2 * BN;
+  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0 && P_BYTES % 1024 == 0, "align");
+};
+
+constexpr int kThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
+
+struct Unit {
+  int b, h;
+  int q0, Lq, k0, Lk;
+};
+
+__device__ __forceinline__ int unit_index(int round, int cta, int grid) {
+  // boustrophedon over the longest-first list: even rounds left to right,
+  // odd rounds right to left
+  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ Unit load_unit(const FwdArgs& a, int u) {
+  Unit t;
+  const int p = u / a.H;
+  t.h = u - p * a.H;
+  t.b = a.order[p];
+  t.q0 = a.q_offsets[t.b];
+  t.Lq = a.q_offsets[t.b + 1] - t.q0;
+  t.k0 = a.kv_offsets[t.b];
+  t.Lk = a.kv_offsets[t.b + 1] - t.k0;
+  if (t.Lq > a.max_q || t.Lk > a.max_kv) {  // the declared bound is violated: skip
+    t.Lq = 0;
+    t.Lk = 0;
+  }
+  return t;
+}
+
+// Key-block range [kb0, kb1) a tile starting at local row m0 may touch.
+template <int BN>
+__device__ __forceinline__ void kv_range(int m0, int Lk, int wl, int wr, int& kb0, int& kb1) {
+  int lo = wl >= 0 ? max(0, m0 - wl) : 0;
+  int hi = wr >= 0 ? min(Lk, m0 + kBlockM + wr) : Lk;
+  if (hi <= lo) {
+    kb0 = kb1 = 0;
+  } else {
+    kb0 = lo / BN;
+    kb1 = (hi + BN - 1) / BN;
+  }
+}
+
+template <class C>
+struct Smem {
+  uint32_t base;  // shared address of the 1024-aligned base
+  uint8_t* ptr;
+  __device__ uint32_t q(int s) const { return base + C::OFF_Q + s * C::Q_BYTES; }
+  __device__ uint32_t k(int s) const { return base + C::OFF_K + s * C::KV_BYTES; }
+  __device__ uint32_t v(int s) const { return base + C::OFF_V + s * C::KV_BYTES; }
+  __device__ uint32_t p() const { return base + C::OFF_P; }
+  __device__ float* bias(int s) const {
+    return reinterpret_cast<float*>(ptr + C::OFF_BIAS) + s * C::BN;
+  }
+  __device__ uint32_t bar(int i) const { return base + C::OFF_BAR + i * 8; }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(ptr + C::OFF_MISC); }
+  __device__ volatile int* abort_flag() const {
+    return reinterpret_cast<volatile int*>(ptr + C::OFF_MISC + 4);
+  }
+};
+
+// ------------------------------------------------------------------ producer
+template <class C>
+__device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtensorMap* tq,
+                              const CUtensorMap* tk, const CUtensorMap* tv) {
+  volatile int* abort = sm.abort_flag();
+  const uint64_t pol_stream = l2_policy_evict_first();
+  const uint64_t pol_keep = l2_policy_evict_last();
+  uint32_t qi = 0, kvi = 0;
+  bool dropped = false;
+  for (int round = 0;; ++round) {
+    const int u = unit_index(round, blockIdx.x, gridDim.x);
+    if (u >= a.n_units) break;
+    const Unit t = load_unit(a, u);
+    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    for (int mt = 0; mt < ntile; ++mt) {
+      const int m0 = mt * kBlockM;
+      int kb0, kb1;
+      kv_range<C::BN>(m0, t.Lk, a.wl, a.wr, kb0, kb1);
+      if (kb1 <= kb0) continue;
+      const int qs = qi % C::NQ;
+      if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((qi / C::NQ) & 1) ^ 1, abort, a.status,
+                     a.timeout_ns, 0x000 + C::B_QEMPTY + qs))
+        return;
+      if ((a.debug_flags & 1) && !dropped && blockIdx.x == 0) {
+        dropped = true;  // test hook: this Q tile is never loaded
+      } else {
+        mbar_arrive_expect_tx(sm.bar(C::B_QFULL + qs), C::Q_BYTES);
+        for (int pnl = 0; pnl < C::NPANEL; ++pnl)
+          tma_load_3d(sm.q(qs) + pnl * kBlockM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + qs),
+                      pnl * C::PANEL_ELEMS, t.h, t.q0 + m0, pol_stream);
+      }
+      ++qi;
+      for (int j = kb0; j < kb1; ++j) {
+        const int ks = kvi % C::NKV;
+        if (!mbar_wait(sm.bar(C::B_KVEMPTY + ks), ((kvi / C::NKV) & 1) ^ 1, abort, a.status,
+                       a.timeout_ns, 0x000 + C::B_KVEMPTY + ks))
+          return;
+        mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + ks), 2 * C::KV_BYTES);
+        for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
+          tma_load_3d(sm.k(ks) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + ks),
+                      pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
+          tma_load_3d(sm.v(ks) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + ks),
+                      pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
+        }
+        ++kvi;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <class C>
+__device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
+  volatile int* abort = sm.abort_flag();
+  constexpr uint32_t idesc_s = make_idesc_bf16(kBlockM, C::BN, 0, 0);
+  constexpr uint32_t idesc_o = make_idesc_bf16(kBlockM, C::D, 0, 1);
+  constexpr uint32_t SBO_QK = 8 * C::PANEL_BYTES;
+  uint32_t qi = 0, kvi = 0, si = 0, pvi = 0, ti = 0;
+
+  auto issue_pv = [&](int idx, uint32_t kv_index) -> bool {
+    const int ks = kv_index % C::NKV;
+    if (!mbar_wait(sm.bar(C::B_PFULL), pvi & 1, abort, a.status, a.timeout_ns,
+                   0x100 + C::B_PFULL))
+      return false;
+    if (idx == 0 && !mbar_wait(sm.bar(C::B_OEMPTY), (ti & 1) ^ 1, abort, a.status, a.timeout_ns,
+                               0x100 + C::B_OEMPTY))
+      return false;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+      // A = P [128 x BN] K-major, 64-key panels with 128-byte swizzle
+      const uint32_t pa = sm.p() + (kk * 16 / 64) * (kBlockM * 128) + (kk * 16 % 64) * 2;
+      const uint64_t adesc = make_smem_desc(pa, 16, 1024, LAYOUT_SW128);
+      // B = V [BN keys x D], N (= D) contiguous: MN-major; 16 keys per step
+      const uint32_t vb = sm.v(ks) + kk * 16 * C::PANEL_BYTES;
+      const uint64_t bdesc = make_smem_desc(vb, C::BN * C::PANEL_BYTES, SBO_QK, C::LAYOUT);
+      mma_bf16_ss(tmem + C::TMEM_O, adesc, bdesc, idesc_o, (idx > 0 || kk > 0) ? 1u : 0u);
+    }
+    mma_commit(sm.bar(C::B_KVEMPTY + ks));
+    mma_commit(sm.bar(C::B_PVDONE));
+    ++pvi;
+    return true;
+  };
+
+  for (int round = 0;; ++round) {
+    const int u = unit_index(round, blockIdx.x, gridDim.x);
+    if (u >= a.n_units) break;
+    const Unit t = load_unit(a, u);
+    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    for (int mt = 0; mt < ntile; ++mt) {
+      int kb0, kb1;
+      kv_range<C::BN>(mt * kBlockM, t.Lk, a.wl, a.wr, kb0, kb1);
+      const int nkv = kb1 - kb0;
+      if (nkv <= 0) continue;
+      const int qs = qi % C::NQ;
+      if (!mbar_wait(sm.bar(C::B_QFULL + qs), (qi / C::NQ) & 1, abort, a.status, a.timeout_ns,
+                     0x100 + C::B_QFULL + qs))
+        return;
+      const uint32_t first_kvi = kvi;
+      for (int idx = 0; idx < nkv; ++idx) {
+        const int ks = kvi % C::NKV;
+        if (!mbar_wait(sm.bar(C::B_KVFULL + ks), (kvi / C::NKV) & 1, abort, a.status,
+                       a.timeout_ns, 0x100 + C::B_KVFULL + ks))
+          return;
+        const int sb = si & 1;
+        if (!mbar_wait(sm.bar(C::B_SEMPTY + sb), ((si >> 1) & 1) ^ 1, abort, a.status,
+                       a.timeout_ns, 0x100 + C::B_SEMPTY + sb))
+          return;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::D / 16; ++kk) {
+          const int pnl = kk * 16 / C::PANEL_ELEMS;
+          const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
+          const uint64_t adesc = make_smem_desc(
+              sm.q(qs) + pnl * kBlockM * C::PANEL_BYTES + within, 16, SBO_QK, C::LAYOUT);
+          const uint64_t bdesc = make_smem_desc(
+              sm.k(ks) + pnl * C::BN * C::PANEL_BYTES + within, 16, SBO_QK, C::LAYOUT);
+          mma_bf16_ss(tmem + C::TMEM_S0 + sb * C::BN, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(sm.bar(C::B_SFULL + sb));
+        ++si;
+        if (idx == nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + qs));
+        ++kvi;
+        if (idx > 0 && !issue_pv(idx - 1, first_kvi + idx - 1)) return;
+      }
+      if (!issue_pv(nkv - 1, first_kvi + nkv - 1)) return;
+      mma_commit(sm.bar(C::B_OFULL));
+      ++qi;
+      ++ti;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ bias warp
+template <class C>
+__device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
+  volatile int* abort = sm.abort_flag();
+  const int lane = threadIdx.x & 31;
+  uint32_t bi = 0;
+  for (int round = 0;; ++round) {
+    const int u = unit_index(round, blockIdx.x, gridDim.x);
+    if (u >= a.n_units) break;
+    const Unit t = load_unit(a, u);
+    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    for (int mt = 0; mt < ntile; ++mt) {
+      int kb0, kb1;
+      kv_range<C::BN>(mt * kBlockM, t.Lk, a.wl, a.wr, kb0, kb1);
+      for (int j = kb0; j < kb1; ++j) {
+        const int bs = bi & 1;
+        bool ok = mbar_wait(sm.bar(C::B_BEMPTY + bs), ((bi >> 1) & 1) ^ 1, abort, a.status,
+                            a.timeout_ns, 0x300 + C::B_BEMPTY + bs);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        float* dst = sm.bias(bs);
+        const float* src = a.bias + (int64_t)t.h * a.total_kv + t.k0;
+        for (int c = lane; c < C::BN; c += 32) {
+          const int key = j * C::BN + c;
+          float beta = 0.f;
+          if (key < t.Lk) {
+            const float g = src[key];
+            if (a.bias_kind == 2) {
+              // log sigma(g) = min(g, 0) - log(1 + exp(-|g|))
+              beta = fminf(g, 0.f) - log1pf(__expf(-fabsf(g)));
+            } else {
+              beta = g;
+            }
+          }
+          dst[c] = softmax ? beta * kLog2e : beta;
+        }
+        mbar_arrive(sm.bar(C::B_BFULL + bs));  // one arrival per lane, after its writes
+        ++bi;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ phi warpgroup
+template <class C, bool SOFTMAX>
+__device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
+  volatile int* abort = sm.abort_flag();
+  const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quarter of this warp
+  const int lane = threadIdx.x & 31;
+  const int r = wq * 32 + lane;             // row of the tile owned by this thread
+  const uint32_t tl = (uint32_t)(wq * 32) << 16;
+  const bool has_bias = a.bias_kind != 0;
+  const bool identity = a.phi == 2;
+  const float sc = SOFTMAX ? a.scale * kLog2e : a.scale;
+  uint32_t si = 0, pvi = 0, ti = 0, bi = 0;
+
+#define PHI_WAIT(bar_, par_, where_)                                                   \
+  do {                                                                               \
+    bool ok_ = mbar_wait(sm.bar(bar_), (par_), abort, a.status, a.timeout_ns, where_); \
+    if (!__all_sync(0xffffffffu, ok_)) return;                                       \
+  } while (0)
+
+  for (int round = 0;; ++round) {
+    const int u = unit_index(round, blockIdx.x, gridDim.x);
+    if (u >= a.n_units) break;
+    const Unit t = load_unit(a, u);
+    if (r == 0 && t.Lq == 0) {
+      // distinguish a violated bound from an empty sample
+      const int Lq = a.q_offsets[t.b + 1] - a.q_offsets[t.b];
+      const int Lk = a.kv_offsets[t.b + 1] - a.kv_offsets[t.b];
+      if (Lq > a.max_q || Lk > a.max_kv) record_error(a.status, 6, t.b);
+    }
+    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    for (int mt = 0; mt < ntile; ++mt) {
+      const int m0 = mt * kBlockM;
+      const int row = m0 + r;
+      const bool row_ok = row < t.Lq;
+      __nv_bfloat16* orow = a.o + ((int64_t)(t.q0 + row) * a.H + t.h) * C::D;
+      int kb0, kb1;
+      kv_range<C::BN>(m0, t.Lk, a.wl, a.wr, kb0, kb1);
+      const int nkv = kb1 - kb0;
+      if (nkv <= 0) {
+        if (row_ok) {
+          uint4 z = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+          if (SOFTMAX && a.lse) a.lse[(int64_t)t.h * a.total_q + t.q0 + row] = -INFINITY;
+        }
+        continue;
+      }
+      // visible keys of this row: [lo, hi]
+      const int lo = a.wl >= 0 ? row - a.wl : INT_MIN;
+      const int hi = min(t.Lk - 1, a.wr >= 0 ? row + a.wr : INT_MAX);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int idx = 0; idx < nkv; ++idx) {
+        const int kbase = (kb0 + idx) * C::BN;
+        const int bs = bi & 1;
+        if (has_bias) PHI_WAIT(C::B_BFULL + bs, (bi >> 1) & 1, 0x400 + C::B_BFULL + bs);
+        const int sb = si & 1;
+        PHI_WAIT(C::B_SFULL + sb, (si >> 1) & 1, 0x400 + C::B_SFULL + sb);
+        tc_fence_after();
+        float s[C::BN];
+#pragma unroll
+        for (int c = 0; c < C::BN / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(tmem + tl + C::TMEM_S0 + sb * C::BN + c * 32, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+        }
+        tc_fence_before();
+        mbar_arrive(sm.bar(C::B_SEMPTY + sb));
+        ++si;
+        const float* bias_s = sm.bias(bs);
+        // scores, mask
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c) {
+          const int key = kbase + c;
+          float x = s[c] * sc;
+          if (has_bias) x += bias_s[c];
+          const bool vis = key >= lo && key <= hi;
+          if (SOFTMAX) {
+            s[c] = vis ? x : -INFINITY;
+          } else {
+            float p;
+            if (identity) {
+              p = x;
+            } else {
+              const float hx = 0.5f * x;
+              p = fmaf(hx, tanh_approx(hx), hx);  // x * sigmoid(x)
+            }
+            s[c] = vis ? p : 0.f;
+          }
+        }
+        if (has_bias) {
+          tc_fence_before();
+          mbar_arrive(sm.bar(C::B_BEMPTY + bs));
+          ++bi;
+        }
+        bool need_rescale = false;
+        float factor = 1.f;
+        if (SOFTMAX) {
+          float bm = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < C::BN; ++c) bm = fmaxf(bm, s[c]);
+          if (idx == 0) {
+            m_run = bm;
+          } else if (bm > m_run + kRescaleThreshold) {
+            factor = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - bm);
+            need_rescale = true;
+            l_run *= factor;
+            m_run = bm;
+          }
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          float lsum = 0.f;
+#pragma unroll
+          for (int c = 0; c < C::BN; ++c) {
+            const float p = ex2_approx(s[c] - m_use);
+            s[c] = p;
+            lsum += p;
+          }
+          l_run += lsum;
+        }
+        // the previous PV must be done before P is overwritten or O rescaled
+        if (idx > 0) PHI_WAIT(C::B_PVDONE, (pvi - 1) & 1, 0x400 + C::B_PVDONE);
+        if (SOFTMAX && __any_sync(0xffffffffu, need_rescale)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < C::D / 32; ++c) {
+            uint32_t raw[32];
+            tmem_ld32(tmem + tl + C::TMEM_O + c * 32, raw);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              raw[e] = __float_as_uint(__uint_as_float(raw[e]) * factor);
+            tmem_st32(tmem + tl + C::TMEM_O + c * 32, raw);
+          }
+          tmem_wait_st();
+        }
+        // P row -> shared memory, 64-key panels, 128-byte swizzle (K-major A operand)
+#pragma unroll
+        for (int ch = 0; ch < C::BN / 8; ++ch) {
+          const int pnl = ch / 8, cir = ch % 8;
+          const uint32_t addr =
+              sm.p() + pnl * (kBlockM * 128) + r * 128 + ((cir ^ (r & 7)) << 4);
+          st_shared_v4(addr, pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]),
+                       pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]),
+                       pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]),
+                       pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sm.bar(C::B_PFULL));
+        ++pvi;
+      }
+      // epilogue: O row from TMEM
+      PHI_WAIT(C::B_OFULL, ti & 1, 0x400 + C::B_OFULL);
+      tc_fence_after();
+      float inv = 1.f;
+      if (SOFTMAX) inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(tmem + tl + C::TMEM_O + c * 32, raw);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(raw[e + 0]) * inv, __uint_as_float(raw[e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(raw[e + 2]) * inv, __uint_as_float(raw[e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(sm.bar(C::B_OEMPTY));
+      ++ti;
+      if (SOFTMAX && row_ok && a.lse) {
+        a.lse[(int64_t)t.h * a.total_q + t.q0 + row] =
+            l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+#undef PHI_WAIT
+}
+
+template <int D, int BN, bool SOFTMAX>
+__global__ void __launch_bounds__(kThreads, 1)
+    gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
+                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+  using C = FwdCfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<C> sm;
+  {
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t aligned = (raw + 1023u) & ~1023u;
+    sm.base = aligned;
+    sm.ptr = smem_raw + (aligned - raw);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(sm.bar(C::B_QFULL + i), 1);
+      mbar_init(sm.bar(C::B_QEMPTY + i), 1);
+    }
+    for (int i = 0; i < C::NKV; ++i) {
+      mbar_init(sm.bar(C::B_KVFULL + i), 1);
+      mbar_init(sm.bar(C::B_KVEMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(sm.bar(C::B_SFULL + i), 1);
+      mbar_init(sm.bar(C::B_SEMPTY + i), 128);
+      mbar_init(sm.bar(C::B_BFULL + i), 32);
+      mbar_init(sm.bar(C::B_BEMPTY + i), 128);
+    }
+    mbar_init(sm.bar(C::B_PFULL), 128);
+    mbar_init(sm.bar(C::B_PVDONE), 1);
+    mbar_init(sm.bar(C::B_OFULL), 1);
+    mbar_init(sm.bar(C::B_OEMPTY), 128);
+    *sm.abort_flag() = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(sm.tmem_slot()), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot();
+
+  if (warp == 0) {
+    if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
+  } else if (warp == 1) {
+    if (lane == 0) role_mma<C>(a, sm, tmem);
+  } else if (warp == 3) {
+    if (a.bias_kind != 0) role_bias<C>(a, sm, SOFTMAX);
+  } else if (warp >= 4) {
+    role_phi<C, SOFTMAX>(a, sm, tmem);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*sm.abort_flag()) {
+    // a role gave up: let copies and MMAs already in flight land before the
+    // shared memory and TMEM they target are released
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+    __syncthreads();
+  }
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, int BN, bool SOFTMAX>
+cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                       const CUtensorMap& tv, int grid, cudaStream_t stream) {
+  using C = FwdCfg<D, BN>;
+  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int forward_block_n(int D, int phi, int max_kv) {
+  (void)D;
+  (void)phi;
+  return max_kv <= 64 ? 64 : 128;
+}
+
+cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
+                           const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                           cudaStream_t stream) {
+  const bool sm = a.phi == 1;
+#define GDPA_FWD_CASE(D_, BN_)                                                  \
+  if (D == D_ && block_n == BN_)                                                \
+    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, grid, stream)           \
+              : launch_one<D_, BN_, false>(a, tq, tk, tv, grid, stream);
+  GDPA_FWD_CASE(32, 64)
+  GDPA_FWD_CASE(32, 128)
+  GDPA_FWD_CASE(64, 64)
+  GDPA_FWD_CASE(64, 128)
+  GDPA_FWD_CASE(128, 64)
+  GDPA_FWD_CASE(128, 128)
+#undef GDPA_FWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gdpa

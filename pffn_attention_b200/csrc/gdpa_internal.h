@@ -1,0 +1,87 @@
+// gdpa_internal.h -- argument blocks shared by the host launcher and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+namespace gdpa {
+
+constexpr int kBlockM = 128;        // query rows per tile (UMMA M)
+constexpr int kMaxSortBatch = 16384;  // batch limit of the single-CTA LPT sort
+
+// Workspace layout (all offsets 256-byte aligned):
+//   [0, 256)                  DeviceStatus
+//   [256, ...)                order[B]      int32   (LPT sample order)
+//   then                      tile_start[B+1] int32
+//   backward only, then       delta[H][total_q] fp32 (softmax rowsum(dO * O))
+//   backward only, then       dQ scratch: grid x slot_rows x D fp32
+struct WorkspaceLayout {
+  size_t order, tile_start, delta, dq_scratch, total;
+  int dq_slot_rows;
+  int grid;
+};
+
+struct FwdArgs {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  const int32_t* order;
+  const float* bias;        // [H][total_kv] or nullptr
+  __nv_bfloat16* o;         // [total_q][H][D]
+  float* lse;               // [H][total_q] or nullptr
+  DeviceStatus* status;
+  int64_t total_q, total_kv;
+  int B, H;
+  int n_units;              // B * H
+  int max_q, max_kv;
+  float scale;
+  int phi;
+  int bias_kind;
+  int wl, wr;
+  int debug_flags;
+  uint64_t timeout_ns;
+};
+
+struct BwdArgs {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  const int32_t* order;
+  const float* bias;        // [H][total_kv] or nullptr
+  const float* lse;         // [H][total_q] (softmax)
+  const float* delta;       // [H][total_q] (softmax)
+  __nv_bfloat16* dq;        // [total_q][H][D]
+  __nv_bfloat16* dk;        // [total_kv][H][D]
+  __nv_bfloat16* dv;        // [total_kv][H][D]
+  float* dq_scratch;        // grid x slot_rows x D
+  DeviceStatus* status;
+  int64_t total_q, total_kv;
+  int B, H;
+  int n_units;
+  int max_q, max_kv;
+  int dq_slot_rows;
+  float scale;
+  int phi;
+  int bias_kind;
+  int wl, wr;
+  int debug_flags;
+  uint64_t timeout_ns;
+};
+
+// Launchers (defined next to their kernels).
+cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
+                            int block_m, int block_n, int wl, int wr, int32_t* tile_start,
+                            int32_t* order, DeviceStatus* status, cudaStream_t stream);
+cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
+                           const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                           cudaStream_t stream);
+int forward_block_n(int D, int phi, int max_kv);
+cudaError_t launch_bwd_preprocess(const __nv_bfloat16* o, const __nv_bfloat16* dout,
+                                  float* delta, int64_t total_q, int H, int D,
+                                  cudaStream_t stream);
+cudaError_t launch_backward(const BwdArgs& a, int D, const CUtensorMap& tq,
+                            const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, int grid, cudaStream_t stream);
+
+}  // namespace gdpa

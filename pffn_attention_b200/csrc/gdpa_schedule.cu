@@ -1,0 +1,142 @@
+// gdpa_schedule.cu -- jagged tile schedule (longest-processing-time order).
+//
+// The GDPA kernel's "tile scheduling" over "jagged sequences" (Kunlun paper
+// review §2.3 "GDPA", last paragraph) is left undefined by the pages; this is
+// the schedule the kernels here use:
+//   ntile_b = ceil(Lq_b / BM); each tile m (first row m0 = m*BM) may see keys
+//   [max(0, m0 - wl), min(Lk_b, m0 + BM + wr)) rounded out to key blocks of BN;
+//   cost_b = sum over tiles of (1 + key blocks);
+//   order  = samples by descending cost, ties by ascending index;
+//   tile_start[p] = query tiles of order[0..p).
+// One CTA: costs into shared memory as 64-bit keys (inverted cost, index) so
+// an ascending bitonic sort yields the order with unique keys, then a block
+// scan of the tile counts.  The kernel also clears the workspace status.
+#include "gdpa_internal.h"
+
+namespace gdpa {
+namespace {
+
+constexpr int kSchedThreads = 1024;
+
+__device__ __forceinline__ unsigned long long sample_cost(int Lq, int Lk, int BM, int BN, int wl,
+                                                          int wr) {
+  const long long ntile = (Lq + BM - 1) / BM;
+  if (wl < 0 && wr < 0) {
+    const long long nkv = Lk > 0 ? (Lk + BN - 1) / BN : 0;
+    return (unsigned long long)(ntile * (1 + nkv));
+  }
+  unsigned long long cost = 0;
+  for (long long m = 0; m < ntile; ++m) {
+    const long long m0 = m * BM;
+    const long long lo = wl >= 0 ? (m0 - wl > 0 ? m0 - wl : 0) : 0;
+    long long hi = Lk;
+    if (wr >= 0 && m0 + BM + wr < hi) hi = m0 + BM + wr;
+    long long nb = 0;
+    if (hi > lo) nb = (hi + BN - 1) / BN - lo / BN;
+    cost += 1 + (unsigned long long)nb;
+  }
+  return cost;
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+    gdpa_schedule_kernel(const int32_t* __restrict__ q_offsets,
+                         const int32_t* __restrict__ kv_offsets, int B, int BM, int BN, int wl,
+                         int wr, int32_t* __restrict__ tile_start, int32_t* __restrict__ order,
+                         DeviceStatus* status) {
+  extern __shared__ unsigned long long keys[];
+  __shared__ long long warp_tot[kSchedThreads / 32];
+  const int tid = threadIdx.x;
+  if (status && tid == 0) {
+    status->code = 0;
+    status->where = 0;
+    status->count = 0;
+  }
+  int n = 1;
+  while (n < B) n <<= 1;
+  for (int i = tid; i < n; i += kSchedThreads) {
+    unsigned long long key = ~0ull;
+    if (i < B) {
+      const int Lq = q_offsets[i + 1] - q_offsets[i];
+      const int Lk = kv_offsets[i + 1] - kv_offsets[i];
+      unsigned long long c = sample_cost(Lq, Lk, BM, BN, wl, wr);
+      if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
+      key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < n; i += kSchedThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          const bool ascending = (i & k) == 0;
+          if ((x > y) == ascending) {
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // order, then an exclusive scan of the tile counts in that order
+  const int chunk = (B + kSchedThreads - 1) / kSchedThreads;
+  const int beg = min(B, tid * chunk), end = min(B, beg + chunk);
+  long long local = 0;
+  for (int p = beg; p < end; ++p) {
+    const int b = (int)(keys[p] & 0xFFFFFFFFull);
+    order[p] = b;
+    const int Lq = q_offsets[b + 1] - q_offsets[b];
+    local += (Lq + BM - 1) / BM;
+  }
+  // block-wide exclusive scan of `local`
+  const int lane = tid & 31, warp = tid >> 5;
+  long long incl = local;
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = warp_tot[lane];
+    long long wi = w;
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += v;
+    }
+    warp_tot[lane] = wi - w;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  long long run = warp_tot[warp] + incl - local;
+  for (int p = beg; p < end; ++p) {
+    tile_start[p] = (int32_t)run;
+    const int b = order[p];
+    const int Lq = q_offsets[b + 1] - q_offsets[b];
+    run += (Lq + BM - 1) / BM;
+  }
+  if (end == B && beg < end) tile_start[B] = (int32_t)run;
+  if (B == 0 && tid == 0) tile_start[0] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
+                            int block_m, int block_n, int wl, int wr, int32_t* tile_start,
+                            int32_t* order, DeviceStatus* status, cudaStream_t stream) {
+  int n = 1;
+  while (n < B) n <<= 1;
+  const size_t smem = (size_t)n * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(gdpa_schedule_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(kMaxSortBatch * sizeof(unsigned long long)));
+  if (e != cudaSuccess) return e;
+  gdpa_schedule_kernel<<<1, kSchedThreads, smem, stream>>>(q_offsets, kv_offsets, B, block_m,
+                                                           block_n, wl, wr, tile_start, order,
+                                                           status);
+  return cudaGetLastError();
+}
+
+}  // namespace gdpa

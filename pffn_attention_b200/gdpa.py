@@ -1,0 +1,208 @@
+"""ctypes binding of libgdpa (include/gdpa.h).
+
+The ``gdpa_*`` functions keep the C names and take raw integers (device
+pointers, sizes, a stream handle); they only marshal arguments.  ``forward``
+and ``backward`` are the torch-facing conveniences: they allocate outputs and
+the workspace with torch, pass pointers, and raise on a non-OK status.  Every
+step of the computation runs in the CUDA library; if ``libgdpa.so`` is
+missing, ``load`` raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdpa.so")
+
+GDPA_OK = 0
+STATUS_NAMES = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
+                3: "GDPA_ERR_WORKSPACE", 4: "GDPA_ERR_CUDA", 5: "GDPA_ERR_TIMEOUT",
+                6: "GDPA_ERR_DEVICE_CHECK"}
+PHI = {"silu": 0, "softmax": 1, "identity": 2}
+BIAS = {"none": 0, "add": 1, "gate": 2}
+
+EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",
+            "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
+            "gdpa_version")
+
+
+class gdpa_params_t(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int),
+                ("total_q", ctypes.c_int64), ("total_kv", ctypes.c_int64),
+                ("max_seqlen_q", ctypes.c_int), ("max_seqlen_kv", ctypes.c_int),
+                ("phi", ctypes.c_int), ("scale", ctypes.c_float),
+                ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+                ("bias_kind", ctypes.c_int), ("debug_flags", ctypes.c_int),
+                ("wait_timeout_us", ctypes.c_int)]
+
+
+class GdpaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libgdpa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libgdpa.so not built at {path}; run python -m pffn_attention_b200.build")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(gdpa_params_t)
+    vp, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p
+    lib.gdpa_workspace_size.argtypes = [P, ctypes.c_int]
+    lib.gdpa_workspace_size.restype = sz
+    lib.gdpa_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, st]
+    lib.gdpa_forward.restype = ctypes.c_int
+    lib.gdpa_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                  st]
+    lib.gdpa_backward.restype = ctypes.c_int
+    lib.gdpa_tile_schedule.argtypes = [P, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, st]
+    lib.gdpa_tile_schedule.restype = ctypes.c_int
+    lib.gdpa_forward_tile_shape.argtypes = [P, ctypes.POINTER(ctypes.c_int),
+                                            ctypes.POINTER(ctypes.c_int)]
+    lib.gdpa_forward_tile_shape.restype = ctypes.c_int
+    lib.gdpa_get_device_status.argtypes = [vp, st]
+    lib.gdpa_get_device_status.restype = ctypes.c_int
+    lib.gdpa_status_string.argtypes = [ctypes.c_int]
+    lib.gdpa_status_string.restype = ctypes.c_char_p
+    lib.gdpa_version.argtypes = []
+    lib.gdpa_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------------- raw C names
+def gdpa_workspace_size(p: gdpa_params_t, backward: int) -> int:
+    return int(load().gdpa_workspace_size(ctypes.byref(p), int(backward)))
+
+
+def gdpa_forward(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, workspace, workspace_bytes,
+                 stream) -> int:
+    return int(load().gdpa_forward(ctypes.byref(p), q, k, v, q_offsets, kv_offsets, bias, o, lse,
+                                   workspace, workspace_bytes, stream))
+
+
+def gdpa_backward(p, q, k, v, o, dout, lse, q_offsets, kv_offsets, bias, dq, dk, dv, dbias,
+                  workspace, workspace_bytes, stream) -> int:
+    return int(load().gdpa_backward(ctypes.byref(p), q, k, v, o, dout, lse, q_offsets, kv_offsets,
+                                    bias, dq, dk, dv, dbias, workspace, workspace_bytes, stream))
+
+
+def gdpa_tile_schedule(p, block_m, block_n, q_offsets, kv_offsets, tile_start, order,
+                       stream) -> int:
+    return int(load().gdpa_tile_schedule(ctypes.byref(p), block_m, block_n, q_offsets, kv_offsets,
+                                         tile_start, order, stream))
+
+
+def gdpa_forward_tile_shape(p):
+    bm, bn = ctypes.c_int(0), ctypes.c_int(0)
+    rc = int(load().gdpa_forward_tile_shape(ctypes.byref(p), ctypes.byref(bm), ctypes.byref(bn)))
+    return rc, bm.value, bn.value
+
+
+def gdpa_get_device_status(workspace, stream) -> int:
+    return int(load().gdpa_get_device_status(workspace, stream))
+
+
+def gdpa_status_string(s: int) -> str:
+    return load().gdpa_status_string(int(s)).decode()
+
+
+def gdpa_version() -> int:
+    return int(load().gdpa_version())
+
+
+# ----------------------------------------------------------------- torch helpers
+def make_params(B, H, D, total_q, total_kv, *, phi=0, scale=1.0, window=(-1, -1),
+                bias_kind=0, max_seqlen_q=0, max_seqlen_kv=0, debug_flags=0,
+                wait_timeout_us=0) -> gdpa_params_t:
+    if isinstance(phi, str):
+        phi = PHI[phi]
+    if isinstance(bias_kind, str):
+        bias_kind = BIAS[bias_kind]
+    return gdpa_params_t(int(B), int(H), int(D), int(total_q), int(total_kv), int(max_seqlen_q),
+                         int(max_seqlen_kv), int(phi), float(scale), int(window[0]),
+                         int(window[1]), int(bias_kind), int(debug_flags), int(wait_timeout_us))
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def workspace_for(p: gdpa_params_t, backward: bool, device):
+    import torch
+    n = gdpa_workspace_size(p, int(backward))
+    if n == 0:
+        raise GdpaError(1, "gdpa_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check(rc: int, where: str):
+    if rc != GDPA_OK:
+        raise GdpaError(rc, where)
+
+
+def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1, -1),
+            bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0, out=None, lse=None,
+            workspace=None, stream=None, params=None):
+    """O (and LSE for softmax) on the device.  Inputs are CUDA tensors:
+    q [total_q,H,D] bf16, k/v [total_kv,H,D] bf16, offsets int32 [B+1]."""
+    import torch
+    total_q, H, D = q.shape
+    total_kv = k.shape[0]
+    B = q_offsets.numel() - 1
+    p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
+                              bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
+                              max_seqlen_kv=max_seqlen_kv)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and p.phi == PHI["softmax"]:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = workspace_for(p, False, q.device)
+    rc = gdpa_forward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(q_offsets), _ptr(kv_offsets), _ptr(bias),
+                      _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "gdpa_forward")
+    return out, lse, workspace
+
+
+def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=1.0,
+             window=(-1, -1), bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0,
+             dq=None, dk=None, dv=None, workspace=None, stream=None, params=None):
+    """dQ, dK, dV on the device (bf16, shapes of q, k, v)."""
+    import torch
+    total_q, H, D = q.shape
+    total_kv = k.shape[0]
+    B = q_offsets.numel() - 1
+    p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
+                              bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
+                              max_seqlen_kv=max_seqlen_kv)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = workspace_for(p, True, q.device)
+    rc = gdpa_backward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                       _ptr(q_offsets), _ptr(kv_offsets), _ptr(bias), _ptr(dq), _ptr(dk),
+                       _ptr(dv), None, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "gdpa_backward")
+    return dq, dk, dv, workspace
+
+
+def device_status(workspace, stream=None) -> int:
+    return gdpa_get_device_status(_ptr(workspace), _stream(stream))

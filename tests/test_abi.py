@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every symbol include/gdpa.h declares;
+host-side argument checks (no GPU needed: they return before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from pffn_attention_b200 import gdpa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdpa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDPA_API\s+[\w\s\*]+?\b(gdpa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return gdpa.load()
+
+
+def test_header_declares_the_api():
+    assert set(declared_symbols()) == set(gdpa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert gdpa.gdpa_version() >= 100
+    for code in range(7):
+        assert gdpa.gdpa_status_string(code) not in ("", "unknown status")
+    assert gdpa.gdpa_status_string(99) == "unknown status"
+
+
+def _params(**kw):
+    base = dict(B=2, H=2, D=64, total_q=10, total_kv=8, phi=0, scale=1.0)
+    base.update(kw)
+    B, H, D, tq, tk = (base.pop(x) for x in ("B", "H", "D", "total_q", "total_kv"))
+    return gdpa.make_params(B, H, D, tq, tk, **base)
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned, never dereferenced: rejected first
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(D=48), 2), (dict(D=256), 2), (dict(phi=7), 2), (dict(bias_kind=5), 2),
+    (dict(H=0), 1), (dict(B=-1), 1), (dict(total_q=-3), 1), (dict(window=(-2, 0)), 1),
+    (dict(B=16385), 2), (dict(scale=float("nan")), 1),
+])
+def test_invalid_params_rejected(lib, kw, expect):
+    p = _params(**kw)
+    rc = gdpa.gdpa_forward(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20, None)
+    assert rc == expect
+    assert gdpa.gdpa_workspace_size(p, 0) == 0
+
+
+def test_null_and_unaligned_pointers_rejected(lib):
+    p = _params()
+    assert gdpa.gdpa_forward(None if False else p, None, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                             FAKE, 1 << 20, None) == 1
+    assert gdpa.gdpa_forward(p, FAKE + 8, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20,
+                             None) == 1
+    assert gdpa.gdpa_forward(p, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, None, FAKE, 1 << 20,
+                             None) == 1
+    # bias pointer given without a bias kind, and a bias kind without a pointer
+    assert gdpa.gdpa_forward(p, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 20,
+                             None) == 1
+    pb = _params(bias_kind=2)
+    assert gdpa.gdpa_forward(pb, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20,
+                             None) == 1
+    assert lib.gdpa_forward(None, None, None, None, None, None, None, None, None, None, 0,
+                            None) == 1
+
+
+def test_workspace_size_grows_with_problem(lib):
+    small = gdpa.gdpa_workspace_size(_params(), 0)
+    big = gdpa.gdpa_workspace_size(_params(B=4000, total_q=4000), 0)
+    assert 256 < small < big
+    bwd = gdpa.gdpa_workspace_size(_params(phi=1, max_seqlen_q=10), 1)
+    assert bwd > gdpa.gdpa_workspace_size(_params(phi=1), 0)
+
+
+def test_tile_shape_query(lib):
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64))
+    assert (rc, bm, bn) == (0, 128, 64)
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=65))
+    assert (rc, bm, bn) == (0, 128, 128)

@@ -128,7 +128,8 @@ def make_workload(cfg: int, B: Optional[int] = None, seed: Optional[int] = None,
 
     ``seed`` defaults to the workload number.  ``q_lens`` / ``kv_lens``
     override the drawn lengths (edge-case tests).  ``overrides`` may replace
-    H, D, phi, scale, window or bias kind for edge-case tests.
+    H, D, phi, scale, window, bias kind, q_std or kv_std for edge-case
+    tests.
     """
     spec = dict(CONFIGS[cfg])
     seed = cfg if seed is None else seed
@@ -154,11 +155,13 @@ def make_workload(cfg: int, B: Optional[int] = None, seed: Optional[int] = None,
     ko = offsets_from_lengths(kl)
     tq, tk = int(qo[-1]), int(ko[-1])
 
+    q_std = overrides.get("q_std", spec["q_std"])
+    kv_std = overrides.get("kv_std", spec["kv_std"])
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
-    q = _normal_bf16((tq, H, D), spec["q_std"], gen, device)
-    k = _normal_bf16((tk, H, D), spec["kv_std"], gen, device)
-    v = _normal_bf16((tk, H, D), spec["kv_std"], gen, device)
+    q = _normal_bf16((tq, H, D), q_std, gen, device)
+    k = _normal_bf16((tk, H, D), kv_std, gen, device)
+    v = _normal_bf16((tk, H, D), kv_std, gen, device)
     bias = None
     if bias_kind != BIAS_NONE:
         bias = torch.randn((H, tk), generator=gen, device=device, dtype=torch.float32)
