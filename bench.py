@@ -1,0 +1,466 @@
+"""GDPA benchmark: useful TFLOP/s of a forward + backward training step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+One step is the whole hot path on one batch: the gated softmax training
+workload (B=4096 samples, H=8, D=128, query lengths uniform in [256, 1024],
+256 context-generated keys per sample, log-sigmoid gate, dO ~ N(0,1)) through
+gdpa_forward then gdpa_backward.  Useful FLOPs count 4*D per visible
+(query, key) pair and head in the forward and 8*D in the backward (padding and
+recomputation excluded).  The inputs (about 15 GB) are larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun, one process per GPU): samples are independent, so each
+rank runs its own full batch (weak scaling) with no collective on the data
+path; the time is the max over ranks of the CUDA-event time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation
+there is) on the host cores, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, make_workload  # noqa: E402
+
+METRIC = "GDPA fwd/bwd useful TFLOP/s on 1 B200; % of dense BF16 tensor peak"
+WORKLOADS = {CONFIGS[c]["name"]: c for c in CONFIGS}
+DEFAULT_WORKLOAD = CONFIGS[5]["name"]
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- accounting
+def visible_pairs_per_sample(w) -> np.ndarray:
+    """Visible (query, key) pairs of each sample (per head)."""
+    ql, kl = w.q_lens.astype(np.int64), w.kv_lens.astype(np.int64)
+    if w.window_left < 0 and w.window_right < 0:
+        return ql * kl
+    out = np.zeros(w.B, np.int64)
+    for b in range(w.B):
+        i = np.arange(ql[b])
+        lo = np.maximum(0, i - w.window_left) if w.window_left >= 0 else np.zeros_like(i)
+        hi = (np.minimum(kl[b] - 1, i + w.window_right) if w.window_right >= 0
+              else np.full_like(i, kl[b] - 1))
+        out[b] = np.maximum(0, hi - lo + 1).sum()
+    return out
+
+
+def useful_flops(w, backward: bool) -> tuple[float, float]:
+    pairs = float(visible_pairs_per_sample(w).sum()) * w.H
+    fwd = 4.0 * w.D * pairs
+    bwd = 8.0 * w.D * pairs if backward else 0.0
+    return fwd, bwd
+
+
+def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
+    """Bytes a perfect kernel must move: each input read once, each output
+    written once (bf16 tensors, fp32 gate/LSE)."""
+    tq, tk, H, D = w.total_q, w.total_kv, w.H, w.D
+    gate = 4.0 * H * tk if w.bias_kind else 0.0
+    lse = 4.0 * H * tq if w.phi == 1 else 0.0
+    fwd = 2.0 * H * D * (tq + 2 * tk + tq) + gate + lse           # Q, K, V -> O (+ LSE)
+    bwd = 0.0
+    if backward:
+        bwd = (2.0 * H * D * (tq * 4 + tk * 4)                     # Q, O, dO, dQ; K, V, dK, dV
+               + gate + lse)
+    return fwd, bwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, \
+            "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (clocks and throttle reasons)."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="gdpa_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from pffn_attention_b200 import gdpa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = WORKLOADS[args.workload]
+    training = cfg == 5
+    # each rank owns an independent batch of the same distribution
+    w = make_workload(cfg, device=dev, seed=cfg + 1000 * rank, with_dout=training)
+    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+    ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
+    p = gdpa.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
+                         window=(w.window_left, w.window_right), bias_kind=w.bias_kind,
+                         max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv)
+    o = torch.empty_like(w.q)
+    lse = torch.empty((w.H, w.total_q), dtype=torch.float32, device=dev)
+    ws_f = gdpa.workspace_for(p, False, dev)
+    if training:
+        dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
+        ws_b = gdpa.workspace_for(p, True, dev)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rc = gdpa.gdpa_forward(p, ptr(w.q), ptr(w.k), ptr(w.v), ptr(qo), ptr(ko), ptr(w.bias),
+                               ptr(o), ptr(lse), ptr(ws_f), ws_f.numel(), sh)
+        if rc:
+            raise gdpa.GdpaError(rc, "gdpa_forward")
+        if ev is not None:
+            ev[1].record(stream)
+        if training:
+            rc = gdpa.gdpa_backward(p, ptr(w.q), ptr(w.k), ptr(w.v), ptr(o), ptr(w.dout), ptr(lse),
+                                    ptr(qo), ptr(ko), ptr(w.bias), ptr(dq), ptr(dk), ptr(dv),
+                                    None, ptr(ws_b), ws_b.numel(), sh)
+            if rc:
+                raise gdpa.GdpaError(rc, "gdpa_backward")
+        if ev is not None:
+            ev[2].record(stream)
+
+    launches_per_step = 2 + (3 if training else 0)  # schedule+fwd, schedule+delta+bwd
+    torch.cuda.synchronize(dev)  # inputs were generated on the default stream
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    st = gdpa.gdpa_get_device_status(ptr(ws_f), sh)
+    if st or (training and gdpa.gdpa_get_device_status(ptr(ws_b), sh)):
+        raise RuntimeError(f"device status after warm-up: {st}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local_rank))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if training else 0.0
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    f_fwd, f_bwd = useful_flops(w, training)
+    b_fwd, b_bwd = algorithmic_bytes(w, training)
+    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+
+    # dominant call: the backward in a training step, else the forward
+    if training:
+        dom_name, dom_ms, dom_bytes, dom_flops = "gdpa_backward", bwd_ms, b_bwd, f_bwd
+    else:
+        dom_name, dom_ms, dom_bytes, dom_flops = "gdpa_forward", fwd_ms, b_fwd, f_fwd
+    achieved_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+                "traffic": None, "kernel": dom_name, "peak_source": peak_src,
+                "tensor_tflops": round(dom_flops / (dom_ms * 1e-3) / 1e12, 1),
+                "tensor_frac": round(dom_flops / (dom_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, p, qo, ko, training, dev, world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "H": w.H, "D": w.D,
+                   "global_batch": w.B * world, "seq_len": f"q U[256,1024] / kv 256"
+                   if cfg == 5 else "see workload", "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "pct_of_peak": {"measured_burst": round(value / world / peaks["bf16_tflops"], 4),
+                        "measured_sustained": round(value / world
+                                                    / peaks["bf16_tflops_sustained"], 4),
+                        "spec": round(value / world / SPEC_BF16_TFLOPS, 4)},
+        "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+        "fwd_tflops": round(f_fwd / (fwd_ms * 1e-3) / 1e12, 1),
+        "bwd_tflops": round(f_bwd / (bwd_ms * 1e-3) / 1e12, 1) if training else None,
+        "roofline": roofline,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    return line, w
+
+
+def run_e2e(args, w, p, qo, ko, training, dev, world):
+    """Same metric through the C ABI with host buffers: every step copies the
+    inputs from pinned host memory and reads all outputs back."""
+    import torch
+
+    from pffn_attention_b200 import gdpa
+
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    names = ["q", "k", "v"] + (["bias"] if w.bias is not None else []) + \
+        (["dout"] if training else [])
+    host_in = {n: pinned_copy(getattr(w, n)) for n in names}
+    host_qo = qo.cpu().pin_memory()
+    host_ko = ko.cpu().pin_memory()
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    dqo, dko = torch.empty_like(qo), torch.empty_like(ko)
+    o = torch.empty_like(dev_in["q"])
+    lse = torch.empty((w.H, w.total_q), dtype=torch.float32, device=dev)
+    outs = {"o": o}
+    if training:
+        outs.update(dq=torch.empty_like(dev_in["q"]), dk=torch.empty_like(dev_in["k"]),
+                    dv=torch.empty_like(dev_in["v"]))
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
+    ws_f = gdpa.workspace_for(p, False, dev)
+    ws_b = gdpa.workspace_for(p, True, dev) if training else None
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
+        host_qo.numel() * 4 + host_ko.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def step():
+        with torch.cuda.stream(stream):
+            for n, t in host_in.items():
+                dev_in[n].copy_(t, non_blocking=True)
+            dqo.copy_(host_qo, non_blocking=True)
+            dko.copy_(host_ko, non_blocking=True)
+        rc = gdpa.gdpa_forward(p, ptr(dev_in["q"]), ptr(dev_in["k"]), ptr(dev_in["v"]), ptr(dqo),
+                               ptr(dko), ptr(dev_in.get("bias")), ptr(o), ptr(lse), ptr(ws_f),
+                               ws_f.numel(), sh)
+        assert rc == 0, rc
+        if training:
+            rc = gdpa.gdpa_backward(p, ptr(dev_in["q"]), ptr(dev_in["k"]), ptr(dev_in["v"]), ptr(o),
+                                    ptr(dev_in["dout"]), ptr(lse), ptr(dqo), ptr(dko),
+                                    ptr(dev_in.get("bias")), ptr(outs["dq"]), ptr(outs["dk"]),
+                                    ptr(outs["dv"]), None, ptr(ws_b), ws_b.numel(), sh)
+            assert rc == 0, rc
+        with torch.cuda.stream(stream):
+            for n, t in outs.items():
+                host_out[n].copy_(t, non_blocking=True)
+
+    steps = max(2, min(args.steps, 5))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    f_fwd, f_bwd = useful_flops(w, training)
+    return {"value": round((f_fwd + f_bwd) * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ----------------------------------------------------------------- the oracle
+def oracle_sample(cfg: int, n_samples: int, seed: int, training: bool):
+    """A fresh batch of n_samples drawn from the workload's distributions."""
+    return make_workload(cfg, B=n_samples, seed=seed, device="cpu", with_dout=training)
+
+
+def time_oracle(sub, training: bool) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward_workload(sub)
+    if training:
+        oracle.backward_workload(sub)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(args, w, training: bool, target_s: float = 12.0) -> dict:
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload."""
+    import oracle
+    cfg = WORKLOADS[args.workload]
+    n = 2
+    dt = time_oracle(oracle_sample(cfg, n, 7000, training), training)
+    n = int(min(w.B, max(2, n * target_s / max(dt, 1e-3))))
+    sub = oracle_sample(cfg, n, 7001, training)
+    dt = time_oracle(sub, training)
+    f_fwd, f_bwd = useful_flops(sub, training)
+    return {"value": round((f_fwd + f_bwd) / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} samples drawn from {args.workload}'s distributions (all {sub.H} "
+                      f"heads, {int(sub.total_q)} query rows), fwd{'+bwd' if training else ''}, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    import oracle
+    cfg = WORKLOADS[args.workload]
+    training = cfg == 5
+    per_step = 6 if training else 64
+    for i in range(args.warmup):
+        time_oracle(oracle_sample(cfg, 2, 100 + i, training), training)
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        sub = oracle_sample(cfg, per_step, 200 + i, training)
+        times.append(time_oracle(sub, training))
+        f, b = useful_flops(sub, training)
+        flops += f + b
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = (f"{per_step} samples per step drawn from {args.workload}'s distributions "
+              f"(all heads)")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total / args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------- main
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        line, w = run_ours(args, rank, world, local)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(args, w, WORKLOADS[args.workload] == 5)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -246,12 +246,88 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
                             const int32_t* q_offsets, const int32_t* kv_offsets,
                             const float* bias, void* dq, void* dk, void* dv, float* dbias,
                             void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
-  (void)q; (void)k; (void)v; (void)o; (void)dout; (void)lse; (void)q_offsets;
-  (void)kv_offsets; (void)bias; (void)dq; (void)dk; (void)dv; (void)dbias; (void)workspace;
-  (void)workspace_bytes; (void)stream;
   gdpa_status_t st = check_params(p);
   if (st != GDPA_OK) return st;
-  return GDPA_ERR_UNSUPPORTED;
+  if (dbias) return GDPA_ERR_UNSUPPORTED;
+  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
+  const bool softmax = p->phi == GDPA_PHI_SOFTMAX;
+  if (p->total_q > 0 && (!q || !dout || !dq || (softmax && (!o || !lse))))
+    return GDPA_ERR_INVALID_ARG;
+  if (p->total_kv > 0 && (!k || !v || !dk || !dv)) return GDPA_ERR_INVALID_ARG;
+  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return GDPA_ERR_INVALID_ARG;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  const WorkspaceLayout L = make_layout(p, 1, sms);
+  if (!workspace || workspace_bytes < L.total) return GDPA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(ws + L.tile_start);
+  float* delta = reinterpret_cast<float*>(ws + L.delta);
+  float* scratch = reinterpret_cast<float*>(ws + L.dq_scratch);
+  cudaStream_t s = (cudaStream_t)stream;
+
+  cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, 128, p->window_left,
+                                  p->window_right, tile_start, order, status, s);
+  if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  if (p->B == 0 || (p->total_q == 0 && p->total_kv == 0)) return GDPA_OK;
+  if (softmax && p->total_q > 0) {
+    e = launch_bwd_preprocess(static_cast<const __nv_bfloat16*>(o),
+                              static_cast<const __nv_bfloat16*>(dout), delta, p->total_q, p->H,
+                              p->D, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
+  CUtensorMap tq, tdo, tk, tv;
+  if (p->total_q > 0) {
+    if (!make_map(&tq, q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+    if (!make_map(&tdo, dout, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+  }
+  if (p->total_kv > 0) {
+    if (!make_map(&tk, k, p->total_kv, p->H, p->D, 128)) return GDPA_ERR_CUDA;
+    if (!make_map(&tv, v, p->total_kv, p->H, p->D, 128)) return GDPA_ERR_CUDA;
+  }
+  if (p->total_q == 0) {  // no query: only zero dK/dV rows are written; maps unused
+    tq = tk;
+    tdo = tk;
+  }
+  if (p->total_kv == 0) {  // no key: only zero dQ rows are written; maps unused
+    tk = tq;
+    tv = tq;
+  }
+  BwdArgs a{};
+  a.q_offsets = q_offsets;
+  a.kv_offsets = kv_offsets;
+  a.order = order;
+  a.bias = bias;
+  a.lse = lse;
+  a.delta = delta;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dq_scratch = scratch;
+  a.status = status;
+  a.total_q = p->total_q;
+  a.total_kv = p->total_kv;
+  a.B = p->B;
+  a.H = p->H;
+  a.n_units = p->B * p->H;
+  a.max_q = eff_max_q(p);
+  a.max_kv = eff_max_kv(p);
+  a.dq_slot_rows = L.dq_slot_rows;
+  a.scale = p->scale;
+  a.phi = p->phi;
+  a.bias_kind = p->bias_kind;
+  a.wl = p->window_left;
+  a.wr = p->window_right;
+  a.debug_flags = p->debug_flags;
+  a.timeout_ns = timeout_ns(p);
+  e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
+  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 
 gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {

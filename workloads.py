@@ -128,8 +128,8 @@ def make_workload(cfg: int, B: Optional[int] = None, seed: Optional[int] = None,
 
     ``seed`` defaults to the workload number.  ``q_lens`` / ``kv_lens``
     override the drawn lengths (edge-case tests).  ``overrides`` may replace
-    H, D, phi, scale, window, bias kind, q_std or kv_std for edge-case
-    tests.
+    H, D, phi, scale, window, bias kind, q_std, kv_std or dout_std for
+    edge-case tests.
     """
     spec = dict(CONFIGS[cfg])
     seed = cfg if seed is None else seed
@@ -165,7 +165,8 @@ def make_workload(cfg: int, B: Optional[int] = None, seed: Optional[int] = None,
     bias = None
     if bias_kind != BIAS_NONE:
         bias = torch.randn((H, tk), generator=gen, device=device, dtype=torch.float32)
-    dout = _normal_bf16((tq, H, D), 1.0, gen, device) if with_dout else None
+    dout_std = overrides.get("dout_std", 1.0)
+    dout = _normal_bf16((tq, H, D), dout_std, gen, device) if with_dout else None
     return Workload(name=spec["name"], B=Bn, H=H, D=D, phi=phi, scale=float(scale),
                     window_left=int(wl), window_right=int(wr), bias_kind=bias_kind,
                     q_lens=ql, kv_lens=kl, q_offsets=qo, kv_offsets=ko,
