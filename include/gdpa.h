@@ -123,6 +123,32 @@ GDPA_API gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, cons
                             void* dk, void* dv, float* dbias, void* workspace,
                             size_t workspace_bytes, gdpa_stream_t stream);
 
+/* Forward for callers that cannot allocate device memory.  (The Kunlun pages
+ * have no counterpart to this entry point; it exists for this library's users.)
+ * Some callers have no way to give the library a workspace: a plugin inside a
+ * host framework that owns all device memory and exposes no allocator, or a
+ * serving process that plans its memory at start-up and must not allocate on
+ * the request path.  This call computes exactly what gdpa_forward computes,
+ * with the forward's scratch (status, sample order, tile prefix) held in a
+ * fixed 131,584-byte array compiled into the library instead of a caller
+ * workspace; every GPU that loads the library keeps its own copy until the
+ * process exits.  It allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).  The caller still passes inputs and outputs.
+ * Limits: B <= 16384, the library's own batch limit; beyond it (or if the
+ * scratch would not fit) it returns GDPA_ERR_WORKSPACE.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and caches it, so make that first call before any
+ * stream capture.  All calls on a device share the one array: calls that
+ * overlap on the GPU (on different streams, or from different host threads)
+ * race and must be serialised by the caller.  Each call overwrites what it
+ * needs, so nothing from an earlier call leaks in.  Device-side status of
+ * these calls is not readable through gdpa_get_device_status. */
+GDPA_API gdpa_status_t gdpa_forward_no_alloc(const gdpa_params_t* p, const void* q,
+                                             const void* k, const void* v,
+                                             const int32_t* q_offsets,
+                                             const int32_t* kv_offsets, const float* bias,
+                                             void* o, float* lse, gdpa_stream_t stream);
+
 /* The jagged tile schedule the kernels use, exported so it can be checked:
  * query tiles of block_m rows, key blocks of block_n keys (both multiples of
  * 16 in [16, 256]); per sample the cost sum over its tiles of (1 + key blocks

@@ -25,7 +25,7 @@ BIAS = {"none": 0, "add": 1, "gate": 2}
 
 EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
-            "gdpa_version")
+            "gdpa_version", "gdpa_forward_no_alloc")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -73,6 +73,8 @@ def load(path: str = LIB_PATH):
     lib.gdpa_get_device_status.restype = ctypes.c_int
     lib.gdpa_status_string.argtypes = [ctypes.c_int]
     lib.gdpa_status_string.restype = ctypes.c_char_p
+    lib.gdpa_forward_no_alloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, st]
+    lib.gdpa_forward_no_alloc.restype = ctypes.c_int
     lib.gdpa_version.argtypes = []
     lib.gdpa_version.restype = ctypes.c_int
     _lib = lib
@@ -88,6 +90,12 @@ def gdpa_forward(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, workspace, wor
                  stream) -> int:
     return int(load().gdpa_forward(ctypes.byref(p), q, k, v, q_offsets, kv_offsets, bias, o, lse,
                                    workspace, workspace_bytes, stream))
+
+
+def gdpa_forward_no_alloc(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, stream) -> int:
+    """Forward with the library's built-in scratch (no caller workspace)."""
+    return int(load().gdpa_forward_no_alloc(ctypes.byref(p), q, k, v, q_offsets, kv_offsets,
+                                            bias, o, lse, stream))
 
 
 def gdpa_backward(p, q, k, v, o, dout, lse, q_offsets, kv_offsets, bias, dq, dk, dv, dbias,

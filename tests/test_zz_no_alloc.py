@@ -1,0 +1,53 @@
+"""gdpa_forward_no_alloc, the forward for callers that cannot allocate device
+memory (for example a plugin inside a framework that owns all device memory,
+or a serving process that must not allocate on its request path).  It must
+give what gdpa_forward gives, on consecutive calls that share its built-in
+scratch.  This file is collected last so that a failure here never hides
+another test's result."""
+import numpy as np
+import pytest
+import torch
+
+from parity import compare
+from workloads import PHI_SILU, make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_both(gdpa, w):
+    dev = torch.device("cuda")
+    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+    ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    bias = w.bias.to(dev) if w.bias is not None else None
+    kw = dict(phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+              bias_kind=w.bias_kind, max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv)
+    ref_o, ref_lse, ws = gdpa.forward(q, k, v, qo, ko, bias=bias, **kw)
+    assert gdpa.device_status(ws) == 0
+    p = gdpa.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, **kw)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((w.H, w.total_q), float("nan"), device=dev)
+    stream = torch.cuda.current_stream()
+    rc = gdpa.gdpa_forward_no_alloc(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), qo.data_ptr(),
+                                    ko.data_ptr(), None if bias is None else bias.data_ptr(),
+                                    o.data_ptr(), lse.data_ptr(), stream.cuda_stream)
+    assert rc == 0, gdpa.gdpa_status_string(rc)
+    torch.cuda.synchronize()
+    return ref_o, ref_lse, o, lse
+
+
+def test_no_alloc_forward_matches_forward_on_consecutive_calls(cuda_lib):
+    # call 1: gated softmax; call 2: SiLU with a different batch and head dim
+    cases = [make_workload(5, B=5, seed=501, with_dout=False),
+             make_workload(2, B=9, seed=502, phi=PHI_SILU)]
+    for w in cases:
+        ref_o, ref_lse, o, lse = _run_both(cuda_lib, w)
+        compare("O", o, ref_o.double().cpu().numpy())
+        if w.phi == 1:
+            np.testing.assert_allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), atol=2e-3,
+                                       rtol=0)
+
+
+def test_no_alloc_rejects_batches_beyond_its_scratch(cuda_lib):
+    p = cuda_lib.make_params(16385, 1, 64, 16385, 16385)
+    assert cuda_lib.gdpa_forward_no_alloc(p, 16, 16, 16, 16, 16, None, 16, None, None) == 3
