@@ -154,7 +154,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     cfg = WORKLOADS[args.workload]
     training = cfg == 5
     # each rank owns an independent batch of the same distribution
-    w = make_workload(cfg, device=dev, seed=cfg + 1000 * rank, with_dout=training)
+    w = make_workload(cfg, B=args.batch, device=dev, seed=cfg + 1000 * rank, with_dout=training)
     qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
     ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
     p = gdpa.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
@@ -252,7 +252,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B": w.B, "H": w.H, "D": w.D,
+        "config": {"workload": args.workload + ("" if args.batch is None else
+                                                f" (batch {args.batch}, profiling)"),
+                   "B": w.B, "H": w.H, "D": w.D,
                    "global_batch": w.B * world, "seq_len": f"q U[256,1024] / kv 256"
                    if cfg == 5 else "see workload", "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (no flush)"},
@@ -427,6 +429,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="samples per rank (default: the workload's full batch); smaller "
+                         "batches are for profiling captures")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -86,8 +86,10 @@ typedef struct {
   int window_left;    /* -1 = unbounded */
   int window_right;   /* -1 = unbounded */
   int bias_kind;      /* GDPA_BIAS_*: none, beta = bias, or beta = log sigmoid(bias) */
-  int debug_flags;    /* 0 in normal use; bit 0 drops one producer arrival so that
-                         the bounded-wait path can be tested (returns TIMEOUT) */
+  int debug_flags;    /* 0 in normal use.  Bit 0 drops one producer arrival so that
+                         the bounded-wait path can be tested (returns TIMEOUT);
+                         bit 1 makes the forward use 128-key blocks even when
+                         every sample has at most 64 keys (tests both tile shapes) */
   int wait_timeout_us;/* bound on any single in-kernel wait; 0 = 2000000 (2 s) */
 } gdpa_params_t;
 
@@ -129,8 +131,8 @@ GDPA_API gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, cons
  * host framework that owns all device memory and exposes no allocator, or a
  * serving process that plans its memory at start-up and must not allocate on
  * the request path.  This call computes exactly what gdpa_forward computes,
- * with the forward's scratch (status, sample order, tile prefix) held in a
- * fixed 131,584-byte array compiled into the library instead of a caller
+ * with the forward's scratch (status, sample order, tile prefix, per-sample
+ * descriptors) held in a fixed 393,728-byte array compiled into the library instead of a caller
  * workspace; every GPU that loads the library keeps its own copy until the
  * process exits.  It allocates nothing (no cudaMalloc, cudaFree or
  * allocating library routine).  The caller still passes inputs and outputs.

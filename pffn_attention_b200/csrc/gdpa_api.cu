@@ -89,6 +89,8 @@ WorkspaceLayout make_layout(const gdpa_params_t* p, int backward, int sms) {
   off += align256((size_t)std::max(p->B, 1) * 4);
   L.tile_start = off;
   off += align256((size_t)(p->B + 1) * 4);
+  L.info = off;
+  off += align256((size_t)std::max(p->B, 1) * 16);
   if (backward) {
     L.delta = off;
     if (p->phi == GDPA_PHI_SOFTMAX) off += align256((size_t)p->H * (size_t)p->total_q * 4);
@@ -154,7 +156,7 @@ gdpa_status_t gdpa_forward_tile_shape(const gdpa_params_t* p, int* block_m, int*
   if (st != GDPA_OK) return st;
   if (!block_m || !block_n) return GDPA_ERR_INVALID_ARG;
   *block_m = kBlockM;
-  *block_n = forward_block_n(p->D, p->phi, eff_max_kv(p));
+  *block_n = forward_block_n(p->D, p->phi, eff_max_kv(p), p->debug_flags);
   return GDPA_OK;
 }
 
@@ -170,7 +172,7 @@ gdpa_status_t gdpa_tile_schedule(const gdpa_params_t* p, int block_m, int block_
   int sms = 0;
   if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, block_m, block_n, p->window_left,
-                                  p->window_right, tile_start, order, nullptr,
+                                  p->window_right, tile_start, order, nullptr, 0, 0, nullptr,
                                   (cudaStream_t)stream);
   return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
@@ -197,11 +199,13 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
   int32_t* tile_start = reinterpret_cast<int32_t*>(ws + L.tile_start);
-  const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p));
+  int4* info = reinterpret_cast<int4*>(ws + L.info);
+  const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p), p->debug_flags);
   cudaStream_t s = (cudaStream_t)stream;
 
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, block_n,
-                                  p->window_left, p->window_right, tile_start, order, status, s);
+                                  p->window_left, p->window_right, tile_start, order, info,
+                                  eff_max_q(p), eff_max_kv(p), status, s);
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
   if (p->B == 0 || p->total_q == 0) return GDPA_OK;
 
@@ -218,6 +222,7 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.q_offsets = q_offsets;
   a.kv_offsets = kv_offsets;
   a.order = order;
+  a.info = info;
   a.bias = bias;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = p->phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
@@ -236,8 +241,7 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.wr = p->window_right;
   a.debug_flags = p->debug_flags;
   a.timeout_ns = timeout_ns(p);
-  const int grid = std::max(1, std::min(a.n_units, sms));
-  e = launch_forward(a, p->D, block_n, tq, tk, tv, grid, s);
+  e = launch_forward(a, p->D, block_n, tq, tk, tv, sms, s);
   return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 
@@ -268,12 +272,14 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
   int32_t* tile_start = reinterpret_cast<int32_t*>(ws + L.tile_start);
+  int4* info = reinterpret_cast<int4*>(ws + L.info);
   float* delta = reinterpret_cast<float*>(ws + L.delta);
   float* scratch = reinterpret_cast<float*>(ws + L.dq_scratch);
   cudaStream_t s = (cudaStream_t)stream;
 
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, 128, p->window_left,
-                                  p->window_right, tile_start, order, status, s);
+                                  p->window_right, tile_start, order, info, eff_max_q(p),
+                                  eff_max_kv(p), status, s);
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
   if (p->B == 0 || (p->total_q == 0 && p->total_kv == 0)) return GDPA_OK;
   if (softmax && p->total_q > 0) {
@@ -303,6 +309,7 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   a.q_offsets = q_offsets;
   a.kv_offsets = kv_offsets;
   a.order = order;
+  a.info = info;
   a.bias = bias;
   a.lse = lse;
   a.delta = delta;

@@ -19,9 +19,10 @@
 // the thread that reads it back, so no atomics or fences are needed, and the
 // slot (rows = max query length) stays in L2.
 //
-// TMEM (512 columns): [0,128) S^T, later dQ; [128,256) dP^T; then dK, dV.
-// Shared memory: K, V of the key block; Q, dO of the tile; P^T and dS^T (bf16,
-// 64-query panels, 128-byte swizzle) for the dV/dK/dQ MMAs.
+// TMEM (512 columns): [0,128) S^T, later dQ; [128,256) dP^T, then P^T (bf16,
+// the A operand of the dV MMA); then dK, dV.
+// Shared memory: K, V of the key block; a 2-stage ring of Q, dO tiles; dS^T
+// (bf16, 64-query panels, 128-byte swizzle) for the dK and dQ MMAs.
 //
 // Warp roles (384 threads): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator,
 // 3 LSE/delta loader, 4-11 two warpgroups that split each tile's 128 query
@@ -48,48 +49,26 @@ struct BwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int QT_BYTES = BM * D * 2;
   static constexpr int PT_BYTES = BN * BM * 2;
+  static constexpr int NQ = 2;         // Q/dO ring stages
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_Q = OFF_V + KV_BYTES;
-  static constexpr int OFF_DO = OFF_Q + QT_BYTES;
-  static constexpr int OFF_PT = OFF_DO + QT_BYTES;
-  static constexpr int OFF_DST = OFF_PT + PT_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;                 // [NQ] Q tiles
+  static constexpr int OFF_DO = OFF_Q + NQ * QT_BYTES;           // [NQ] dO tiles
+  static constexpr int OFF_DST = OFF_DO + NQ * QT_BYTES;
   static constexpr int OFF_ROW = OFF_DST + PT_BYTES;   // float [2][2][BM]: LSE*log2e, delta
   static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * BM * 4;
-  static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_QFULL = 2, B_QEMPTY = 3, B_SFULL = 4,
-                       B_PFULL = 5, B_DQFULL = 6, B_DQEMPTY = 7, B_DKVFULL = 8,
-                       B_DKVEMPTY = 9, B_RFULL = 10, B_REMPTY = 12, NBARS = 14;
+  static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_QFULL = 2, B_QEMPTY = 4, B_SFULL = 6,
+                       B_PFULL = 7, B_DQFULL = 8, B_DQEMPTY = 9, B_DKVFULL = 10,
+                       B_DKVEMPTY = 11, B_RFULL = 12, B_REMPTY = 14, NBARS = 16;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr int T_S = 0, T_DP = 128, T_DK = 256, T_DV = 256 + D;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES;  // base is 1024-aligned (checked at entry)
+  static constexpr int T_S = 0, T_DP = 128, T_PT = 128, T_DK = 256, T_DV = 256 + D;
   static constexpr int TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-struct BUnit {
-  int b, h, q0, Lq, k0, Lk;
-};
-
-__device__ __forceinline__ int bunit_index(int round, int cta, int grid) {
-  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
-}
-
-__device__ __forceinline__ BUnit load_bunit(const BwdArgs& a, int u) {
-  BUnit t;
-  const int p = u / a.H;
-  t.h = u - p * a.H;
-  t.b = a.order[p];
-  t.q0 = a.q_offsets[t.b];
-  t.Lq = a.q_offsets[t.b + 1] - t.q0;
-  t.k0 = a.kv_offsets[t.b];
-  t.Lk = a.kv_offsets[t.b + 1] - t.k0;
-  if (t.Lq > a.max_q || t.Lk > a.max_kv) {
-    t.Lq = 0;
-    t.Lk = 0;
-  }
-  return t;
-}
+using BUnit = GdpaUnit;
 
 // Key blocks [kb0, kb1) query tile m0 may see (same rule as the forward).
 __device__ __forceinline__ void bwd_kv_range(int m0, int Lk, int wl, int wr, int& kb0, int& kb1) {
@@ -109,9 +88,8 @@ struct BSmem {
   uint8_t* ptr;
   __device__ uint32_t k() const { return base + C::OFF_K; }
   __device__ uint32_t v() const { return base + C::OFF_V; }
-  __device__ uint32_t q() const { return base + C::OFF_Q; }
-  __device__ uint32_t dout() const { return base + C::OFF_DO; }
-  __device__ uint32_t pt() const { return base + C::OFF_PT; }
+  __device__ uint32_t q(int s) const { return base + C::OFF_Q + s * C::QT_BYTES; }
+  __device__ uint32_t dout(int s) const { return base + C::OFF_DO + s * C::QT_BYTES; }
   __device__ uint32_t dst() const { return base + C::OFF_DST; }
   __device__ float* lse2(int s) const {
     return reinterpret_cast<float*>(ptr + C::OFF_ROW) + s * 2 * C::BM;
@@ -164,10 +142,9 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
   uint32_t kvi = 0, qi = 0;
-  for (int round = 0;; ++round) {
-    const int u = bunit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const BUnit t = load_bunit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  BUnit t;
+  while (units.next(t)) {
     bool ok = for_each_pair(
         t, a.wl, a.wr,
         [&](int kb, int mt, bool first, bool) -> bool {
@@ -184,14 +161,15 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
             }
             ++kvi;
           }
-          if (!mbar_wait(sm.bar(C::B_QEMPTY), (qi & 1) ^ 1, abort, a.status, a.timeout_ns,
-                         0x1000 + C::B_QEMPTY))
+          const int qs = qi % C::NQ;
+          if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((qi / C::NQ) & 1) ^ 1, abort, a.status,
+                         a.timeout_ns, 0x1000 + C::B_QEMPTY + qs))
             return false;
-          mbar_arrive_expect_tx(sm.bar(C::B_QFULL), 2 * C::QT_BYTES);
+          mbar_arrive_expect_tx(sm.bar(C::B_QFULL + qs), 2 * C::QT_BYTES);
           for (int p = 0; p < C::NPANEL; ++p) {
-            tma_load_3d(sm.q() + p * C::BM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL),
+            tma_load_3d(sm.q(qs) + p * C::BM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + qs),
                         p * C::PANEL_ELEMS, t.h, t.q0 + mt * kBlockM, pol_stream);
-            tma_load_3d(sm.dout() + p * C::BM * C::PANEL_BYTES, tdo, sm.bar(C::B_QFULL),
+            tma_load_3d(sm.dout(qs) + p * C::BM * C::PANEL_BYTES, tdo, sm.bar(C::B_QFULL + qs),
                         p * C::PANEL_ELEMS, t.h, t.q0 + mt * kBlockM, pol_stream);
           }
           ++qi;
@@ -211,10 +189,9 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
   constexpr uint32_t id_dq = make_idesc_bf16(kBlockM, C::D, 1, 1);  // dQ
   constexpr uint32_t SBO = 8 * C::PANEL_BYTES;
   uint32_t kvi = 0, qi = 0, pi = 0, dqi = 0, bi = 0;
-  for (int round = 0;; ++round) {
-    const int u = bunit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const BUnit t = load_bunit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  BUnit t;
+  while (units.next(t)) {
     bool ok = for_each_pair(
         t, a.wl, a.wr,
         [&](int kb, int mt, bool first, bool last) -> bool {
@@ -225,8 +202,9 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
                            0x1100 + C::B_KVFULL))
               return false;
           }
-          if (!mbar_wait(sm.bar(C::B_QFULL), qi & 1, abort, a.status, a.timeout_ns,
-                         0x1100 + C::B_QFULL))
+          const int qs = qi % C::NQ;
+          if (!mbar_wait(sm.bar(C::B_QFULL + qs), (qi / C::NQ) & 1, abort, a.status,
+                         a.timeout_ns, 0x1100 + C::B_QFULL + qs))
             return false;
           // S^T and dP^T regions are free once the previous dQ has been read
           if (!mbar_wait(sm.bar(C::B_DQEMPTY), (dqi & 1) ^ 1, abort, a.status, a.timeout_ns,
@@ -239,8 +217,8 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
             const int w = (kk * 16 % C::PANEL_ELEMS) * 2;
             const uint64_t dk_ = make_smem_desc(sm.k() + p * C::BN * C::PANEL_BYTES + w, 16, SBO,
                                                 C::LAYOUT);
-            const uint64_t dq_ = make_smem_desc(sm.q() + p * C::BM * C::PANEL_BYTES + w, 16, SBO,
-                                                C::LAYOUT);
+            const uint64_t dq_ = make_smem_desc(sm.q(qs) + p * C::BM * C::PANEL_BYTES + w, 16,
+                                                SBO, C::LAYOUT);
             mma_bf16_ss(tmem + C::T_S, dk_, dq_, id_st, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
@@ -249,8 +227,8 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
             const int w = (kk * 16 % C::PANEL_ELEMS) * 2;
             const uint64_t dv_ = make_smem_desc(sm.v() + p * C::BN * C::PANEL_BYTES + w, 16, SBO,
                                                 C::LAYOUT);
-            const uint64_t do_ = make_smem_desc(sm.dout() + p * C::BM * C::PANEL_BYTES + w, 16,
-                                                SBO, C::LAYOUT);
+            const uint64_t do_ = make_smem_desc(sm.dout(qs) + p * C::BM * C::PANEL_BYTES + w,
+                                                16, SBO, C::LAYOUT);
             mma_bf16_ss(tmem + C::T_DP, dv_, do_, id_st, kk > 0 ? 1u : 0u);
           }
           mma_commit(sm.bar(C::B_SFULL));
@@ -263,21 +241,22 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
                                   a.timeout_ns, 0x1100 + C::B_DKVEMPTY))
             return false;
           tc_fence_after();
-          // dV += P^T dO ; dK += dS^T Q   (K = 128 queries)
+          // dV += P^T dO (P^T from TMEM) ; dK += dS^T Q   (K = 128 queries)
 #pragma unroll
           for (int kk = 0; kk < kBlockM / 16; ++kk) {
             const uint32_t a_off = (kk * 16 / 64) * (128 * 128) + (kk * 16 % 64) * 2;
-            const uint64_t pa = make_smem_desc(sm.pt() + a_off, 16, 1024, LAYOUT_SW128);
             const uint64_t sa = make_smem_desc(sm.dst() + a_off, 16, 1024, LAYOUT_SW128);
-            const uint64_t ob = make_smem_desc(sm.dout() + kk * 16 * C::PANEL_BYTES,
+            const uint64_t ob = make_smem_desc(sm.dout(qs) + kk * 16 * C::PANEL_BYTES,
                                                C::BM * C::PANEL_BYTES, SBO, C::LAYOUT);
-            const uint64_t qb = make_smem_desc(sm.q() + kk * 16 * C::PANEL_BYTES,
+            const uint64_t qb = make_smem_desc(sm.q(qs) + kk * 16 * C::PANEL_BYTES,
                                                C::BM * C::PANEL_BYTES, SBO, C::LAYOUT);
             const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-            mma_bf16_ss(tmem + C::T_DV, pa, ob, id_kv, acc);
+            // queries 16kk..16kk+15 of P^T: warpgroup kk/4's columns, 8 per step
+            mma_bf16_ts(tmem + C::T_DV, tmem + C::T_PT + (kk / 4) * 64 + (kk % 4) * 8, ob, id_kv,
+                        acc);
             mma_bf16_ss(tmem + C::T_DK, sa, qb, id_kv, acc);
           }
-          mma_commit(sm.bar(C::B_QEMPTY));
+          mma_commit(sm.bar(C::B_QEMPTY + qs));
           ++qi;
           // dQ = dS K   (M = 128 queries from dS^T, MN-major; K = 128 keys)
 #pragma unroll
@@ -309,10 +288,9 @@ __device__ void bwd_rows(const BwdArgs& a, const BSmem<C>& sm) {
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
   uint32_t ri = 0;
-  for (int round = 0;; ++round) {
-    const int u = bunit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const BUnit t = load_bunit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  BUnit t;
+  while (units.next(t)) {
     bool ok = for_each_pair(
         t, a.wl, a.wr,
         [&](int, int mt, bool, bool) -> bool {
@@ -340,17 +318,6 @@ __device__ void bwd_rows(const BwdArgs& a, const BSmem<C>& sm) {
         [&](int) { return true; });
     if (!ok) return;
   }
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
 }
 
 // Read NCOL (16 or 32 multiple) fp32 columns of this thread's TMEM lane.
@@ -401,6 +368,7 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
   constexpr int HALF_D = C::D / 2;
   constexpr bool SOFTMAX = PHI == 1;
   const float sc = SOFTMAX ? a.scale * kLog2eB : a.scale;
+  const uint64_t pol_keep = l2_policy_evict_last();
   uint32_t si = 0, dqi = 0, bi = 0, ri = 0;
 
 #define BWD_WAIT(bar_, par_, where_)                                                     \
@@ -409,15 +377,9 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
     if (!__all_sync(0xffffffffu, ok_)) return false;                                   \
   } while (0)
 
-  for (int round = 0;; ++round) {
-    const int u = bunit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const BUnit t = load_bunit(a, u);
-    if (ctid == 0 && t.Lq == 0 && t.Lk == 0) {
-      const int Lq = a.q_offsets[t.b + 1] - a.q_offsets[t.b];
-      const int Lk = a.kv_offsets[t.b + 1] - a.kv_offsets[t.b];
-      if (Lq > a.max_q || Lk > a.max_kv) record_error(a.status, 6, t.b);
-    }
+  UnitStream units(a.info, a.H, a.n_units);
+  BUnit t;
+  while (units.next(t)) {
     // dQ rows of query tiles that no key block reaches are zero
     {
       const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
@@ -496,21 +458,27 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
               s[e] = vis ? p : 0.f;
               dp[e] = vis ? ds : 0.f;
             }
-            // P^T and dS^T rows -> panel g (queries 64g .. 64g+63), 128-byte swizzle
+            // P^T row -> TMEM, two bf16 per column, into this warpgroup's own dP^T
+            // columns that have already been read: queries 64g+32ch.. at column
+            // T_PT + 64g + 16ch
+            {
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
+              tmem_st16(tmem + tl + C::T_PT + g * 64 + ch * 16, pk);
+            }
+            // dS^T row -> panel g (queries 64g .. 64g+63), 128-byte swizzle
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
               const int cir = ch * 4 + q8;    // 16-byte chunk within the 128-byte row
               const uint32_t off = g * (128 * 128) + r * 128 + ((cir ^ (r & 7)) << 4);
-              st_shared_v4(sm.pt() + off, pack_bf16x2(s[q8 * 8 + 0], s[q8 * 8 + 1]),
-                           pack_bf16x2(s[q8 * 8 + 2], s[q8 * 8 + 3]),
-                           pack_bf16x2(s[q8 * 8 + 4], s[q8 * 8 + 5]),
-                           pack_bf16x2(s[q8 * 8 + 6], s[q8 * 8 + 7]));
               st_shared_v4(sm.dst() + off, pack_bf16x2(dp[q8 * 8 + 0], dp[q8 * 8 + 1]),
                            pack_bf16x2(dp[q8 * 8 + 2], dp[q8 * 8 + 3]),
                            pack_bf16x2(dp[q8 * 8 + 4], dp[q8 * 8 + 5]),
                            pack_bf16x2(dp[q8 * 8 + 6], dp[q8 * 8 + 7]));
             }
           }
+          tmem_wait_st();
           fence_proxy_async_smem();
           tc_fence_before();
           if (SOFTMAX) {
@@ -532,12 +500,14 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
             const bool dq_first = kb == b0, dq_last = kb == b1 - 1;
             const int qrow = m0 + r;
             if (qrow < t.Lq) {
+              // The scratch row is this thread's alone: kept in L2 (evict-last) between
+              // key blocks and discarded after its last read, so it never reaches HBM.
               float* scr = a.dq_scratch +
                            ((int64_t)blockIdx.x * a.dq_slot_rows + qrow) * C::D + g * HALF_D;
               if (!dq_first) {
 #pragma unroll
                 for (int e = 0; e < HALF_D; e += 4) {
-                  const float4 v = *reinterpret_cast<const float4*>(scr + e);
+                  const float4 v = ld_global_v4_hint(scr + e, pol_keep);
                   dqv[e] += v.x;
                   dqv[e + 1] += v.y;
                   dqv[e + 2] += v.z;
@@ -545,14 +515,18 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
                 }
               }
               if (dq_last) {
+                if (!dq_first && HALF_D * 4 >= 128) {
+#pragma unroll
+                  for (int e = 0; e < HALF_D; e += 32) discard_l2_line(scr + e);
+                }
                 store_row_bf16<HALF_D>(
                     a.dq + ((int64_t)(t.q0 + qrow) * a.H + t.h) * C::D + g * HALF_D, dqv,
                     a.scale);
               } else {
 #pragma unroll
                 for (int e = 0; e < HALF_D; e += 4)
-                  *reinterpret_cast<float4*>(scr + e) =
-                      make_float4(dqv[e], dqv[e + 1], dqv[e + 2], dqv[e + 3]);
+                  st_global_v4_hint(scr + e, make_float4(dqv[e], dqv[e + 1], dqv[e + 2], dqv[e + 3]),
+                                    pol_keep);
               }
             }
           }
@@ -598,20 +572,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ CUtensorMap tdo) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   BSmem<C> sm;
-  {
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t aligned = (raw + 1023u) & ~1023u;
-    sm.base = aligned;
-    sm.ptr = smem_raw + (aligned - raw);
+  sm.base = smem_u32(smem_raw);
+  sm.ptr = smem_raw;
+  if (sm.base & 1023u) {  // swizzled TMA tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_error(a.status, 2, 0x7001);
+    return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(sm.bar(C::B_KVFULL), 1);
     mbar_init(sm.bar(C::B_KVEMPTY), 1);
-    mbar_init(sm.bar(C::B_QFULL), 1);
-    mbar_init(sm.bar(C::B_QEMPTY), 1);
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(sm.bar(C::B_QFULL + i), 1);
+      mbar_init(sm.bar(C::B_QEMPTY + i), 1);
+    }
     mbar_init(sm.bar(C::B_SFULL), 1);
     mbar_init(sm.bar(C::B_PFULL), 256);
     mbar_init(sm.bar(C::B_DQFULL), 1);

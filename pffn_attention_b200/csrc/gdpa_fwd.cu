@@ -25,6 +25,7 @@
 // Every wait is bounded; on expiry the kernel records GDPA_ERR_TIMEOUT in the
 // workspace status, all roles leave their loops, TMEM is freed and the kernel
 // returns.
+#include <algorithm>
 #include <cfloat>
 #include <climits>
 
@@ -48,12 +49,15 @@ struct FwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int NQ = 2;
-  static constexpr int NKV = (D == 128 && BN == 128) ? 2 : 3;
+  // K/V ring: 2 stages of 64 KB for D = 128 with 128-key blocks, else 3-4
+  static constexpr int NKV = (D == 128 && BN == 128) ? 2 : (D * BN <= 64 * 64 ? 4 : 3);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NKV * KV_BYTES;
   static constexpr int OFF_P = OFF_V + NKV * KV_BYTES;
-  static constexpr int OFF_BIAS = OFF_P + P_BYTES;          // float [2][BN]
+  static constexpr int OFF_STAGE = OFF_P + P_BYTES;        // O staging when D > BN
+  static constexpr int STAGE_BYTES = D > BN ? BM * D * 2 : 0;
+  static constexpr int OFF_BIAS = OFF_STAGE + STAGE_BYTES;   // float [2][BN]
   static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;     // uint64 barriers
   // barrier indices
   static constexpr int B_QFULL = 0;
@@ -71,7 +75,7 @@ struct FwdCfg {
   static constexpr int NBARS = B_BEMPTY + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;      // tmem addr, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // + alignment slack
+  static constexpr int SMEM_ALLOC = SMEM_BYTES;  // base is 1024-aligned (checked at entry)
   // TMEM: S buffers at columns [0, BN) and [BN, 2BN); O at [2BN, 2BN + D).
   static constexpr int TMEM_S0 = 0;
   static constexpr int TMEM_O = 2 * BN;
@@ -85,32 +89,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
-struct Unit {
-  int b, h;
-  int q0, Lq, k0, Lk;
-};
-
-__device__ __forceinline__ int unit_index(int round, int cta, int grid) {
-  // boustrophedon over the longest-first list: even rounds left to right,
-  // odd rounds right to left
-  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
-}
-
-__device__ __forceinline__ Unit load_unit(const FwdArgs& a, int u) {
-  Unit t;
-  const int p = u / a.H;
-  t.h = u - p * a.H;
-  t.b = a.order[p];
-  t.q0 = a.q_offsets[t.b];
-  t.Lq = a.q_offsets[t.b + 1] - t.q0;
-  t.k0 = a.kv_offsets[t.b];
-  t.Lk = a.kv_offsets[t.b + 1] - t.k0;
-  if (t.Lq > a.max_q || t.Lk > a.max_kv) {  // the declared bound is violated: skip
-    t.Lq = 0;
-    t.Lk = 0;
-  }
-  return t;
-}
+using Unit = GdpaUnit;
 
 // Key-block range [kb0, kb1) a tile starting at local row m0 may touch.
 template <int BN>
@@ -125,6 +104,16 @@ __device__ __forceinline__ void kv_range(int m0, int Lk, int wl, int wr, int& kb
   }
 }
 
+// K/V stay in shared memory for all query tiles of a unit when there is no
+// band (every tile sees every key block), the unit has more than one tile,
+// and its key blocks fit in the K/V ring.  Otherwise each tile streams the
+// blocks it can see.
+template <class C>
+__device__ __forceinline__ bool kv_resident(const FwdArgs& a, const Unit& t, int& nkb) {
+  nkb = (t.Lk + C::BN - 1) / C::BN;
+  return a.wl < 0 && a.wr < 0 && t.Lq > kBlockM && nkb > 0 && nkb <= C::NKV;
+}
+
 template <class C>
 struct Smem {
   uint32_t base;  // shared address of the 1024-aligned base
@@ -133,6 +122,19 @@ struct Smem {
   __device__ uint32_t k(int s) const { return base + C::OFF_K + s * C::KV_BYTES; }
   __device__ uint32_t v(int s) const { return base + C::OFF_V + s * C::KV_BYTES; }
   __device__ uint32_t p() const { return base + C::OFF_P; }
+  // O staging of warp w, row j (0..31), 16-byte chunk cc, chunks XOR-swizzled by
+  // row.  With D <= BN it lies in the P rows 32w..32w+31 of each 64-key panel
+  // (only warp w writes those); otherwise in a separate region.
+  __device__ uint32_t stage(int w, int j, int cc) const {
+    constexpr int ROWB = C::D * 2;
+    constexpr int SW = (ROWB / 16) >= 8 ? 7 : 3;
+    const uint32_t b = j * ROWB + ((cc ^ (j & SW)) << 4);
+    if constexpr (C::D <= C::BN) {
+      return base + C::OFF_P + (b >> 12) * (kBlockM * 128) + w * 32 * 128 + (b & 4095);
+    } else {
+      return base + C::OFF_STAGE + w * 32 * ROWB + b;
+    }
+  }
   __device__ float* bias(int s) const {
     return reinterpret_cast<float*>(ptr + C::OFF_BIAS) + s * C::BN;
   }
@@ -152,11 +154,27 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   const uint64_t pol_keep = l2_policy_evict_last();
   uint32_t qi = 0, kvi = 0;
   bool dropped = false;
-  for (int round = 0;; ++round) {
-    const int u = unit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const Unit t = load_unit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  Unit t;
+  while (units.next(t)) {
     const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    int nkb;
+    const bool resident = kv_resident<C>(a, t, nkb);
+    auto load_kv = [&](int j) -> bool {
+      const int ks = kvi % C::NKV;
+      if (!mbar_wait(sm.bar(C::B_KVEMPTY + ks), ((kvi / C::NKV) & 1) ^ 1, abort, a.status,
+                     a.timeout_ns, 0x000 + C::B_KVEMPTY + ks))
+        return false;
+      mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + ks), 2 * C::KV_BYTES);
+      for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
+        tma_load_3d(sm.k(ks) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + ks),
+                    pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
+        tma_load_3d(sm.v(ks) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + ks),
+                    pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
+      }
+      ++kvi;
+      return true;
+    };
     for (int mt = 0; mt < ntile; ++mt) {
       const int m0 = mt * kBlockM;
       int kb0, kb1;
@@ -175,20 +193,9 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
                       pnl * C::PANEL_ELEMS, t.h, t.q0 + m0, pol_stream);
       }
       ++qi;
-      for (int j = kb0; j < kb1; ++j) {
-        const int ks = kvi % C::NKV;
-        if (!mbar_wait(sm.bar(C::B_KVEMPTY + ks), ((kvi / C::NKV) & 1) ^ 1, abort, a.status,
-                       a.timeout_ns, 0x000 + C::B_KVEMPTY + ks))
-          return;
-        mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + ks), 2 * C::KV_BYTES);
-        for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
-          tma_load_3d(sm.k(ks) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + ks),
-                      pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
-          tma_load_3d(sm.v(ks) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + ks),
-                      pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
-        }
-        ++kvi;
-      }
+      if (resident && mt > 0) continue;  // the unit's blocks are already in the ring
+      for (int j = kb0; j < kb1; ++j)
+        if (!load_kv(j)) return;
     }
   }
 }
@@ -202,7 +209,7 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   constexpr uint32_t SBO_QK = 8 * C::PANEL_BYTES;
   uint32_t qi = 0, kvi = 0, si = 0, pvi = 0, ti = 0;
 
-  auto issue_pv = [&](int idx, uint32_t kv_index) -> bool {
+  auto issue_pv = [&](int idx, uint32_t kv_index, bool release_kv) -> bool {
     const int ks = kv_index % C::NKV;
     if (!mbar_wait(sm.bar(C::B_PFULL), pvi & 1, abort, a.status, a.timeout_ns,
                    0x100 + C::B_PFULL))
@@ -221,17 +228,19 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
       const uint64_t bdesc = make_smem_desc(vb, C::BN * C::PANEL_BYTES, SBO_QK, C::LAYOUT);
       mma_bf16_ss(tmem + C::TMEM_O, adesc, bdesc, idesc_o, (idx > 0 || kk > 0) ? 1u : 0u);
     }
-    mma_commit(sm.bar(C::B_KVEMPTY + ks));
+    if (release_kv) mma_commit(sm.bar(C::B_KVEMPTY + ks));
     mma_commit(sm.bar(C::B_PVDONE));
     ++pvi;
     return true;
   };
 
-  for (int round = 0;; ++round) {
-    const int u = unit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const Unit t = load_unit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  Unit t;
+  while (units.next(t)) {
     const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
+    int nkb;
+    const bool resident = kv_resident<C>(a, t, nkb);
+    const uint32_t unit_kvi = kvi;  // first ring index of a resident unit
     for (int mt = 0; mt < ntile; ++mt) {
       int kb0, kb1;
       kv_range<C::BN>(mt * kBlockM, t.Lk, a.wl, a.wr, kb0, kb1);
@@ -241,10 +250,12 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
       if (!mbar_wait(sm.bar(C::B_QFULL + qs), (qi / C::NQ) & 1, abort, a.status, a.timeout_ns,
                      0x100 + C::B_QFULL + qs))
         return;
+      if (resident) kvi = unit_kvi;  // every tile walks the same resident stages
       const uint32_t first_kvi = kvi;
       for (int idx = 0; idx < nkv; ++idx) {
         const int ks = kvi % C::NKV;
-        if (!mbar_wait(sm.bar(C::B_KVFULL + ks), (kvi / C::NKV) & 1, abort, a.status,
+        if ((!resident || mt == 0) &&
+            !mbar_wait(sm.bar(C::B_KVFULL + ks), (kvi / C::NKV) & 1, abort, a.status,
                        a.timeout_ns, 0x100 + C::B_KVFULL + ks))
           return;
         const int sb = si & 1;
@@ -266,12 +277,17 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         ++si;
         if (idx == nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + qs));
         ++kvi;
-        if (idx > 0 && !issue_pv(idx - 1, first_kvi + idx - 1)) return;
+        if (idx > 0 && !issue_pv(idx - 1, first_kvi + idx - 1, !resident)) return;
       }
-      if (!issue_pv(nkv - 1, first_kvi + nkv - 1)) return;
+      if (!issue_pv(nkv - 1, first_kvi + nkv - 1, !resident)) return;
       mma_commit(sm.bar(C::B_OFULL));
       ++qi;
       ++ti;
+    }
+    if (resident) {
+      // release the unit's stages once every MMA that reads them has completed
+      for (int idx = 0; idx < nkb; ++idx) mma_commit(sm.bar(C::B_KVEMPTY + (unit_kvi + idx) % C::NKV));
+      kvi = unit_kvi + nkb;
     }
   }
 }
@@ -282,10 +298,9 @@ __device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
   uint32_t bi = 0;
-  for (int round = 0;; ++round) {
-    const int u = unit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const Unit t = load_unit(a, u);
+  UnitStream units(a.info, a.H, a.n_units);
+  Unit t;
+  while (units.next(t)) {
     const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
     for (int mt = 0; mt < ntile; ++mt) {
       int kb0, kb1;
@@ -337,27 +352,20 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
     if (!__all_sync(0xffffffffu, ok_)) return;                                       \
   } while (0)
 
-  for (int round = 0;; ++round) {
-    const int u = unit_index(round, blockIdx.x, gridDim.x);
-    if (u >= a.n_units) break;
-    const Unit t = load_unit(a, u);
-    if (r == 0 && t.Lq == 0) {
-      // distinguish a violated bound from an empty sample
-      const int Lq = a.q_offsets[t.b + 1] - a.q_offsets[t.b];
-      const int Lk = a.kv_offsets[t.b + 1] - a.kv_offsets[t.b];
-      if (Lq > a.max_q || Lk > a.max_kv) record_error(a.status, 6, t.b);
-    }
+  UnitStream units(a.info, a.H, a.n_units);
+  Unit t;
+  while (units.next(t)) {
     const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
     for (int mt = 0; mt < ntile; ++mt) {
       const int m0 = mt * kBlockM;
       const int row = m0 + r;
       const bool row_ok = row < t.Lq;
-      __nv_bfloat16* orow = a.o + ((int64_t)(t.q0 + row) * a.H + t.h) * C::D;
       int kb0, kb1;
       kv_range<C::BN>(m0, t.Lk, a.wl, a.wr, kb0, kb1);
       const int nkv = kb1 - kb0;
       if (nkv <= 0) {
         if (row_ok) {
+          __nv_bfloat16* orow = a.o + ((int64_t)(t.q0 + row) * a.H + t.h) * C::D;
           uint4 z = make_uint4(0, 0, 0, 0);
           for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
           if (SOFTMAX && a.lse) a.lse[(int64_t)t.h * a.total_q + t.q0 + row] = -INFINITY;
@@ -375,28 +383,26 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         const int sb = si & 1;
         PHI_WAIT(C::B_SFULL + sb, (si >> 1) & 1, 0x400 + C::B_SFULL + sb);
         tc_fence_after();
-        float s[C::BN];
+        uint32_t sv[C::BN];  // S row, then P (fp32 bits), in place
 #pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + tl + C::TMEM_S0 + sb * C::BN + c * 32, raw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
-        }
+        for (int c = 0; c < C::BN / 32; ++c)
+          tmem_ld32p(tmem + tl + C::TMEM_S0 + sb * C::BN + c * 32, sv + c * 32);
+        tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(sm.bar(C::B_SEMPTY + sb));
         ++si;
         const float* bias_s = sm.bias(bs);
+        // visible columns of this block: [clo, chi] (no shift of an unbounded side)
+        const int clo = a.wl >= 0 ? lo - kbase : INT_MIN;
+        const int chi = hi - kbase;  // hi <= Lk - 1 always
         // scores, mask
 #pragma unroll
         for (int c = 0; c < C::BN; ++c) {
-          const int key = kbase + c;
-          float x = s[c] * sc;
+          float x = __uint_as_float(sv[c]) * sc;
           if (has_bias) x += bias_s[c];
-          const bool vis = key >= lo && key <= hi;
+          const bool vis = c >= clo && c <= chi;
           if (SOFTMAX) {
-            s[c] = vis ? x : -INFINITY;
+            sv[c] = __float_as_uint(vis ? x : -INFINITY);
           } else {
             float p;
             if (identity) {
@@ -405,7 +411,7 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
               const float hx = 0.5f * x;
               p = fmaf(hx, tanh_approx(hx), hx);  // x * sigmoid(x)
             }
-            s[c] = vis ? p : 0.f;
+            sv[c] = __float_as_uint(vis ? p : 0.f);
           }
         }
         if (has_bias) {
@@ -416,9 +422,13 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         bool need_rescale = false;
         float factor = 1.f;
         if (SOFTMAX) {
-          float bm = -INFINITY;
+          // 4 independent partial maxima, then a tree: no BN-long dependency chain
+          float pm[4];
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c) bm = fmaxf(bm, s[c]);
+          for (int k = 0; k < 4; ++k) pm[k] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < C::BN; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(sv[c]));
+          const float bm = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
           if (idx == 0) {
             m_run = bm;
           } else if (bm > m_run + kRescaleThreshold) {
@@ -428,28 +438,30 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
             m_run = bm;
           }
           const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-          float lsum = 0.f;
+          float ps[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ps[k] = 0.f;
 #pragma unroll
           for (int c = 0; c < C::BN; ++c) {
-            const float p = ex2_approx(s[c] - m_use);
-            s[c] = p;
-            lsum += p;
+            const float p = ex2_approx(__uint_as_float(sv[c]) - m_use);
+            sv[c] = __float_as_uint(p);
+            ps[c & 3] += p;
           }
-          l_run += lsum;
+          l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
         // the previous PV must be done before P is overwritten or O rescaled
         if (idx > 0) PHI_WAIT(C::B_PVDONE, (pvi - 1) & 1, 0x400 + C::B_PVDONE);
         if (SOFTMAX && __any_sync(0xffffffffu, need_rescale)) {
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < C::D / 32; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(tmem + tl + C::TMEM_O + c * 32, raw);
+          for (int c = 0; c < C::D / 16; ++c) {
+            uint32_t raw[16];
+            tmem_ld16(tmem + tl + C::TMEM_O + c * 16, raw);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
+            for (int e = 0; e < 16; ++e)
               raw[e] = __float_as_uint(__uint_as_float(raw[e]) * factor);
-            tmem_st32(tmem + tl + C::TMEM_O + c * 32, raw);
+            tmem_st16(tmem + tl + C::TMEM_O + c * 16, raw);
           }
           tmem_wait_st();
         }
@@ -459,38 +471,54 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
           const int pnl = ch / 8, cir = ch % 8;
           const uint32_t addr =
               sm.p() + pnl * (kBlockM * 128) + r * 128 + ((cir ^ (r & 7)) << 4);
-          st_shared_v4(addr, pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]),
-                       pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]),
-                       pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]),
-                       pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]));
+          const uint32_t* q8 = sv + ch * 8;
+          st_shared_v4(addr, pack_bf16x2(__uint_as_float(q8[0]), __uint_as_float(q8[1])),
+                       pack_bf16x2(__uint_as_float(q8[2]), __uint_as_float(q8[3])),
+                       pack_bf16x2(__uint_as_float(q8[4]), __uint_as_float(q8[5])),
+                       pack_bf16x2(__uint_as_float(q8[6]), __uint_as_float(q8[7])));
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(sm.bar(C::B_PFULL));
         ++pvi;
       }
-      // epilogue: O row from TMEM
+      // epilogue: O row from TMEM -> bf16 -> this warp's staging rows in shared
+      // memory -> whole rows to global memory (coalesced); the staging area of
+      // warp wq lies inside the P rows that only this warp writes
       PHI_WAIT(C::B_OFULL, ti & 1, 0x400 + C::B_OFULL);
       tc_fence_after();
       float inv = 1.f;
       if (SOFTMAX) inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
+#pragma unroll 1  // keeps the epilogue's registers out of the way of the hot loop
       for (int c = 0; c < C::D / 32; ++c) {
         uint32_t raw[32];
         tmem_ld32(tmem + tl + C::TMEM_O + c * 32, raw);
         tmem_wait_ld();
-        if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(raw[e + 0]) * inv, __uint_as_float(raw[e + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(raw[e + 2]) * inv, __uint_as_float(raw[e + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
-          }
+        for (int e = 0; e < 32; e += 8) {
+          const int cc = (c * 32 + e) / 8;  // 16-byte chunk of the row
+          st_shared_v4(sm.stage(wq, lane, cc),
+                       pack_bf16x2(__uint_as_float(raw[e + 0]) * inv, __uint_as_float(raw[e + 1]) * inv),
+                       pack_bf16x2(__uint_as_float(raw[e + 2]) * inv, __uint_as_float(raw[e + 3]) * inv),
+                       pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv),
+                       pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv));
         }
       }
+      __syncwarp();
+      {
+        constexpr int NCH = C::D / 8;  // 16-byte chunks per row
+#pragma unroll 1
+        for (int it = 0; it < NCH; ++it) {
+          const int lin = it * 32 + lane;
+          const int j = lin / NCH, cc = lin % NCH;  // row of this warp, chunk
+          const int grow = m0 + wq * 32 + j;
+          const uint4 v = ld_shared_v4(sm.stage(wq, j, cc));
+          if (grow < t.Lq)
+            *reinterpret_cast<uint4*>(a.o + ((int64_t)(t.q0 + grow) * a.H + t.h) * C::D +
+                                      cc * 8) = v;
+        }
+      }
+      __syncwarp();
       tc_fence_before();
       mbar_arrive(sm.bar(C::B_OEMPTY));
       ++ti;
@@ -508,13 +536,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
   using C = FwdCfg<D, BN>;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
-  {
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t aligned = (raw + 1023u) & ~1023u;
-    sm.base = aligned;
-    sm.ptr = smem_raw + (aligned - raw);
+  sm.base = smem_u32(smem_raw);
+  sm.ptr = smem_raw;
+  if (sm.base & 1023u) {  // swizzled TMA tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_error(a.status, 2, 0x7000);
+    return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -582,32 +610,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int BN, bool SOFTMAX>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                       const CUtensorMap& tv, int grid, cudaStream_t stream) {
+                       const CUtensorMap& tv, int sms, cudaStream_t stream) {
   using C = FwdCfg<D, BN>;
   auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  // persistent: exactly the CTAs that are resident at once
+  const int grid = std::max(1, std::min(a.n_units, per_sm * sms));
   kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int forward_block_n(int D, int phi, int max_kv) {
+int forward_block_n(int D, int phi, int max_kv, int debug_flags) {
   (void)D;
   (void)phi;
-  return max_kv <= 64 ? 64 : 128;
+  return (max_kv <= 64 && !(debug_flags & 2)) ? 64 : 128;
 }
 
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                           const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream) {
   const bool sm = a.phi == 1;
-#define GDPA_FWD_CASE(D_, BN_)                                                  \
-  if (D == D_ && block_n == BN_)                                                \
-    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, grid, stream)           \
-              : launch_one<D_, BN_, false>(a, tq, tk, tv, grid, stream);
+#define GDPA_FWD_CASE(D_, BN_)                                                       \
+  if (D == D_ && block_n == BN_)                                                     \
+    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, sms, stream)                 \
+              : launch_one<D_, BN_, false>(a, tq, tk, tv, sms, stream);
   GDPA_FWD_CASE(32, 64)
   GDPA_FWD_CASE(32, 128)
   GDPA_FWD_CASE(64, 64)

@@ -16,10 +16,11 @@ constexpr int kMaxSortBatch = 16384;  // batch limit of the single-CTA LPT sort
 //   [0, 256)                  DeviceStatus
 //   [256, ...)                order[B]      int32   (LPT sample order)
 //   then                      tile_start[B+1] int32
+//   then                      info[B]       int4    {q0, Lq, k0, Lk} of order[p]
 //   backward only, then       delta[H][total_q] fp32 (softmax rowsum(dO * O))
 //   backward only, then       dQ scratch: grid x slot_rows x D fp32
 struct WorkspaceLayout {
-  size_t order, tile_start, delta, dq_scratch, total;
+  size_t order, tile_start, info, delta, dq_scratch, total;
   int dq_slot_rows;
   int grid;
 };
@@ -28,6 +29,7 @@ struct FwdArgs {
   const int32_t* q_offsets;
   const int32_t* kv_offsets;
   const int32_t* order;
+  const int4* info;         // per sorted sample {q0, Lq, k0, Lk}
   const float* bias;        // [H][total_kv] or nullptr
   __nv_bfloat16* o;         // [total_q][H][D]
   float* lse;               // [H][total_q] or nullptr
@@ -48,6 +50,7 @@ struct BwdArgs {
   const int32_t* q_offsets;
   const int32_t* kv_offsets;
   const int32_t* order;
+  const int4* info;         // per sorted sample {q0, Lq, k0, Lk}
   const float* bias;        // [H][total_kv] or nullptr
   const float* lse;         // [H][total_q] (softmax)
   const float* delta;       // [H][total_q] (softmax)
@@ -72,16 +75,51 @@ struct BwdArgs {
 // Launchers (defined next to their kernels).
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
-                            int32_t* order, DeviceStatus* status, cudaStream_t stream);
+                            int32_t* order, int4* info, int max_q, int max_kv,
+                            DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                           const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream);
-int forward_block_n(int D, int phi, int max_kv);
+int forward_block_n(int D, int phi, int max_kv, int debug_flags);
 cudaError_t launch_bwd_preprocess(const __nv_bfloat16* o, const __nv_bfloat16* dout,
                                   float* delta, int64_t total_q, int H, int D,
                                   cudaStream_t stream);
 cudaError_t launch_backward(const BwdArgs& a, int D, const CUtensorMap& tq,
                             const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, int grid, cudaStream_t stream);
+
+// A CTA's walk over (sample, head) units: unit u = p * H + h of the sorted
+// sample list, boustrophedon over the grid (even rounds left to right, odd
+// rounds right to left).  The next unit's descriptor is loaded one unit ahead
+// so its latency hides behind the current unit.
+struct GdpaUnit {
+  int h, q0, Lq, k0, Lk;
+};
+
+struct UnitStream {
+  const int4* info;
+  int H, n_units, round, u;
+  int4 nxt;
+  __device__ __forceinline__ static int index(int round, int cta, int grid) {
+    return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+  }
+  __device__ __forceinline__ UnitStream(const int4* info_, int H_, int n_units_)
+      : info(info_), H(H_), n_units(n_units_), round(0) {
+    u = index(0, blockIdx.x, gridDim.x);
+    nxt = u < n_units ? __ldg(info + u / H) : make_int4(0, 0, 0, 0);
+  }
+  __device__ __forceinline__ bool next(GdpaUnit& t) {
+    if (u >= n_units) return false;
+    t.h = u % H;
+    t.q0 = nxt.x;
+    t.Lq = nxt.y;
+    t.k0 = nxt.z;
+    t.Lk = nxt.w;
+    ++round;
+    u = index(round, blockIdx.x, gridDim.x);
+    if (u < n_units) nxt = __ldg(info + u / H);
+    return true;
+  }
+};
 
 }  // namespace gdpa

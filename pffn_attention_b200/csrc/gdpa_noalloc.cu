@@ -6,7 +6,8 @@
 // allocator hook, or a serving process that plans all of its memory at start
 // and must not allocate (or ask its caller to allocate) on the request path.
 // For them this entry point runs the same forward kernels with their scratch
-// (the status block, the longest-first sample order and the query-tile prefix)
+// (the status block, the longest-first sample order, the query-tile prefix
+// and the per-sample descriptors)
 // in a fixed array compiled into the library.  It never calls cudaMalloc,
 // cudaFree or any allocating routine.
 //
@@ -23,13 +24,15 @@
 
 namespace {
 
-// status (256 B) + order[16384] (64 KiB) + tile_start[16385] (rounded up to
-// 256 B): enough for the largest batch the library accepts.
+// status (256 B) + order[16384] (64 KiB) + tile_start[16385] + info[16384]
+// (16 B each), each rounded up to 256 B: enough for the largest batch the
+// library accepts.
 constexpr int kNoAllocMaxBatch = 16384;
 constexpr size_t kRound = 256;
 constexpr size_t kNoAllocBytes =
     256 + ((kNoAllocMaxBatch * 4 + kRound - 1) / kRound) * kRound +
-    (((kNoAllocMaxBatch + 1) * 4 + kRound - 1) / kRound) * kRound;
+    (((kNoAllocMaxBatch + 1) * 4 + kRound - 1) / kRound) * kRound +
+    ((kNoAllocMaxBatch * 16 + kRound - 1) / kRound) * kRound;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 

@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kSchedThreads)
     gdpa_schedule_kernel(const int32_t* __restrict__ q_offsets,
                          const int32_t* __restrict__ kv_offsets, int B, int BM, int BN, int wl,
                          int wr, int32_t* __restrict__ tile_start, int32_t* __restrict__ order,
-                         DeviceStatus* status) {
+                         int4* __restrict__ info, int max_q, int max_kv, DeviceStatus* status) {
   extern __shared__ unsigned long long keys[];
   __shared__ long long warp_tot[kSchedThreads / 32];
   const int tid = threadIdx.x;
@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kSchedThreads)
     status->where = 0;
     status->count = 0;
   }
+  __syncthreads();
   int n = 1;
   while (n < B) n <<= 1;
   for (int i = tid; i < n; i += kSchedThreads) {
@@ -88,8 +89,15 @@ __global__ void __launch_bounds__(kSchedThreads)
   for (int p = beg; p < end; ++p) {
     const int b = (int)(keys[p] & 0xFFFFFFFFull);
     order[p] = b;
-    const int Lq = q_offsets[b + 1] - q_offsets[b];
+    const int q0 = q_offsets[b], Lq = q_offsets[b + 1] - q0;
+    const int k0 = kv_offsets[b], Lk = kv_offsets[b + 1] - k0;
     local += (Lq + BM - 1) / BM;
+    if (info) {
+      // a sample longer than the declared bound is reported and skipped
+      const bool bad = Lq > max_q || Lk > max_kv;
+      if (bad && status) record_error(status, 6, b);
+      info[p] = make_int4(q0, bad ? 0 : Lq, k0, bad ? 0 : Lk);
+    }
   }
   // block-wide exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5;
@@ -125,7 +133,8 @@ __global__ void __launch_bounds__(kSchedThreads)
 
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
-                            int32_t* order, DeviceStatus* status, cudaStream_t stream) {
+                            int32_t* order, int4* info, int max_q, int max_kv,
+                            DeviceStatus* status, cudaStream_t stream) {
   int n = 1;
   while (n < B) n <<= 1;
   const size_t smem = (size_t)n * sizeof(unsigned long long);
@@ -135,7 +144,7 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
   if (e != cudaSuccess) return e;
   gdpa_schedule_kernel<<<1, kSchedThreads, smem, stream>>>(q_offsets, kv_offsets, B, block_m,
                                                            block_n, wl, wr, tile_start, order,
-                                                           status);
+                                                           info, max_q, max_kv, status);
   return cudaGetLastError();
 }
 

@@ -89,5 +89,7 @@ def test_workspace_size_grows_with_problem(lib):
 def test_tile_shape_query(lib):
     rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64))
     assert (rc, bm, bn) == (0, 128, 64)
-    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=65))
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=2000))
+    assert (rc, bm, bn) == (0, 128, 128)
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64, debug_flags=2))
     assert (rc, bm, bn) == (0, 128, 128)

@@ -140,3 +140,25 @@ def _sampled_full(gdpa, cfg, n_samples=6):
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_full_size_sampled(cuda_lib, cfg):
     _sampled_full(cuda_lib, cfg)
+
+
+# -------------------------------------------------- 128-key blocks where 64 would be chosen
+@pytest.mark.parametrize("cfg,B", [(1, None), (2, 6)])
+def test_workload_parity_128_key_variant(cuda_lib, cfg, B):
+    w = make_workload(cfg, B=B, with_dout=False)
+    dev = torch.device("cuda")
+    p = cuda_lib.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
+                             window=(w.window_left, w.window_right), bias_kind=w.bias_kind,
+                             max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv, debug_flags=2)
+    rc, bm, bn = cuda_lib.gdpa_forward_tile_shape(p)
+    assert (rc, bm, bn) == (0, 128, 128)
+    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+    ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
+    bias = w.bias.to(dev) if w.bias is not None else None
+    o, lse, ws = cuda_lib.forward(w.q.to(dev), w.k.to(dev), w.v.to(dev), qo, ko, bias=bias,
+                                  params=p)
+    assert cuda_lib.device_status(ws) == 0
+    ro, rlse = oracle.forward_workload(w)
+    compare("O", o, ro)
+    if w.phi == PHI_SOFTMAX:
+        compare_lse(lse, rlse)
