@@ -498,36 +498,67 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
             int b0, b1;
             bwd_kv_range(m0, t.Lk, a.wl, a.wr, b0, b1);
             const bool dq_first = kb == b0, dq_last = kb == b1 - 1;
-            const int qrow = m0 + r;
-            if (qrow < t.Lq) {
-              // The scratch row is this thread's alone: kept in L2 (evict-last) between
-              // key blocks and discarded after its last read, so it never reaches HBM.
-              float* scr = a.dq_scratch +
-                           ((int64_t)blockIdx.x * a.dq_slot_rows + qrow) * C::D + g * HALF_D;
+            if (!(dq_first && dq_last)) {
+              // Partial dQ across key blocks, in this CTA's scratch slot laid out
+              // thread-major ([tile][half g][16-byte chunk][row]) so each warp access
+              // is 512 contiguous bytes.  Only this thread reads what it wrote; the
+              // slot stays in L2 (evict-last) and is discarded after its last read.
+              constexpr int NCH4 = HALF_D / 4;
+              float4* scr4 = reinterpret_cast<float4*>(a.dq_scratch) +
+                             ((((int64_t)blockIdx.x * (a.dq_slot_rows / kBlockM) + mt) * 2 + g) *
+                              NCH4) * kBlockM + r;
               if (!dq_first) {
 #pragma unroll
-                for (int e = 0; e < HALF_D; e += 4) {
-                  const float4 v = ld_global_v4_hint(scr + e, pol_keep);
-                  dqv[e] += v.x;
-                  dqv[e + 1] += v.y;
-                  dqv[e + 2] += v.z;
-                  dqv[e + 3] += v.w;
+                for (int c = 0; c < NCH4; ++c) {
+                  const float4 v = ld_global_v4_hint(reinterpret_cast<const float*>(scr4 + c * kBlockM),
+                                                     pol_keep);
+                  dqv[4 * c] += v.x;
+                  dqv[4 * c + 1] += v.y;
+                  dqv[4 * c + 2] += v.z;
+                  dqv[4 * c + 3] += v.w;
                 }
               }
-              if (dq_last) {
-                if (!dq_first && HALF_D * 4 >= 128) {
+              if (!dq_last) {
 #pragma unroll
-                  for (int e = 0; e < HALF_D; e += 32) discard_l2_line(scr + e);
-                }
-                store_row_bf16<HALF_D>(
-                    a.dq + ((int64_t)(t.q0 + qrow) * a.H + t.h) * C::D + g * HALF_D, dqv,
-                    a.scale);
-              } else {
-#pragma unroll
-                for (int e = 0; e < HALF_D; e += 4)
-                  st_global_v4_hint(scr + e, make_float4(dqv[e], dqv[e + 1], dqv[e + 2], dqv[e + 3]),
+                for (int c = 0; c < NCH4; ++c)
+                  st_global_v4_hint(reinterpret_cast<float*>(scr4 + c * kBlockM),
+                                    make_float4(dqv[4 * c], dqv[4 * c + 1], dqv[4 * c + 2],
+                                                dqv[4 * c + 3]),
                                     pol_keep);
+              } else {
+                __syncwarp();  // every lane of the warp has its values: drop the lines
+                if ((lane & 7) == 0) {
+#pragma unroll
+                  for (int c = 0; c < NCH4; ++c) discard_l2_line(scr4 + c * kBlockM);
+                }
               }
+            }
+            if (dq_last) {
+              // final dQ rows (bf16): staged in this warp's own dS^T rows (free once
+              // the dQ MMA completed), then written as whole row segments
+              constexpr int RB = HALF_D * 2;              // bytes of this half row
+              constexpr int CPR = RB / 16;                // 16-byte chunks per half row
+              constexpr int SWM = (CPR >= 8 ? 8 : CPR) - 1;
+              const uint32_t stage = sm.dst() + g * (128 * 128) + wq * 32 * 128;
+#pragma unroll
+              for (int c = 0; c < CPR; ++c)
+                st_shared_v4(stage + lane * 128 + ((c ^ (lane & SWM)) << 4),
+                             pack_bf16x2(dqv[8 * c + 0] * a.scale, dqv[8 * c + 1] * a.scale),
+                             pack_bf16x2(dqv[8 * c + 2] * a.scale, dqv[8 * c + 3] * a.scale),
+                             pack_bf16x2(dqv[8 * c + 4] * a.scale, dqv[8 * c + 5] * a.scale),
+                             pack_bf16x2(dqv[8 * c + 6] * a.scale, dqv[8 * c + 7] * a.scale));
+              __syncwarp();
+#pragma unroll 1
+              for (int it = 0; it < CPR; ++it) {
+                const int lin = it * 32 + lane;
+                const int j = lin / CPR, c = lin % CPR;   // row of this warp, chunk
+                const uint4 v = ld_shared_v4(stage + j * 128 + ((c ^ (j & SWM)) << 4));
+                const int grow = m0 + wq * 32 + j;
+                if (grow < t.Lq)
+                  *reinterpret_cast<uint4*>(a.dq + ((int64_t)(t.q0 + grow) * a.H + t.h) * C::D +
+                                            g * HALF_D + c * 8) = v;
+              }
+              __syncwarp();
             }
           }
           if (last) {

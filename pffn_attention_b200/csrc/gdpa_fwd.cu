@@ -201,6 +201,9 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
 }
 
 // ------------------------------------------------------------------ MMA issuer
+// The issuer keeps one PV behind: S of the next key block (of this tile, or of
+// the next tile or unit) is issued before the PV of the current one, so the
+// phi warpgroup finds its next S ready when it finishes a block or a tile.
 template <class C>
 __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   volatile int* abort = sm.abort_flag();
@@ -209,13 +212,23 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   constexpr uint32_t SBO_QK = 8 * C::PANEL_BYTES;
   uint32_t qi = 0, kvi = 0, si = 0, pvi = 0, ti = 0;
 
-  auto issue_pv = [&](int idx, uint32_t kv_index, bool release_kv) -> bool {
-    const int ks = kv_index % C::NKV;
+  struct PendingPV {
+    bool valid;
+    bool first;         // first key block of its tile (overwrites O)
+    bool last;          // last key block of its tile (O complete afterwards)
+    int ks;             // K/V stage holding V
+    bool release_kv;    // streamed block: free its stage after this PV
+    uint32_t unit_kvi;  // resident unit ending with this PV: free its stages
+    int unit_nkb;       //   (0 when not)
+  } pend = {false, false, false, 0, false, 0u, 0};
+
+  auto issue_pending = [&]() -> bool {
+    if (!pend.valid) return true;
     if (!mbar_wait(sm.bar(C::B_PFULL), pvi & 1, abort, a.status, a.timeout_ns,
                    0x100 + C::B_PFULL))
       return false;
-    if (idx == 0 && !mbar_wait(sm.bar(C::B_OEMPTY), (ti & 1) ^ 1, abort, a.status, a.timeout_ns,
-                               0x100 + C::B_OEMPTY))
+    if (pend.first && !mbar_wait(sm.bar(C::B_OEMPTY), (ti & 1) ^ 1, abort, a.status,
+                                 a.timeout_ns, 0x100 + C::B_OEMPTY))
       return false;
     tc_fence_after();
 #pragma unroll
@@ -224,13 +237,20 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
       const uint32_t pa = sm.p() + (kk * 16 / 64) * (kBlockM * 128) + (kk * 16 % 64) * 2;
       const uint64_t adesc = make_smem_desc(pa, 16, 1024, LAYOUT_SW128);
       // B = V [BN keys x D], N (= D) contiguous: MN-major; 16 keys per step
-      const uint32_t vb = sm.v(ks) + kk * 16 * C::PANEL_BYTES;
+      const uint32_t vb = sm.v(pend.ks) + kk * 16 * C::PANEL_BYTES;
       const uint64_t bdesc = make_smem_desc(vb, C::BN * C::PANEL_BYTES, SBO_QK, C::LAYOUT);
-      mma_bf16_ss(tmem + C::TMEM_O, adesc, bdesc, idesc_o, (idx > 0 || kk > 0) ? 1u : 0u);
+      mma_bf16_ss(tmem + C::TMEM_O, adesc, bdesc, idesc_o, (!pend.first || kk > 0) ? 1u : 0u);
     }
-    if (release_kv) mma_commit(sm.bar(C::B_KVEMPTY + ks));
+    if (pend.release_kv) mma_commit(sm.bar(C::B_KVEMPTY + pend.ks));
     mma_commit(sm.bar(C::B_PVDONE));
     ++pvi;
+    if (pend.last) {
+      mma_commit(sm.bar(C::B_OFULL));
+      ++ti;
+    }
+    for (int idx = 0; idx < pend.unit_nkb; ++idx)
+      mma_commit(sm.bar(C::B_KVEMPTY + (pend.unit_kvi + idx) % C::NKV));
+    pend.valid = false;
     return true;
   };
 
@@ -251,9 +271,11 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
                      0x100 + C::B_QFULL + qs))
         return;
       if (resident) kvi = unit_kvi;  // every tile walks the same resident stages
-      const uint32_t first_kvi = kvi;
       for (int idx = 0; idx < nkv; ++idx) {
         const int ks = kvi % C::NKV;
+        // a resident unit frees its stages with its last PV; the next unit's
+        // first load may need them, so that PV is not deferred past this wait
+        if (pend.valid && pend.unit_nkb > 0 && !issue_pending()) return;
         if ((!resident || mt == 0) &&
             !mbar_wait(sm.bar(C::B_KVFULL + ks), (kvi / C::NKV) & 1, abort, a.status,
                        a.timeout_ns, 0x100 + C::B_KVFULL + ks))
@@ -275,21 +297,21 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         }
         mma_commit(sm.bar(C::B_SFULL + sb));
         ++si;
-        if (idx == nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + qs));
+        if (idx == nkv - 1) {
+          mma_commit(sm.bar(C::B_QEMPTY + qs));
+          ++qi;
+        }
         ++kvi;
-        if (idx > 0 && !issue_pv(idx - 1, first_kvi + idx - 1, !resident)) return;
+        // the previous block's PV, now that this block's S is on its way
+        if (!issue_pending()) return;
+        const bool last_of_unit = resident && mt == ntile - 1 && idx == nkv - 1;
+        pend = {true, idx == 0, idx == nkv - 1, ks, !resident,
+                last_of_unit ? unit_kvi : 0u, last_of_unit ? nkb : 0};
       }
-      if (!issue_pv(nkv - 1, first_kvi + nkv - 1, !resident)) return;
-      mma_commit(sm.bar(C::B_OFULL));
-      ++qi;
-      ++ti;
     }
-    if (resident) {
-      // release the unit's stages once every MMA that reads them has completed
-      for (int idx = 0; idx < nkb; ++idx) mma_commit(sm.bar(C::B_KVEMPTY + (unit_kvi + idx) % C::NKV));
-      kvi = unit_kvi + nkb;
-    }
+    if (resident) kvi = unit_kvi + nkb;
   }
+  issue_pending();
 }
 
 // ------------------------------------------------------------------ bias warp
@@ -391,27 +413,54 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         tc_fence_before();
         mbar_arrive(sm.bar(C::B_SEMPTY + sb));
         ++si;
-        const float* bias_s = sm.bias(bs);
+        const float2* bias2 = reinterpret_cast<const float2*>(sm.bias(bs));
         // visible columns of this block: [clo, chi] (no shift of an unbounded side)
         const int clo = a.wl >= 0 ? lo - kbase : INT_MIN;
         const int chi = hi - kbase;  // hi <= Lk - 1 always
-        // scores, mask
+        const bool full = clo <= 0 && chi >= C::BN - 1;
+        const uint64_t sc2 = f2_pack(sc, sc);
+        // scores x = scale * s + beta, two columns per packed instruction
 #pragma unroll
-        for (int c = 0; c < C::BN; ++c) {
-          float x = __uint_as_float(sv[c]) * sc;
-          if (has_bias) x += bias_s[c];
-          const bool vis = c >= clo && c <= chi;
-          if (SOFTMAX) {
-            sv[c] = __float_as_uint(vis ? x : -INFINITY);
+        for (int c = 0; c < C::BN; c += 2) {
+          uint64_t x2 = f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+          if (has_bias) {
+            const float2 b = bias2[c >> 1];
+            x2 = f2_fma(x2, sc2, f2_pack(b.x, b.y));
           } else {
-            float p;
-            if (identity) {
-              p = x;
-            } else {
-              const float hx = 0.5f * x;
-              p = fmaf(hx, tanh_approx(hx), hx);  // x * sigmoid(x)
+            x2 = f2_mul(x2, sc2);
+          }
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          sv[c] = __float_as_uint(x0);
+          sv[c + 1] = __float_as_uint(x1);
+        }
+        if (!full) {  // band edges and the ragged last key block
+          const float fill = SOFTMAX ? -INFINITY : 0.f;
+#pragma unroll
+          for (int c = 0; c < C::BN; ++c)
+            if (c < clo || c > chi) sv[c] = __float_as_uint(fill);
+        }
+        if (!SOFTMAX) {
+          if (!identity) {
+            const uint64_t half2 = f2_pack(0.5f, 0.5f);
+#pragma unroll
+            for (int c = 0; c < C::BN; c += 2) {
+              // silu(x) = h + h tanh(h), h = x / 2
+              const uint64_t h2 =
+                  f2_mul(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), half2);
+              float h0, h1;
+              f2_unpack(h2, h0, h1);
+              const uint64_t p2 = f2_fma(h2, f2_pack(tanh_approx(h0), tanh_approx(h1)), h2);
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
+              sv[c] = __float_as_uint(p0);
+              sv[c + 1] = __float_as_uint(p1);
             }
-            sv[c] = __float_as_uint(vis ? p : 0.f);
+            if (!full) {  // silu(0) = 0 already; keep masked columns exactly zero
+#pragma unroll
+              for (int c = 0; c < C::BN; ++c)
+                if (c < clo || c > chi) sv[c] = 0u;
+            }
           }
         }
         if (has_bias) {
@@ -422,13 +471,15 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         bool need_rescale = false;
         float factor = 1.f;
         if (SOFTMAX) {
-          // 4 independent partial maxima, then a tree: no BN-long dependency chain
+          // 4 independent partial maxima over 3-input max: no BN-long chain
           float pm[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) pm[k] = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(sv[c]));
-          const float bm = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+          for (int c = 0; c < C::BN; c += 2)
+            pm[(c >> 1) & 3] = fmax3(pm[(c >> 1) & 3], __uint_as_float(sv[c]),
+                                     __uint_as_float(sv[c + 1]));
+          const float bm = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
           if (idx == 0) {
             m_run = bm;
           } else if (bm > m_run + kRescaleThreshold) {
@@ -438,16 +489,23 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
             m_run = bm;
           }
           const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-          float ps[4];
+          const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
+          uint64_t ps2[2] = {0ull, 0ull};  // packed partial sums
 #pragma unroll
-          for (int k = 0; k < 4; ++k) ps[k] = 0.f;
-#pragma unroll
-          for (int c = 0; c < C::BN; ++c) {
-            const float p = ex2_approx(__uint_as_float(sv[c]) - m_use);
-            sv[c] = __float_as_uint(p);
-            ps[c & 3] += p;
+          for (int c = 0; c < C::BN; c += 2) {
+            const uint64_t d2 =
+                f2_add(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), neg_m2);
+            float d0, d1;
+            f2_unpack(d2, d0, d1);
+            const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
+            sv[c] = __float_as_uint(p0);
+            sv[c + 1] = __float_as_uint(p1);
+            ps2[(c >> 1) & 1] = f2_add(ps2[(c >> 1) & 1], f2_pack(p0, p1));
           }
-          l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+          float s0, s1, s2, s3;
+          f2_unpack(ps2[0], s0, s1);
+          f2_unpack(ps2[1], s2, s3);
+          l_run += (s0 + s1) + (s2 + s3);
         }
         // the previous PV must be done before P is overwritten or O rescaled
         if (idx > 0) PHI_WAIT(C::B_PVDONE, (pvi - 1) & 1, 0x400 + C::B_PVDONE);
