@@ -81,6 +81,35 @@ def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
     return fwd, bwd
 
 
+KERNEL_SOURCES = {
+    "gdpa_backward": ["gdpa_bwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_forward": ["gdpa_fwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "pffn_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, n_samples: int):
+    """DRAM bytes per launch from the committed ncu capture (profiles/
+    traffic.json), scaled by samples; None when the kernel's sources changed
+    since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return d["dram_bytes"] / d["samples"] * n_samples
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -89,6 +118,28 @@ def load_peaks():
         return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, \
             "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- ranks
+def rank_seed(cfg: int, rank: int) -> int:
+    """Each rank draws its own batch: independent samples, no shared data."""
+    return cfg + 1000 * rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The job's time is the slowest rank's (MAX all-reduce of one number)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank's useful FLOPs over the slowest time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------------- clocks
@@ -154,7 +205,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     cfg = WORKLOADS[args.workload]
     training = cfg == 5
     # each rank owns an independent batch of the same distribution
-    w = make_workload(cfg, B=args.batch, device=dev, seed=cfg + 1000 * rank, with_dout=training)
+    w = make_workload(cfg, B=args.batch, device=dev, seed=rank_seed(cfg, rank),
+                      with_dout=training)
     qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
     ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
     p = gdpa.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
@@ -220,15 +272,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if training else 0.0
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
 
     f_fwd, f_bwd = useful_flops(w, training)
     b_fwd, b_bwd = algorithmic_bytes(w, training)
-    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(f_fwd + f_bwd, world, ms_per_step)
     peaks, peak_src = load_peaks()
 
     # dominant call: the backward in a training step, else the forward
@@ -237,9 +286,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     else:
         dom_name, dom_ms, dom_bytes, dom_flops = "gdpa_forward", fwd_ms, b_fwd, f_fwd
     achieved_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = measured_traffic(dom_name, w.B)
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-                "traffic": None, "kernel": dom_name, "peak_source": peak_src,
+                "traffic": None if traffic is None else round(traffic / 1e9, 3),
+                "traffic_unit": "GB per launch", "algorithmic": round(dom_bytes / 1e9, 3),
+                "kernel": dom_name, "peak_source": peak_src,
                 "tensor_tflops": round(dom_flops / (dom_ms * 1e-3) / 1e12, 1),
                 "tensor_frac": round(dom_flops / (dom_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
 
@@ -338,14 +390,9 @@ def run_e2e(args, w, p, qo, ko, training, dev, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
     f_fwd, f_bwd = useful_flops(w, training)
-    return {"value": round((f_fwd + f_bwd) * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    return {"value": round(job_tflops(f_fwd + f_bwd, world, ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
 
@@ -365,7 +412,7 @@ def time_oracle(sub, training: bool) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(args, w, training: bool, target_s: float = 12.0) -> dict:
+def cpu_baseline(args, w, training: bool, target_s: float = 16.0) -> dict:
     """The fp64 oracle, as it stands, on a bounded sample of the same workload."""
     import oracle
     cfg = WORKLOADS[args.workload]
