@@ -88,8 +88,7 @@ typedef struct {
   int bias_kind;      /* GDPA_BIAS_*: none, beta = bias, or beta = log sigmoid(bias) */
   int debug_flags;    /* 0 in normal use.  Bit 0 drops one producer arrival so that
                          the bounded-wait path can be tested (returns TIMEOUT);
-                         bit 1 makes the forward use 128-key blocks even when
-                         every sample has at most 64 keys (tests both tile shapes) */
+                         other bits are reserved and ignored */
   int wait_timeout_us;/* bound on any single in-kernel wait; 0 = 2000000 (2 s) */
 } gdpa_params_t;
 

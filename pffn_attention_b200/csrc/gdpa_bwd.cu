@@ -35,6 +35,11 @@ namespace gdpa {
 namespace {
 
 constexpr int kBwdThreads = 384;
+constexpr int kRegsLaunch = 168;   // 65536 / 384 rounded down to a multiple of 8
+constexpr int kRegsControl = 96;   // warpgroup 0
+constexpr int kRegsPhi = 200;      // warpgroups 1 and 2
+static_assert(128 * kRegsControl + 256 * kRegsPhi <= kBwdThreads * kRegsLaunch,
+              "register split exceeds the launch's registers");
 constexpr float kLog2eB = 1.4426950408889634f;
 
 template <int D_>
@@ -160,6 +165,21 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
                           p * C::PANEL_ELEMS, t.h, t.k0 + kb * C::BN, pol_keep);
             }
             ++kvi;
+            // warm L2 with the key block that follows (this unit's next block or
+            // the next unit's first), whose load waits for this block's release
+            const int nkb = (t.Lk + C::BN - 1) / C::BN;
+            BUnit nt = t;
+            int nb = kb + 1;
+            if (nb >= nkb) {
+              nb = 0;
+              if (!units.peek(nt)) nt.Lk = 0;
+            }
+            if (nb * C::BN < nt.Lk) {
+              for (int p = 0; p < C::NPANEL; ++p) {
+                tma_prefetch_l2_3d(tk, p * C::PANEL_ELEMS, nt.h, nt.k0 + nb * C::BN, pol_keep);
+                tma_prefetch_l2_3d(tv, p * C::PANEL_ELEMS, nt.h, nt.k0 + nb * C::BN, pol_keep);
+              }
+            }
           }
           const int qs = qi % C::NQ;
           if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((qi / C::NQ) & 1) ^ 1, abort, a.status,
@@ -486,77 +506,91 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
           }
           ++ri;
           mbar_arrive(sm.bar(C::B_PFULL));
-          // dQ of this pair: thread = query row, columns [g*D/2, (g+1)*D/2)
+          // dQ of this pair: thread = query row, columns [g*D/2, (g+1)*D/2).
+          // Partial dQ across key blocks lives in this CTA's scratch slot laid out
+          // thread-major ([tile][half g][16-byte chunk][row]) so each warp access
+          // is 512 contiguous bytes.  Only this thread reads what it wrote; the
+          // slot stays in L2 (evict-last) and is discarded after its last read.
+          // The earlier blocks' partial is fetched now, while the dV, dK and dQ
+          // MMAs run, so its latency is off the path.
+          int b0, b1;
+          bwd_kv_range(m0, t.Lk, a.wl, a.wr, b0, b1);
+          const bool dq_first = kb == b0, dq_last = kb == b1 - 1;
+          constexpr int NCH4 = HALF_D / 4;
+          float4* scr4 = reinterpret_cast<float4*>(a.dq_scratch) +
+                         ((((int64_t)blockIdx.x * (a.dq_slot_rows / kBlockM) + mt) * 2 + g) *
+                          NCH4) * kBlockM + r;
+          float4 part[NCH4];
+          if (!dq_first) {
+#pragma unroll
+            for (int c = 0; c < NCH4; ++c)
+              part[c] = ld_global_v4_hint(reinterpret_cast<const float*>(scr4 + c * kBlockM),
+                                          pol_keep);
+          }
           BWD_WAIT(C::B_DQFULL, dqi & 1, 0x1400 + C::B_DQFULL);
           ++dqi;
           tc_fence_after();
-          float dqv[HALF_D];
-          tmem_row<HALF_D>(tmem + tl + C::T_S + g * HALF_D, dqv);
-          tc_fence_before();
-          mbar_arrive(sm.bar(C::B_DQEMPTY));
           {
-            int b0, b1;
-            bwd_kv_range(m0, t.Lk, a.wl, a.wr, b0, b1);
-            const bool dq_first = kb == b0, dq_last = kb == b1 - 1;
-            if (!(dq_first && dq_last)) {
-              // Partial dQ across key blocks, in this CTA's scratch slot laid out
-              // thread-major ([tile][half g][16-byte chunk][row]) so each warp access
-              // is 512 contiguous bytes.  Only this thread reads what it wrote; the
-              // slot stays in L2 (evict-last) and is discarded after its last read.
-              constexpr int NCH4 = HALF_D / 4;
-              float4* scr4 = reinterpret_cast<float4*>(a.dq_scratch) +
-                             ((((int64_t)blockIdx.x * (a.dq_slot_rows / kBlockM) + mt) * 2 + g) *
-                              NCH4) * kBlockM + r;
+            // 32 columns (8 float4 of the partial) at a time; the last chunk's TMEM
+            // read releases the dQ columns.  The final rows (bf16) are staged in
+            // this warp's own dS^T rows (free once the dQ MMA completed), then
+            // written as whole row segments.
+            constexpr int CW = HALF_D < 32 ? HALF_D : 32;
+            constexpr int NCHUNK = HALF_D / CW;
+            constexpr int CPR = HALF_D * 2 / 16;          // 16-byte chunks per half row
+            constexpr int SWM = (CPR >= 8 ? 8 : CPR) - 1;
+            const uint32_t stage = sm.dst() + g * (128 * 128) + wq * 32 * 128;
+#pragma unroll
+            for (int ck = 0; ck < NCHUNK; ++ck) {
+              float v[CW];
+              tmem_row<CW>(tmem + tl + C::T_S + g * HALF_D + ck * CW, v);
+              if (ck == NCHUNK - 1) {
+                tc_fence_before();
+                mbar_arrive(sm.bar(C::B_DQEMPTY));
+              }
               if (!dq_first) {
 #pragma unroll
-                for (int c = 0; c < NCH4; ++c) {
-                  const float4 v = ld_global_v4_hint(reinterpret_cast<const float*>(scr4 + c * kBlockM),
-                                                     pol_keep);
-                  dqv[4 * c] += v.x;
-                  dqv[4 * c + 1] += v.y;
-                  dqv[4 * c + 2] += v.z;
-                  dqv[4 * c + 3] += v.w;
+                for (int c = 0; c < CW / 4; ++c) {
+                  const float4 pc = part[ck * (CW / 4) + c];
+                  v[4 * c] += pc.x;
+                  v[4 * c + 1] += pc.y;
+                  v[4 * c + 2] += pc.z;
+                  v[4 * c + 3] += pc.w;
                 }
               }
               if (!dq_last) {
 #pragma unroll
-                for (int c = 0; c < NCH4; ++c)
-                  st_global_v4_hint(reinterpret_cast<float*>(scr4 + c * kBlockM),
-                                    make_float4(dqv[4 * c], dqv[4 * c + 1], dqv[4 * c + 2],
-                                                dqv[4 * c + 3]),
+                for (int c = 0; c < CW / 4; ++c)
+                  st_global_v4_hint(reinterpret_cast<float*>(scr4 + (ck * (CW / 4) + c) * kBlockM),
+                                    make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]),
                                     pol_keep);
               } else {
-                __syncwarp();  // every lane of the warp has its values: drop the lines
-                if ((lane & 7) == 0) {
 #pragma unroll
-                  for (int c = 0; c < NCH4; ++c) discard_l2_line(scr4 + c * kBlockM);
+                for (int c8 = 0; c8 < CW / 8; ++c8) {
+                  const int c = ck * (CW / 8) + c8;
+                  st_shared_v4(stage + lane * 128 + ((c ^ (lane & SWM)) << 4),
+                               pack_bf16x2(v[8 * c8 + 0] * a.scale, v[8 * c8 + 1] * a.scale),
+                               pack_bf16x2(v[8 * c8 + 2] * a.scale, v[8 * c8 + 3] * a.scale),
+                               pack_bf16x2(v[8 * c8 + 4] * a.scale, v[8 * c8 + 5] * a.scale),
+                               pack_bf16x2(v[8 * c8 + 6] * a.scale, v[8 * c8 + 7] * a.scale));
                 }
               }
             }
             if (dq_last) {
-              // final dQ rows (bf16): staged in this warp's own dS^T rows (free once
-              // the dQ MMA completed), then written as whole row segments
-              constexpr int RB = HALF_D * 2;              // bytes of this half row
-              constexpr int CPR = RB / 16;                // 16-byte chunks per half row
-              constexpr int SWM = (CPR >= 8 ? 8 : CPR) - 1;
-              const uint32_t stage = sm.dst() + g * (128 * 128) + wq * 32 * 128;
+              __syncwarp();  // the warp's rows are staged and its partial was read
+              if (!dq_first && (lane & 7) == 0) {
 #pragma unroll
-              for (int c = 0; c < CPR; ++c)
-                st_shared_v4(stage + lane * 128 + ((c ^ (lane & SWM)) << 4),
-                             pack_bf16x2(dqv[8 * c + 0] * a.scale, dqv[8 * c + 1] * a.scale),
-                             pack_bf16x2(dqv[8 * c + 2] * a.scale, dqv[8 * c + 3] * a.scale),
-                             pack_bf16x2(dqv[8 * c + 4] * a.scale, dqv[8 * c + 5] * a.scale),
-                             pack_bf16x2(dqv[8 * c + 6] * a.scale, dqv[8 * c + 7] * a.scale));
-              __syncwarp();
+                for (int c = 0; c < NCH4; ++c) discard_l2_line(scr4 + c * kBlockM);
+              }
 #pragma unroll 1
               for (int it = 0; it < CPR; ++it) {
                 const int lin = it * 32 + lane;
-                const int j = lin / CPR, c = lin % CPR;   // row of this warp, chunk
-                const uint4 v = ld_shared_v4(stage + j * 128 + ((c ^ (j & SWM)) << 4));
-                const int grow = m0 + wq * 32 + j;
+                const int jr = lin / CPR, c = lin % CPR;   // row of this warp, chunk
+                const uint4 vv = ld_shared_v4(stage + jr * 128 + ((c ^ (jr & SWM)) << 4));
+                const int grow = m0 + wq * 32 + jr;
                 if (grow < t.Lq)
                   *reinterpret_cast<uint4*>(a.dq + ((int64_t)(t.q0 + grow) * a.H + t.h) * C::D +
-                                            g * HALF_D + c * 8) = v;
+                                            g * HALF_D + c * 8) = vv;
               }
               __syncwarp();
             }
@@ -647,13 +681,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  if (warp == 0) {
-    if (lane == 0) bwd_producer<C>(a, sm, &tq, &tk, &tv, &tdo);
-  } else if (warp == 1) {
-    if (lane == 0) bwd_mma<C>(a, sm, tmem);
-  } else if (warp == 3) {
-    if (PHI == 1) bwd_rows<C>(a, sm);
-  } else if (warp >= 4) {
+  // Registers: the launch gives 384 x 168; warpgroup 0 (producer, MMA issuer,
+  // allocator, row loader) needs few, the two phi warpgroups take the rest:
+  // 128 x 96 + 256 x 200 = 63488 <= 64512.  Each budget is set inside its own
+  // branch so the compiler allocates each role's code against it.
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      if (lane == 0) bwd_producer<C>(a, sm, &tq, &tk, &tv, &tdo);
+    } else if (warp == 1) {
+      if (lane == 0) bwd_mma<C>(a, sm, tmem);
+    } else if (warp == 3) {
+      if (PHI == 1) bwd_rows<C>(a, sm);
+    }
+  } else {
+    setmaxnreg_inc<kRegsPhi>();
     bwd_phi<C, PHI>(a, sm, tmem);
   }
   __syncwarp();
@@ -713,8 +755,14 @@ cudaError_t launch_bwd_one(const BwdArgs& a, const CUtensorMap& tq, const CUtens
                            cudaStream_t stream) {
   using C = BwdCfg<D>;
   auto kern = gdpa_bwd_kernel<D, PHI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_ALLOC);
+  // The phi warpgroups raise their register budget with setmaxnreg, which
+  // waits until the block's launch registers cover it: never launch a build
+  // whose per-thread count would leave that wait unsatisfiable.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kBwdThreads < 128 * kRegsControl + 256 * kRegsPhi) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   kern<<<grid, kBwdThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv, tdo);
   return cudaGetLastError();

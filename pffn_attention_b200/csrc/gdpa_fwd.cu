@@ -7,21 +7,28 @@
 // identity (element-wise) or a row softmax with running max and sum (Kunlun
 // reproduction notes, "Core equations": softmax(QK^T/sqrt(d) + log sigma(G))).
 //
-// One persistent CTA per SM walks (sample, head) units in longest-first order.
-// For each 128-row query tile of the unit it walks the key blocks the tile can
-// see (all of them, or the band of the sliding window, Kunlun paper review
-// §2.5), so padding rows and invisible key blocks are never loaded.
+// One persistent CTA per SM walks (sample, head) units in longest-first order
+// and, within a unit, its 128-row query tiles.  Tiles alternate between two
+// slots, each with its own phi warpgroup, Q buffer and TMEM (S of one 128-key
+// block and the O accumulator: 2 x 256 columns), so one slot's MMAs run while
+// the other slot's phi warpgroup works.  P (bf16) goes back into TMEM over the
+// S columns it came from and is the A operand of the PV MMA.  K/V blocks come
+// through one ring shared by both slots; a unit without a band whose blocks
+// fit in the ring loads them once for all its tiles.  A tile only loads the
+// key blocks it can see (all of them, or the band of the sliding window,
+// Kunlun paper review §2.5).  128-key blocks keep the MMA count low: a
+// tcgen05.mma of 128 x N x 16 costs about the same for N = 64 and N = 128.
 //
-// Warp roles (256 threads):
-//   warp 0     TMA producer: Q tile (2 buffers), K and V blocks (ring of stages)
-//   warp 1     MMA issuer (one thread): S = Q K^T into TMEM (2 buffers),
-//              O += P V into TMEM
-//   warp 2     TMEM allocator
-//   warp 3     bias warp: beta for each key block (log sigma(G) for the gate)
-//   warps 4-7  phi / epilogue warpgroup: one thread per query row; reads S
-//              from TMEM, applies the mask and phi, writes P (bf16) to shared
-//              memory for the PV MMA, rescales O when the running max moves,
-//              and writes O (bf16) and LSE at the end of the tile.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles, K/V blocks (tile order)
+//   warp 1      MMA issuer (one thread), event driven over both slots:
+//               S = Q K^T into the slot's free S buffer, O += P V
+//   warp 2      TMEM allocator; bias warp of slot 0
+//   warp 3      bias warp of slot 1: beta of each key block (log sigma(G))
+//   warps 4-7   phi / epilogue warpgroup of slot 0, warps 8-11 of slot 1: one
+//               thread per query row; reads S from TMEM, applies the mask and
+//               phi, writes P to TMEM, rescales O when the running max moves,
+//               and writes O (bf16) and LSE at the end of the tile.
 // Every wait is bounded; on expiry the kernel records GDPA_ERR_TIMEOUT in the
 // workspace status, all roles leave their loops, TMEM is freed and the kernel
 // returns.
@@ -34,60 +41,66 @@
 namespace gdpa {
 namespace {
 
-template <int D_, int BN_>
+constexpr int kThreads = 384;
+constexpr int kBN = 128;  // keys per block
+constexpr int kRegsLaunch = 168;   // 65536 / 384 rounded down to a multiple of 8
+constexpr int kRegsControl = 104;  // warpgroup 0: producer, MMA issuer, allocator, bias
+constexpr int kRegsPhi = 200;      // the two phi warpgroups
+static_assert(128 * kRegsControl + 256 * kRegsPhi <= kThreads * kRegsLaunch,
+              "register split exceeds the launch's registers");
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
+
+template <int D_>
 struct FwdCfg {
   static constexpr int D = D_;
-  static constexpr int BN = BN_;
+  static constexpr int BN = kBN;
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
-  // (64 B, 64-byte swizzle) when D = 32.  P panels are always 64 keys wide.
+  // (64 B, 64-byte swizzle) when D = 32.
   static constexpr int PANEL_ELEMS = D >= 64 ? 64 : 32;
   static constexpr int PANEL_BYTES = PANEL_ELEMS * 2;
   static constexpr int NPANEL = D / PANEL_ELEMS;
   static constexpr uint32_t LAYOUT = D >= 64 ? LAYOUT_SW128 : LAYOUT_SW64;
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int NQ = 2;
-  // K/V ring: 2 stages of 64 KB for D = 128 with 128-key blocks, else 3-4
-  static constexpr int NKV = (D == 128 && BN == 128) ? 2 : (D * BN <= 64 * 64 ? 4 : 3);
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NKV * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NKV * KV_BYTES;
-  static constexpr int OFF_STAGE = OFF_P + P_BYTES;        // O staging when D > BN
-  static constexpr int STAGE_BYTES = D > BN ? BM * D * 2 : 0;
-  static constexpr int OFF_BIAS = OFF_STAGE + STAGE_BYTES;   // float [2][BN]
-  static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;     // uint64 barriers
-  // barrier indices
+  static constexpr int KV_BYTES = BN * D * 2;  // one K (or V) block
+  // K/V ring: 128 KB of stages (2 for D = 128, 4 for D = 64, 8 for D = 32)
+  static constexpr int NKV = (64 * 1024) / KV_BYTES;
+  static constexpr int STAGE_WARP = 32 * 128;  // O staging: 32 rows x 128 B per phi warp
+  static constexpr int OFF_Q = 0;                                // [2 slots]
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;              // [NKV]
+  static constexpr int OFF_V = OFF_K + NKV * KV_BYTES;           // [NKV]
+  static constexpr int OFF_STAGE = OFF_V + NKV * KV_BYTES;       // [8 phi warps]
+  static constexpr int OFF_BIAS = OFF_STAGE + 8 * STAGE_WARP;    // float [2 slots][2][BN]
+  static constexpr int OFF_KVCNT = OFF_BIAS + 2 * 2 * BN * 4;    // int [3][8]
+  static constexpr int OFF_BAR = OFF_KVCNT + 3 * 8 * 4;
+  // barrier indices (per slot s: [s]; bias buffers of slot s: [2s + b])
   static constexpr int B_QFULL = 0;
-  static constexpr int B_QEMPTY = B_QFULL + NQ;
-  static constexpr int B_KVFULL = B_QEMPTY + NQ;
+  static constexpr int B_QEMPTY = B_QFULL + 2;
+  static constexpr int B_KVFULL = B_QEMPTY + 2;
   static constexpr int B_KVEMPTY = B_KVFULL + NKV;
   static constexpr int B_SFULL = B_KVEMPTY + NKV;
-  static constexpr int B_SEMPTY = B_SFULL + 2;
-  static constexpr int B_PFULL = B_SEMPTY + 2;
-  static constexpr int B_PVDONE = B_PFULL + 1;
-  static constexpr int B_OFULL = B_PVDONE + 1;
-  static constexpr int B_OEMPTY = B_OFULL + 1;
-  static constexpr int B_BFULL = B_OEMPTY + 1;   // 2 bias buffers
-  static constexpr int B_BEMPTY = B_BFULL + 2;
-  static constexpr int NBARS = B_BEMPTY + 2;
-  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;      // tmem addr, abort flag
+  static constexpr int B_PFULL = B_SFULL + 2;
+  static constexpr int B_PVDONE = B_PFULL + 2;
+  static constexpr int B_OFULL = B_PVDONE + 2;
+  static constexpr int B_OEMPTY = B_OFULL + 2;
+  static constexpr int B_BFULL = B_OEMPTY + 2;
+  static constexpr int B_BEMPTY = B_BFULL + 4;
+  static constexpr int NBARS = B_BEMPTY + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem addr, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES;  // base is 1024-aligned (checked at entry)
-  // TMEM: S buffers at columns [0, BN) and [BN, 2BN); O at [2BN, 2BN + D).
-  static constexpr int TMEM_S0 = 0;
-  static constexpr int TMEM_O = 2 * BN;
-  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  // TMEM: slot s at column 256 s: S (then P over its first BN / 2 columns)
+  // at +0, O at +BN.
+  static constexpr int TMEM_SLOT = 256;
+  static constexpr int TMEM_O = BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(BN + D <= TMEM_SLOT, "TMEM slot");
+  static_assert(NKV >= 2 && NKV <= 8, "K/V ring");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-  static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0 && P_BYTES % 1024 == 0, "align");
+  static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "align");
 };
-
-constexpr int kThreads = 256;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
 using Unit = GdpaUnit;
 
@@ -104,39 +117,100 @@ __device__ __forceinline__ void kv_range(int m0, int Lk, int wl, int wr, int& kb
   }
 }
 
-// K/V stay in shared memory for all query tiles of a unit when there is no
-// band (every tile sees every key block), the unit has more than one tile,
-// and its key blocks fit in the K/V ring.  Otherwise each tile streams the
-// blocks it can see.
+// One query tile of the CTA's walk.
+struct FTile {
+  int h, q0, Lq, k0, Lk;
+  int m0, kb0, kb1;     // first local row; visible key blocks [kb0, kb1)
+  int ntile;            // query tiles of the unit
+  uint32_t kv0;         // K/V ring index of block kb0 (the tile's blocks are consecutive)
+  bool resident;        // the unit's blocks are loaded once, at its first tile
+  bool unit_first;      // first tile of its unit
+  int slot;             // 0 or 1: tiles alternate between the two slots
+};
+
+// The CTA's tiles in the order every role uses.  Units come from UnitStream
+// (longest first, boustrophedon over the grid); K/V ring indices advance by
+// the unit's block count at a resident unit's first tile and by the visible
+// block count at every tile of a streamed unit.
 template <class C>
-__device__ __forceinline__ bool kv_resident(const FwdArgs& a, const Unit& t, int& nkb) {
-  nkb = (t.Lk + C::BN - 1) / C::BN;
-  return a.wl < 0 && a.wr < 0 && t.Lq > kBlockM && nkb > 0 && nkb <= C::NKV;
-}
+struct TileWalk {
+  UnitStream units;
+  Unit t;
+  int wl, wr, ntile, mt, nkb;
+  uint32_t g, kvi, unit_kv0;
+  bool resident, in_unit;
+  __device__ explicit TileWalk(const FwdArgs& a)
+      : units(a.info, a.H, a.n_units), t{}, wl(a.wl), wr(a.wr), ntile(0), mt(0), nkb(0), g(0),
+        kvi(0), unit_kv0(0), resident(false), in_unit(false) {}
+  __device__ bool next(FTile& x) {
+    for (;;) {
+      if (!in_unit) {
+        if (!units.next(t)) return false;
+        ntile = (t.Lq + kBlockM - 1) / kBlockM;
+        nkb = (t.Lk + C::BN - 1) / C::BN;
+        resident = wl < 0 && wr < 0 && nkb > 0 && nkb <= C::NKV;
+        unit_kv0 = kvi;
+        if (resident && ntile > 0) kvi += nkb;
+        mt = 0;
+        in_unit = true;
+      }
+      if (mt >= ntile) {
+        in_unit = false;
+        continue;
+      }
+      x.h = t.h;
+      x.q0 = t.q0;
+      x.Lq = t.Lq;
+      x.k0 = t.k0;
+      x.Lk = t.Lk;
+      x.m0 = mt * kBlockM;
+      kv_range<C::BN>(x.m0, t.Lk, wl, wr, x.kb0, x.kb1);
+      x.ntile = ntile;
+      x.resident = resident;
+      x.unit_first = mt == 0;
+      if (resident) {
+        x.kv0 = unit_kv0 + x.kb0;
+      } else {
+        x.kv0 = kvi;
+        if (x.kb1 > x.kb0) kvi += x.kb1 - x.kb0;
+      }
+      x.slot = (int)(g & 1);
+      ++g;
+      ++mt;
+      return true;
+    }
+  }
+  // next tile of slot s
+  __device__ bool next_slot(FTile& x, int s) {
+    while (next(x))
+      if (x.slot == s) return true;
+    return false;
+  }
+};
 
 template <class C>
 struct Smem {
   uint32_t base;  // shared address of the 1024-aligned base
   uint8_t* ptr;
   __device__ uint32_t q(int s) const { return base + C::OFF_Q + s * C::Q_BYTES; }
-  __device__ uint32_t k(int s) const { return base + C::OFF_K + s * C::KV_BYTES; }
-  __device__ uint32_t v(int s) const { return base + C::OFF_V + s * C::KV_BYTES; }
-  __device__ uint32_t p() const { return base + C::OFF_P; }
-  // O staging of warp w, row j (0..31), 16-byte chunk cc, chunks XOR-swizzled by
-  // row.  With D <= BN it lies in the P rows 32w..32w+31 of each 64-key panel
-  // (only warp w writes those); otherwise in a separate region.
-  __device__ uint32_t stage(int w, int j, int cc) const {
-    constexpr int ROWB = C::D * 2;
-    constexpr int SW = (ROWB / 16) >= 8 ? 7 : 3;
-    const uint32_t b = j * ROWB + ((cc ^ (j & SW)) << 4);
-    if constexpr (C::D <= C::BN) {
-      return base + C::OFF_P + (b >> 12) * (kBlockM * 128) + w * 32 * 128 + (b & 4095);
-    } else {
-      return base + C::OFF_STAGE + w * 32 * ROWB + b;
-    }
+  __device__ uint32_t k(int st) const { return base + C::OFF_K + st * C::KV_BYTES; }
+  __device__ uint32_t v(int st) const { return base + C::OFF_V + st * C::KV_BYTES; }
+  // O staging of phi warp pw (0..7), row j (0..31), 16-byte chunk c of a
+  // 128-byte row segment, chunks XOR-swizzled by row (mask m)
+  __device__ uint32_t stage(int pw, int j, int c, int m) const {
+    return base + C::OFF_STAGE + pw * C::STAGE_WARP + j * 128 + ((c ^ (j & m)) << 4);
   }
-  __device__ float* bias(int s) const {
-    return reinterpret_cast<float*>(ptr + C::OFF_BIAS) + s * C::BN;
+  __device__ float* bias(int s, int b) const {
+    return reinterpret_cast<float*>(ptr + C::OFF_BIAS) + (s * 2 + b) * C::BN;
+  }
+  // issuer-private per stage: [0] ring index (+1) its count was set for,
+  // [1] PVs still to read it
+  __device__ int* kv_count(int i) const {
+    return reinterpret_cast<int*>(ptr + C::OFF_KVCNT) + i * 8;
+  }
+  // per stage: the ring index the producer is loading into it
+  __device__ volatile int* kv_tag() const {
+    return reinterpret_cast<volatile int*>(ptr + C::OFF_KVCNT) + 2 * 8;
   }
   __device__ uint32_t bar(int i) const { return base + C::OFF_BAR + i * 8; }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(ptr + C::OFF_MISC); }
@@ -146,227 +220,271 @@ struct Smem {
 };
 
 // ------------------------------------------------------------------ producer
+// Q of each tile into its slot's buffer; K/V blocks into the ring in ring-index
+// order (a resident unit's blocks at its first tile, a streamed tile's visible
+// blocks at the tile).  While a unit's blocks load, the next unit's first
+// blocks are prefetched into L2.
 template <class C>
 __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtensorMap* tq,
                               const CUtensorMap* tk, const CUtensorMap* tv) {
   volatile int* abort = sm.abort_flag();
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
-  uint32_t qi = 0, kvi = 0;
+  uint32_t nq[2] = {0u, 0u};
   bool dropped = false;
-  UnitStream units(a.info, a.H, a.n_units);
-  Unit t;
-  while (units.next(t)) {
-    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
-    int nkb;
-    const bool resident = kv_resident<C>(a, t, nkb);
-    auto load_kv = [&](int j) -> bool {
-      const int ks = kvi % C::NKV;
-      if (!mbar_wait(sm.bar(C::B_KVEMPTY + ks), ((kvi / C::NKV) & 1) ^ 1, abort, a.status,
-                     a.timeout_ns, 0x000 + C::B_KVEMPTY + ks))
-        return false;
-      mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + ks), 2 * C::KV_BYTES);
-      for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
-        tma_load_3d(sm.k(ks) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + ks),
-                    pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
-        tma_load_3d(sm.v(ks) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + ks),
-                    pnl * C::PANEL_ELEMS, t.h, t.k0 + j * C::BN, pol_keep);
-      }
-      ++kvi;
-      return true;
-    };
-    for (int mt = 0; mt < ntile; ++mt) {
-      const int m0 = mt * kBlockM;
-      int kb0, kb1;
-      kv_range<C::BN>(m0, t.Lk, a.wl, a.wr, kb0, kb1);
-      if (kb1 <= kb0) continue;
-      const int qs = qi % C::NQ;
-      if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((qi / C::NQ) & 1) ^ 1, abort, a.status,
-                     a.timeout_ns, 0x000 + C::B_QEMPTY + qs))
-        return;
-      if ((a.debug_flags & 1) && !dropped && blockIdx.x == 0) {
-        dropped = true;  // test hook: this Q tile is never loaded
-      } else {
-        mbar_arrive_expect_tx(sm.bar(C::B_QFULL + qs), C::Q_BYTES);
-        for (int pnl = 0; pnl < C::NPANEL; ++pnl)
-          tma_load_3d(sm.q(qs) + pnl * kBlockM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + qs),
-                      pnl * C::PANEL_ELEMS, t.h, t.q0 + m0, pol_stream);
-      }
-      ++qi;
-      if (resident && mt > 0) continue;  // the unit's blocks are already in the ring
-      for (int j = kb0; j < kb1; ++j)
-        if (!load_kv(j)) return;
+  TileWalk<C> walk(a);
+  FTile x;
+  auto load_kv = [&](uint32_t ring, int kb) -> bool {
+    const int st = (int)(ring % C::NKV);
+    if (!mbar_wait(sm.bar(C::B_KVEMPTY + st), ((ring / C::NKV) & 1) ^ 1, abort, a.status,
+                   a.timeout_ns, 0x000 + C::B_KVEMPTY + st))
+      return false;
+    sm.kv_tag()[st] = (int)ring;  // published by the arrive below (release)
+    mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + st), 2 * C::KV_BYTES);
+    for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
+      tma_load_3d(sm.k(st) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + st),
+                  pnl * C::PANEL_ELEMS, x.h, x.k0 + kb * C::BN, pol_keep);
+      tma_load_3d(sm.v(st) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + st),
+                  pnl * C::PANEL_ELEMS, x.h, x.k0 + kb * C::BN, pol_keep);
     }
+    return true;
+  };
+  while (walk.next(x)) {
+    if (x.kb1 <= x.kb0) continue;  // no visible keys: the phi warpgroup writes zeros
+    const int s = x.slot;
+    if (!mbar_wait(sm.bar(C::B_QEMPTY + s), (nq[s] & 1) ^ 1, abort, a.status, a.timeout_ns,
+                   0x000 + C::B_QEMPTY + s))
+      return;
+    if ((a.debug_flags & 1) && !dropped && blockIdx.x == 0) {
+      dropped = true;  // test hook: this Q tile is never loaded
+    } else {
+      mbar_arrive_expect_tx(sm.bar(C::B_QFULL + s), C::Q_BYTES);
+      for (int pnl = 0; pnl < C::NPANEL; ++pnl)
+        tma_load_3d(sm.q(s) + pnl * kBlockM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + s),
+                    pnl * C::PANEL_ELEMS, x.h, x.q0 + x.m0, pol_stream);
+    }
+    ++nq[s];
+    if (x.resident && !x.unit_first) continue;  // the unit's blocks are in the ring
+    if (x.unit_first) {
+      // warm L2 with the next unit's first blocks (its loads wait for ring stages)
+      Unit nt;
+      if (walk.units.peek(nt)) {
+        const int nb = min((nt.Lk + C::BN - 1) / C::BN, 2);
+        for (int j = 0; j < nb; ++j)
+          for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
+            tma_prefetch_l2_3d(tk, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
+            tma_prefetch_l2_3d(tv, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
+          }
+      }
+    }
+    for (int kb = x.kb0; kb < x.kb1; ++kb)
+      if (!load_kv(x.kv0 + (uint32_t)(kb - x.kb0), kb)) return;
   }
 }
 
 // ------------------------------------------------------------------ MMA issuer
-// The issuer keeps one PV behind: S of the next key block (of this tile, or of
-// the next tile or unit) is issued before the PV of the current one, so the
-// phi warpgroup finds its next S ready when it finishes a block or a tile.
+// Per slot: S of block i goes once the slot's previous PV has completed (P
+// lives in the S columns); PV of block i goes once the phi warpgroup has
+// written P (and, for the tile's first block, the epilogue has read the
+// previous O).  The issuer polls both slots without blocking and issues
+// whatever is ready, so one slot's MMAs run while the other slot's phi works.
+//
+// A K/V stage is released when every PV that reads it has been issued: its
+// use count (tiles of a resident unit, or 1) is set at its first use and
+// counted down at each PV; the commit after the last covers all earlier MMAs.
 template <class C>
 __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   volatile int* abort = sm.abort_flag();
   constexpr uint32_t idesc_s = make_idesc_bf16(kBlockM, C::BN, 0, 0);
   constexpr uint32_t idesc_o = make_idesc_bf16(kBlockM, C::D, 0, 1);
-  constexpr uint32_t SBO_QK = 8 * C::PANEL_BYTES;
-  uint32_t qi = 0, kvi = 0, si = 0, pvi = 0, ti = 0;
+  constexpr uint32_t SBO = 8 * C::PANEL_BYTES;
+  // Base descriptors of Q slot 0, K and V stage 0.  Every operand tile the
+  // issuer names lies at a fixed offset from one of them, and the start
+  // address field (address >> 4, 14 bits) cannot overflow below 256 KB of
+  // shared memory, so an operand's descriptor is base + (offset >> 4).
+  const uint64_t qdesc0 = make_smem_desc(sm.q(0), 16, SBO, C::LAYOUT);
+  const uint64_t kdesc0 = make_smem_desc(sm.k(0), 16, SBO, C::LAYOUT);
+  const uint64_t vdesc0 = make_smem_desc(sm.v(0), C::BN * C::PANEL_BYTES, SBO, C::LAYOUT);
+  int* kv_ring = sm.kv_count(0);  // ring index a stage's count was set for (+1)
+  int* kv_left = sm.kv_count(1);  // PVs still to read the stage
+  for (int i = 0; i < C::NKV; ++i) {
+    kv_ring[i] = 0;
+    kv_left[i] = 0;
+  }
 
-  struct PendingPV {
-    bool valid;
-    bool first;         // first key block of its tile (overwrites O)
-    bool last;          // last key block of its tile (O complete afterwards)
-    int ks;             // K/V stage holding V
-    bool release_kv;    // streamed block: free its stage after this PV
-    uint32_t unit_kvi;  // resident unit ending with this PV: free its stages
-    int unit_nkb;       //   (0 when not)
-  } pend = {false, false, false, 0, false, 0u, 0};
-
-  auto issue_pending = [&]() -> bool {
-    if (!pend.valid) return true;
-    if (!mbar_wait(sm.bar(C::B_PFULL), pvi & 1, abort, a.status, a.timeout_ns,
-                   0x100 + C::B_PFULL))
-      return false;
-    if (pend.first && !mbar_wait(sm.bar(C::B_OEMPTY), (ti & 1) ^ 1, abort, a.status,
-                                 a.timeout_ns, 0x100 + C::B_OEMPTY))
-      return false;
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < C::BN / 16; ++kk) {
-      // A = P [128 x BN] K-major, 64-key panels with 128-byte swizzle
-      const uint32_t pa = sm.p() + (kk * 16 / 64) * (kBlockM * 128) + (kk * 16 % 64) * 2;
-      const uint64_t adesc = make_smem_desc(pa, 16, 1024, LAYOUT_SW128);
-      // B = V [BN keys x D], N (= D) contiguous: MN-major; 16 keys per step
-      const uint32_t vb = sm.v(pend.ks) + kk * 16 * C::PANEL_BYTES;
-      const uint64_t bdesc = make_smem_desc(vb, C::BN * C::PANEL_BYTES, SBO_QK, C::LAYOUT);
-      mma_bf16_ss(tmem + C::TMEM_O, adesc, bdesc, idesc_o, (!pend.first || kk > 0) ? 1u : 0u);
-    }
-    if (pend.release_kv) mma_commit(sm.bar(C::B_KVEMPTY + pend.ks));
-    mma_commit(sm.bar(C::B_PVDONE));
-    ++pvi;
-    if (pend.last) {
-      mma_commit(sm.bar(C::B_OFULL));
-      ++ti;
-    }
-    for (int idx = 0; idx < pend.unit_nkb; ++idx)
-      mma_commit(sm.bar(C::B_KVEMPTY + (pend.unit_kvi + idx) % C::NKV));
-    pend.valid = false;
-    return true;
+  struct Slot {
+    uint32_t kv0;         // ring index of the tile's first block
+    int nkv, ntile;       // blocks of the tile; tiles of its unit
+    bool resident, have;
+    int ns, npv;          // S and PV issued for the tile
+    uint32_t pc, tq;      // PV and non-empty tile counts of the slot
   };
-
-  UnitStream units(a.info, a.H, a.n_units);
-  Unit t;
-  while (units.next(t)) {
-    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
-    int nkb;
-    const bool resident = kv_resident<C>(a, t, nkb);
-    const uint32_t unit_kvi = kvi;  // first ring index of a resident unit
-    for (int mt = 0; mt < ntile; ++mt) {
-      int kb0, kb1;
-      kv_range<C::BN>(mt * kBlockM, t.Lk, a.wl, a.wr, kb0, kb1);
-      const int nkv = kb1 - kb0;
-      if (nkv <= 0) continue;
-      const int qs = qi % C::NQ;
-      if (!mbar_wait(sm.bar(C::B_QFULL + qs), (qi / C::NQ) & 1, abort, a.status, a.timeout_ns,
-                     0x100 + C::B_QFULL + qs))
-        return;
-      if (resident) kvi = unit_kvi;  // every tile walks the same resident stages
-      for (int idx = 0; idx < nkv; ++idx) {
-        const int ks = kvi % C::NKV;
-        // a resident unit frees its stages with its last PV; the next unit's
-        // first load may need them, so that PV is not deferred past this wait
-        if (pend.valid && pend.unit_nkb > 0 && !issue_pending()) return;
-        if ((!resident || mt == 0) &&
-            !mbar_wait(sm.bar(C::B_KVFULL + ks), (kvi / C::NKV) & 1, abort, a.status,
-                       a.timeout_ns, 0x100 + C::B_KVFULL + ks))
-          return;
-        const int sb = si & 1;
-        if (!mbar_wait(sm.bar(C::B_SEMPTY + sb), ((si >> 1) & 1) ^ 1, abort, a.status,
-                       a.timeout_ns, 0x100 + C::B_SEMPTY + sb))
-          return;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::D / 16; ++kk) {
-          const int pnl = kk * 16 / C::PANEL_ELEMS;
-          const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
-          const uint64_t adesc = make_smem_desc(
-              sm.q(qs) + pnl * kBlockM * C::PANEL_BYTES + within, 16, SBO_QK, C::LAYOUT);
-          const uint64_t bdesc = make_smem_desc(
-              sm.k(ks) + pnl * C::BN * C::PANEL_BYTES + within, 16, SBO_QK, C::LAYOUT);
-          mma_bf16_ss(tmem + C::TMEM_S0 + sb * C::BN, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(sm.bar(C::B_SFULL + sb));
-        ++si;
-        if (idx == nkv - 1) {
-          mma_commit(sm.bar(C::B_QEMPTY + qs));
-          ++qi;
-        }
-        ++kvi;
-        // the previous block's PV, now that this block's S is on its way
-        if (!issue_pending()) return;
-        const bool last_of_unit = resident && mt == ntile - 1 && idx == nkv - 1;
-        pend = {true, idx == 0, idx == nkv - 1, ks, !resident,
-                last_of_unit ? unit_kvi : 0u, last_of_unit ? nkb : 0};
+  Slot sl[2];
+  TileWalk<C> walk0(a), walk1(a);
+  auto advance = [&](Slot& z, TileWalk<C>& w, int s) {
+    FTile x;
+    z.have = false;
+    while (w.next_slot(x, s)) {
+      if (x.kb1 > x.kb0) {
+        z.have = true;
+        z.kv0 = x.kv0;
+        z.nkv = x.kb1 - x.kb0;
+        z.ntile = x.ntile;
+        z.resident = x.resident;
+        break;
       }
     }
-    if (resident) kvi = unit_kvi + nkb;
+    z.ns = z.npv = 0;
+  };
+  sl[0].pc = sl[0].tq = 0;
+  sl[1].pc = sl[1].tq = 0;
+  advance(sl[0], walk0, 0);
+  advance(sl[1], walk1, 1);
+
+  uint64_t idle_since = 0;
+  uint32_t idle_polls = 0;
+  while (sl[0].have || sl[1].have) {
+    bool progress = false;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      Slot& z = sl[s];
+      if (!z.have) continue;
+      const uint32_t tslot = tmem + s * C::TMEM_SLOT;
+      // ---- S = Q K^T of block ns
+      if (z.ns < z.nkv && z.ns == z.npv) {
+        const uint32_t ring = z.kv0 + (uint32_t)z.ns;
+        const int st = (int)(ring % C::NKV);
+        bool ok = z.ns > 0 || mbar_test_wait(sm.bar(C::B_QFULL + s), z.tq & 1);
+        // The other slot may be far ahead or behind in the ring: the stage's
+        // full barrier identifies this ring index's phase only once the
+        // producer has started loading it (the previous content's phase done).
+        ok = ok && sm.kv_tag()[st] == (int)ring;
+        ok = ok && mbar_test_wait(sm.bar(C::B_KVFULL + st), (ring / C::NKV) & 1);
+        ok = ok && (z.pc == 0 || mbar_test_wait(sm.bar(C::B_PVDONE + s), (z.pc - 1) & 1));
+        if (ok) {
+          tc_fence_after();
+          const uint64_t qd = qdesc0 + (uint64_t)((s * C::Q_BYTES) >> 4);
+          const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < C::D / 16; ++kk) {
+            // K-major operands: 32 bytes per 16 elements within a 64-element
+            // panel, then the next panel (offsets added to the start address field)
+            const int pnl = kk * 16 / C::PANEL_ELEMS;
+            const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
+            mma_bf16_ss(tslot, desc_add(qd, (pnl * kBlockM * C::PANEL_BYTES + within) >> 4),
+                        desc_add(kd, (pnl * C::BN * C::PANEL_BYTES + within) >> 4), idesc_s,
+                        kk > 0 ? 1u : 0u);
+          }
+          mma_commit(sm.bar(C::B_SFULL + s));
+          if (z.ns == z.nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + s));
+          ++z.ns;
+          progress = true;
+        }
+      }
+      // ---- O += P V of block npv
+      if (z.npv < z.ns) {
+        bool ok = mbar_test_wait(sm.bar(C::B_PFULL + s), z.pc & 1);
+        ok = ok && (z.npv > 0 || mbar_test_wait(sm.bar(C::B_OEMPTY + s), (z.tq & 1) ^ 1));
+        if (ok) {
+          const uint32_t ring = z.kv0 + (uint32_t)z.npv;
+          const int st = (int)(ring % C::NKV);
+          tc_fence_after();
+          const uint64_t vd = vdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            // A = P [128 x BN] from TMEM (bf16 pairs, 8 columns per 16 keys);
+            // B = V [BN keys x D], N (= D) contiguous: MN-major, 16 keys per step
+            mma_bf16_ts(tslot + C::TMEM_O, tslot + kk * 8,
+                        desc_add(vd, (kk * 16 * C::PANEL_BYTES) >> 4), idesc_o,
+                        (z.npv > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(sm.bar(C::B_PVDONE + s));
+          if (kv_ring[st] != (int)ring + 1) {
+            kv_ring[st] = (int)ring + 1;
+            kv_left[st] = z.resident ? z.ntile : 1;
+          }
+          if (--kv_left[st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + st));
+          ++z.npv;
+          ++z.pc;
+          if (z.npv == z.nkv) {
+            mma_commit(sm.bar(C::B_OFULL + s));
+            ++z.tq;
+            advance(z, s == 0 ? walk0 : walk1, s);
+          }
+          progress = true;
+        }
+      }
+    }
+    if (progress) {
+      idle_since = 0;
+      idle_polls = 0;
+    } else if ((++idle_polls & 255u) == 0) {
+      // nothing has been ready for a while: give up (bounded) if nothing moves.
+      // The poll itself does not sleep: a sleeping issuer notices a finished
+      // phi block or MMA only when it wakes, which stalls both slots.
+      const uint64_t now = globaltimer_ns();
+      if (idle_since == 0) idle_since = now;
+      if (*abort) return;
+      if (now - idle_since > a.timeout_ns) {
+        *abort = 1;
+        record_error(a.status, 5, 0x100);
+        return;
+      }
+    }
   }
-  issue_pending();
 }
 
-// ------------------------------------------------------------------ bias warp
+// ------------------------------------------------------------------ bias warps
+// beta of each key block a tile of slot s sees, into the slot's 2-buffer ring.
 template <class C>
-__device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
+__device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, int s, bool softmax) {
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
-  uint32_t bi = 0;
-  UnitStream units(a.info, a.H, a.n_units);
-  Unit t;
-  while (units.next(t)) {
-    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
-    for (int mt = 0; mt < ntile; ++mt) {
-      int kb0, kb1;
-      kv_range<C::BN>(mt * kBlockM, t.Lk, a.wl, a.wr, kb0, kb1);
-      for (int j = kb0; j < kb1; ++j) {
-        const int bs = bi & 1;
-        bool ok = mbar_wait(sm.bar(C::B_BEMPTY + bs), ((bi >> 1) & 1) ^ 1, abort, a.status,
-                            a.timeout_ns, 0x300 + C::B_BEMPTY + bs);
-        if (!__all_sync(0xffffffffu, ok)) return;
-        float* dst = sm.bias(bs);
-        const float* src = a.bias + (int64_t)t.h * a.total_kv + t.k0;
-        for (int c = lane; c < C::BN; c += 32) {
-          const int key = j * C::BN + c;
-          float beta = 0.f;
-          if (key < t.Lk) {
-            const float g = src[key];
-            if (a.bias_kind == 2) {
-              // log sigma(g) = min(g, 0) - log(1 + exp(-|g|))
-              beta = fminf(g, 0.f) - log1pf(__expf(-fabsf(g)));
-            } else {
-              beta = g;
-            }
+  uint32_t bc = 0;
+  TileWalk<C> walk(a);
+  FTile x;
+  while (walk.next_slot(x, s)) {
+    for (int j = x.kb0; j < x.kb1; ++j) {
+      const int bb = bc & 1;
+      bool ok = mbar_wait(sm.bar(C::B_BEMPTY + 2 * s + bb), ((bc >> 1) & 1) ^ 1, abort, a.status,
+                          a.timeout_ns, 0x300 + C::B_BEMPTY + 2 * s + bb);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      float* dst = sm.bias(s, bb);
+      const float* src = a.bias + (int64_t)x.h * a.total_kv + x.k0;
+      for (int c = lane; c < C::BN; c += 32) {
+        const int key = j * C::BN + c;
+        float beta = 0.f;
+        if (key < x.Lk) {
+          const float g = src[key];
+          if (a.bias_kind == 2) {
+            // log sigma(g) = min(g, 0) - log(1 + exp(-|g|))
+            beta = fminf(g, 0.f) - log1pf(__expf(-fabsf(g)));
+          } else {
+            beta = g;
           }
-          dst[c] = softmax ? beta * kLog2e : beta;
         }
-        mbar_arrive(sm.bar(C::B_BFULL + bs));  // one arrival per lane, after its writes
-        ++bi;
+        dst[c] = softmax ? beta * kLog2e : beta;
       }
+      mbar_arrive(sm.bar(C::B_BFULL + 2 * s + bb));  // one arrival per lane, after its writes
+      ++bc;
     }
   }
 }
 
-// ------------------------------------------------------------------ phi warpgroup
+// ------------------------------------------------------------------ phi warpgroups
 template <class C, bool SOFTMAX>
-__device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
+__device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
   volatile int* abort = sm.abort_flag();
-  const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quarter of this warp
+  const int warp = threadIdx.x >> 5;
+  const int wq = warp & 3;                  // TMEM lane quarter of this warp
+  const int pw = warp - 4;                  // phi warp index: its O staging slice
   const int lane = threadIdx.x & 31;
   const int r = wq * 32 + lane;             // row of the tile owned by this thread
-  const uint32_t tl = (uint32_t)(wq * 32) << 16;
+  const uint32_t tslot = tmem + ((uint32_t)(wq * 32) << 16) + s * C::TMEM_SLOT;
   const bool has_bias = a.bias_kind != 0;
   const bool identity = a.phi == 2;
   const float sc = SOFTMAX ? a.scale * kLog2e : a.scale;
-  uint32_t si = 0, pvi = 0, ti = 0, bi = 0;
+  uint32_t nsb = 0, tq = 0, bc = 0;  // S blocks, non-empty tiles, bias blocks of the slot
 
 #define PHI_WAIT(bar_, par_, where_)                                                   \
   do {                                                                               \
@@ -374,226 +492,219 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
     if (!__all_sync(0xffffffffu, ok_)) return;                                       \
   } while (0)
 
-  UnitStream units(a.info, a.H, a.n_units);
-  Unit t;
-  while (units.next(t)) {
-    const int ntile = (t.Lq + kBlockM - 1) / kBlockM;
-    for (int mt = 0; mt < ntile; ++mt) {
-      const int m0 = mt * kBlockM;
-      const int row = m0 + r;
-      const bool row_ok = row < t.Lq;
-      int kb0, kb1;
-      kv_range<C::BN>(m0, t.Lk, a.wl, a.wr, kb0, kb1);
-      const int nkv = kb1 - kb0;
-      if (nkv <= 0) {
-        if (row_ok) {
-          __nv_bfloat16* orow = a.o + ((int64_t)(t.q0 + row) * a.H + t.h) * C::D;
-          uint4 z = make_uint4(0, 0, 0, 0);
-          for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
-          if (SOFTMAX && a.lse) a.lse[(int64_t)t.h * a.total_q + t.q0 + row] = -INFINITY;
-        }
-        continue;
+  TileWalk<C> walk(a);
+  FTile x;
+  while (walk.next_slot(x, s)) {
+    const int row = x.m0 + r;
+    const bool row_ok = row < x.Lq;
+    const int nkv = x.kb1 - x.kb0;
+    if (nkv <= 0) {
+      if (row_ok) {
+        __nv_bfloat16* orow = a.o + ((int64_t)(x.q0 + row) * a.H + x.h) * C::D;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+        if (SOFTMAX && a.lse) a.lse[(int64_t)x.h * a.total_q + x.q0 + row] = -INFINITY;
       }
-      // visible keys of this row: [lo, hi]
-      const int lo = a.wl >= 0 ? row - a.wl : INT_MIN;
-      const int hi = min(t.Lk - 1, a.wr >= 0 ? row + a.wr : INT_MAX);
-      float m_run = -INFINITY, l_run = 0.f;
-      for (int idx = 0; idx < nkv; ++idx) {
-        const int kbase = (kb0 + idx) * C::BN;
-        const int bs = bi & 1;
-        if (has_bias) PHI_WAIT(C::B_BFULL + bs, (bi >> 1) & 1, 0x400 + C::B_BFULL + bs);
-        const int sb = si & 1;
-        PHI_WAIT(C::B_SFULL + sb, (si >> 1) & 1, 0x400 + C::B_SFULL + sb);
-        tc_fence_after();
-        uint32_t sv[C::BN];  // S row, then P (fp32 bits), in place
-#pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c)
-          tmem_ld32p(tmem + tl + C::TMEM_S0 + sb * C::BN + c * 32, sv + c * 32);
+      continue;
+    }
+    // visible keys of this row: [lo, hi]
+    const int lo = a.wl >= 0 ? row - a.wl : INT_MIN;
+    const int hi = min(x.Lk - 1, a.wr >= 0 ? row + a.wr : INT_MAX);
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int idx = 0; idx < nkv; ++idx) {
+      const int kbase = (x.kb0 + idx) * C::BN;
+      const int bb = bc & 1;
+      if (has_bias) PHI_WAIT(C::B_BFULL + 2 * s + bb, (bc >> 1) & 1, 0x400 + C::B_BFULL + 2 * s + bb);
+      PHI_WAIT(C::B_SFULL + s, nsb & 1, 0x400 + C::B_SFULL + s);
+      tc_fence_after();
+      const float2* bias2 = reinterpret_cast<const float2*>(sm.bias(s, bb));
+      // visible columns of this block: [clo, chi] (no shift of an unbounded side)
+      const int clo = a.wl >= 0 ? lo - kbase : INT_MIN;
+      const int chi = hi - kbase;  // hi <= Lk - 1 always
+      const bool full = clo <= 0 && chi >= C::BN - 1;
+      const uint64_t sc2 = f2_pack(sc, sc);
+      // scores of 32 columns starting at c0: x = scale * s + beta (masked
+      // columns: -inf for softmax, 0 otherwise), two columns per instruction
+      auto scores = [&](int c0, uint32_t (&v)[32]) {
+        tmem_ld32(tslot + c0, v);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(sm.bar(C::B_SEMPTY + sb));
-        ++si;
-        const float2* bias2 = reinterpret_cast<const float2*>(sm.bias(bs));
-        // visible columns of this block: [clo, chi] (no shift of an unbounded side)
-        const int clo = a.wl >= 0 ? lo - kbase : INT_MIN;
-        const int chi = hi - kbase;  // hi <= Lk - 1 always
-        const bool full = clo <= 0 && chi >= C::BN - 1;
-        const uint64_t sc2 = f2_pack(sc, sc);
-        // scores x = scale * s + beta, two columns per packed instruction
 #pragma unroll
-        for (int c = 0; c < C::BN; c += 2) {
-          uint64_t x2 = f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+        for (int e = 0; e < 32; e += 2) {
+          uint64_t x2 = f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
           if (has_bias) {
-            const float2 b = bias2[c >> 1];
-            x2 = f2_fma(x2, sc2, f2_pack(b.x, b.y));
+            const float2 bv = bias2[(c0 + e) >> 1];
+            x2 = f2_fma(x2, sc2, f2_pack(bv.x, bv.y));
           } else {
             x2 = f2_mul(x2, sc2);
           }
           float x0, x1;
           f2_unpack(x2, x0, x1);
-          sv[c] = __float_as_uint(x0);
-          sv[c + 1] = __float_as_uint(x1);
+          v[e] = __float_as_uint(x0);
+          v[e + 1] = __float_as_uint(x1);
         }
         if (!full) {  // band edges and the ragged last key block
           const float fill = SOFTMAX ? -INFINITY : 0.f;
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c)
-            if (c < clo || c > chi) sv[c] = __float_as_uint(fill);
+          for (int e = 0; e < 32; ++e)
+            if (c0 + e < clo || c0 + e > chi) v[e] = __float_as_uint(fill);
         }
-        if (!SOFTMAX) {
-          if (!identity) {
-            const uint64_t half2 = f2_pack(0.5f, 0.5f);
+      };
+      bool need_rescale = false;
+      float factor = 1.f;
+      if (SOFTMAX) {
+        // pass 1: the block's row maximum (4 independent partial maxima)
+        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int c0 = 0; c0 < C::BN; c0 += 32) {
+          uint32_t v[32];
+          scores(c0, v);
 #pragma unroll
-            for (int c = 0; c < C::BN; c += 2) {
-              // silu(x) = h + h tanh(h), h = x / 2
-              const uint64_t h2 =
-                  f2_mul(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), half2);
-              float h0, h1;
-              f2_unpack(h2, h0, h1);
-              const uint64_t p2 = f2_fma(h2, f2_pack(tanh_approx(h0), tanh_approx(h1)), h2);
-              float p0, p1;
-              f2_unpack(p2, p0, p1);
-              sv[c] = __float_as_uint(p0);
-              sv[c + 1] = __float_as_uint(p1);
-            }
-            if (!full) {  // silu(0) = 0 already; keep masked columns exactly zero
-#pragma unroll
-              for (int c = 0; c < C::BN; ++c)
-                if (c < clo || c > chi) sv[c] = 0u;
-            }
-          }
+          for (int e = 0; e < 32; e += 2)
+            pm[(e >> 1) & 3] = fmax3(pm[(e >> 1) & 3], __uint_as_float(v[e]),
+                                     __uint_as_float(v[e + 1]));
         }
-        if (has_bias) {
-          tc_fence_before();
-          mbar_arrive(sm.bar(C::B_BEMPTY + bs));
-          ++bi;
+        const float bm = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
+        if (idx == 0) {
+          m_run = bm;
+        } else if (bm > m_run + kRescaleThreshold) {
+          factor = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - bm);
+          need_rescale = true;
+          l_run *= factor;
+          m_run = bm;
         }
-        bool need_rescale = false;
-        float factor = 1.f;
+      }
+      // pass 2: P = phi(x), 32 columns at a time, written back as bf16 pairs over
+      // the S columns: chunk c0 lands in columns [c0/2, c0/2 + 16), which only
+      // hold S columns of chunks already read
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
+      const uint64_t half2 = f2_pack(0.5f, 0.5f);
+      uint64_t ps2[2] = {0ull, 0ull};  // packed partial sums (softmax)
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::BN; c0 += 32) {
+        uint32_t v[32];
+        scores(c0, v);
         if (SOFTMAX) {
-          // 4 independent partial maxima over 3-input max: no BN-long chain
-          float pm[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) pm[k] = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < C::BN; c += 2)
-            pm[(c >> 1) & 3] = fmax3(pm[(c >> 1) & 3], __uint_as_float(sv[c]),
-                                     __uint_as_float(sv[c + 1]));
-          const float bm = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
-          if (idx == 0) {
-            m_run = bm;
-          } else if (bm > m_run + kRescaleThreshold) {
-            factor = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - bm);
-            need_rescale = true;
-            l_run *= factor;
-            m_run = bm;
-          }
-          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-          const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
-          uint64_t ps2[2] = {0ull, 0ull};  // packed partial sums
-#pragma unroll
-          for (int c = 0; c < C::BN; c += 2) {
+          for (int e = 0; e < 32; e += 2) {
             const uint64_t d2 =
-                f2_add(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), neg_m2);
+                f2_add(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), neg_m2);
             float d0, d1;
             f2_unpack(d2, d0, d1);
             const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
-            sv[c] = __float_as_uint(p0);
-            sv[c + 1] = __float_as_uint(p1);
-            ps2[(c >> 1) & 1] = f2_add(ps2[(c >> 1) & 1], f2_pack(p0, p1));
+            v[e] = __float_as_uint(p0);
+            v[e + 1] = __float_as_uint(p1);
+            ps2[(e >> 1) & 1] = f2_add(ps2[(e >> 1) & 1], f2_pack(p0, p1));
           }
-          float s0, s1, s2, s3;
-          f2_unpack(ps2[0], s0, s1);
-          f2_unpack(ps2[1], s2, s3);
-          l_run += (s0 + s1) + (s2 + s3);
-        }
-        // the previous PV must be done before P is overwritten or O rescaled
-        if (idx > 0) PHI_WAIT(C::B_PVDONE, (pvi - 1) & 1, 0x400 + C::B_PVDONE);
-        if (SOFTMAX && __any_sync(0xffffffffu, need_rescale)) {
-          tc_fence_after();
+        } else if (!identity) {
 #pragma unroll
-          for (int c = 0; c < C::D / 16; ++c) {
-            uint32_t raw[16];
-            tmem_ld16(tmem + tl + C::TMEM_O + c * 16, raw);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              raw[e] = __float_as_uint(__uint_as_float(raw[e]) * factor);
-            tmem_st16(tmem + tl + C::TMEM_O + c * 16, raw);
+          for (int e = 0; e < 32; e += 2) {
+            // silu(x) = h + h tanh(h), h = x / 2 (masked columns: silu(0) = 0)
+            const uint64_t h2 =
+                f2_mul(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), half2);
+            float h0, h1;
+            f2_unpack(h2, h0, h1);
+            const uint64_t p2 = f2_fma(h2, f2_pack(tanh_approx(h0), tanh_approx(h1)), h2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            v[e] = __float_as_uint(p0);
+            v[e + 1] = __float_as_uint(p1);
           }
-          tmem_wait_st();
         }
-        // P row -> shared memory, 64-key panels, 128-byte swizzle (K-major A operand)
+        uint32_t pk[16];
 #pragma unroll
-        for (int ch = 0; ch < C::BN / 8; ++ch) {
-          const int pnl = ch / 8, cir = ch % 8;
-          const uint32_t addr =
-              sm.p() + pnl * (kBlockM * 128) + r * 128 + ((cir ^ (r & 7)) << 4);
-          const uint32_t* q8 = sv + ch * 8;
-          st_shared_v4(addr, pack_bf16x2(__uint_as_float(q8[0]), __uint_as_float(q8[1])),
-                       pack_bf16x2(__uint_as_float(q8[2]), __uint_as_float(q8[3])),
-                       pack_bf16x2(__uint_as_float(q8[4]), __uint_as_float(q8[5])),
-                       pack_bf16x2(__uint_as_float(q8[6]), __uint_as_float(q8[7])));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(sm.bar(C::B_PFULL));
-        ++pvi;
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        tmem_st16(tslot + c0 / 2, pk);
       }
-      // epilogue: O row from TMEM -> bf16 -> this warp's staging rows in shared
-      // memory -> whole rows to global memory (coalesced); the staging area of
-      // warp wq lies inside the P rows that only this warp writes
-      PHI_WAIT(C::B_OFULL, ti & 1, 0x400 + C::B_OFULL);
-      tc_fence_after();
-      float inv = 1.f;
-      if (SOFTMAX) inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll 1  // keeps the epilogue's registers out of the way of the hot loop
-      for (int c = 0; c < C::D / 32; ++c) {
+      if (has_bias) {
+        mbar_arrive(sm.bar(C::B_BEMPTY + 2 * s + bb));
+        ++bc;
+      }
+      if (SOFTMAX) {
+        float s0, s1, s2, s3;
+        f2_unpack(ps2[0], s0, s1);
+        f2_unpack(ps2[1], s2, s3);
+        l_run += (s0 + s1) + (s2 + s3);
+      }
+      if (SOFTMAX && __any_sync(0xffffffffu, need_rescale)) {
+        // O must hold every earlier PV of the tile before it is rescaled: the
+        // commit of the previous block's PV covers all of them
+        PHI_WAIT(C::B_PVDONE + s, (nsb - 1) & 1, 0x400 + C::B_PVDONE + s);
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < C::D / 16; ++c) {
+          uint32_t raw[16];
+          tmem_ld16(tslot + C::TMEM_O + c * 16, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * factor);
+          tmem_st16(tslot + C::TMEM_O + c * 16, raw);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(sm.bar(C::B_PFULL + s));
+      ++nsb;
+    }
+    // epilogue: O row from TMEM -> bf16 -> this warp's staging rows in shared
+    // memory -> 128-byte row segments to global memory, 64 columns per pass
+    PHI_WAIT(C::B_OFULL + s, tq & 1, 0x400 + C::B_OFULL + s);
+    tc_fence_after();
+    float inv = 1.f;
+    if (SOFTMAX) inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    constexpr int PW = C::D < 64 ? C::D : 64;  // columns per pass
+    constexpr int NPASS = C::D / PW;
+    constexpr int CPR = PW * 2 / 16;           // 16-byte chunks per row segment
+    constexpr int SWM = CPR - 1;
+#pragma unroll 1
+    for (int ps = 0; ps < NPASS; ++ps) {
+#pragma unroll
+      for (int c = 0; c < PW / 32; ++c) {
         uint32_t raw[32];
-        tmem_ld32(tmem + tl + C::TMEM_O + c * 32, raw);
+        tmem_ld32(tslot + C::TMEM_O + ps * PW + c * 32, raw);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          const int cc = (c * 32 + e) / 8;  // 16-byte chunk of the row
-          st_shared_v4(sm.stage(wq, lane, cc),
+          const int cc = (c * 32 + e) / 8;  // 16-byte chunk of the row segment
+          st_shared_v4(sm.stage(pw, lane, cc, SWM),
                        pack_bf16x2(__uint_as_float(raw[e + 0]) * inv, __uint_as_float(raw[e + 1]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 2]) * inv, __uint_as_float(raw[e + 3]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv));
         }
       }
+      if (ps == NPASS - 1) {  // O fully read: the slot's next tile may overwrite it
+        tc_fence_before();
+        mbar_arrive(sm.bar(C::B_OEMPTY + s));
+      }
       __syncwarp();
-      {
-        constexpr int NCH = C::D / 8;  // 16-byte chunks per row
 #pragma unroll 1
-        for (int it = 0; it < NCH; ++it) {
-          const int lin = it * 32 + lane;
-          const int j = lin / NCH, cc = lin % NCH;  // row of this warp, chunk
-          const int grow = m0 + wq * 32 + j;
-          const uint4 v = ld_shared_v4(sm.stage(wq, j, cc));
-          if (grow < t.Lq)
-            *reinterpret_cast<uint4*>(a.o + ((int64_t)(t.q0 + grow) * a.H + t.h) * C::D +
-                                      cc * 8) = v;
-        }
+      for (int it = 0; it < CPR; ++it) {
+        const int lin = it * 32 + lane;
+        const int j = lin / CPR, cc = lin % CPR;  // row of this warp, chunk
+        const int grow = x.m0 + wq * 32 + j;
+        const uint4 v = ld_shared_v4(sm.stage(pw, j, cc, SWM));
+        if (grow < x.Lq)
+          *reinterpret_cast<uint4*>(a.o + ((int64_t)(x.q0 + grow) * a.H + x.h) * C::D +
+                                    ps * PW + cc * 8) = v;
       }
       __syncwarp();
-      tc_fence_before();
-      mbar_arrive(sm.bar(C::B_OEMPTY));
-      ++ti;
-      if (SOFTMAX && row_ok && a.lse) {
-        a.lse[(int64_t)t.h * a.total_q + t.q0 + row] =
-            l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-      }
+    }
+    ++tq;
+    if (SOFTMAX && row_ok && a.lse) {
+      a.lse[(int64_t)x.h * a.total_q + x.q0 + row] =
+          l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 #undef PHI_WAIT
 }
 
-template <int D, int BN, bool SOFTMAX>
+template <int D, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
-  using C = FwdCfg<D, BN>;
+  using C = FwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
   sm.base = smem_u32(smem_raw);
@@ -604,24 +715,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NQ; ++i) {
-      mbar_init(sm.bar(C::B_QFULL + i), 1);
-      mbar_init(sm.bar(C::B_QEMPTY + i), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(sm.bar(C::B_QFULL + s), 1);
+      mbar_init(sm.bar(C::B_QEMPTY + s), 1);
+      mbar_init(sm.bar(C::B_SFULL + s), 1);
+      mbar_init(sm.bar(C::B_PFULL + s), 128);
+      mbar_init(sm.bar(C::B_PVDONE + s), 1);
+      mbar_init(sm.bar(C::B_OFULL + s), 1);
+      mbar_init(sm.bar(C::B_OEMPTY + s), 128);
     }
     for (int i = 0; i < C::NKV; ++i) {
       mbar_init(sm.bar(C::B_KVFULL + i), 1);
       mbar_init(sm.bar(C::B_KVEMPTY + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(sm.bar(C::B_SFULL + i), 1);
-      mbar_init(sm.bar(C::B_SEMPTY + i), 128);
+    for (int i = 0; i < 4; ++i) {
       mbar_init(sm.bar(C::B_BFULL + i), 32);
       mbar_init(sm.bar(C::B_BEMPTY + i), 128);
     }
-    mbar_init(sm.bar(C::B_PFULL), 128);
-    mbar_init(sm.bar(C::B_PVDONE), 1);
-    mbar_init(sm.bar(C::B_OFULL), 1);
-    mbar_init(sm.bar(C::B_OEMPTY), 128);
+    for (int i = 0; i < 8; ++i) sm.kv_tag()[i] = -1;
     *sm.abort_flag() = 0;
     fence_mbar_init();
   }
@@ -639,14 +750,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  if (warp == 0) {
-    if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
-  } else if (warp == 1) {
-    if (lane == 0) role_mma<C>(a, sm, tmem);
-  } else if (warp == 3) {
-    if (a.bias_kind != 0) role_bias<C>(a, sm, SOFTMAX);
-  } else if (warp >= 4) {
-    role_phi<C, SOFTMAX>(a, sm, tmem);
+  // Registers: warpgroup 0 needs few, the phi warpgroups (a 128-column S row
+  // each) take the rest; each budget is set inside its own branch.
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
+    } else if (warp == 1) {
+      if (lane == 0) role_mma<C>(a, sm, tmem);
+    } else {
+      if (a.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
+    }
+  } else {
+    setmaxnreg_inc<kRegsPhi>();
+    role_phi<C, SOFTMAX>(a, sm, tmem, (warp - 4) >> 2);
   }
   __syncwarp();
   tc_fence_before();
@@ -666,20 +783,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BN, bool SOFTMAX>
+template <int D, bool SOFTMAX>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, int sms, cudaStream_t stream) {
-  using C = FwdCfg<D, BN>;
-  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_ALLOC);
+  using C = FwdCfg<D>;
+  auto kern = gdpa_fwd_kernel<D, SOFTMAX>;
+  // the phi warpgroups raise their register budget with setmaxnreg, which waits
+  // until the block's launch registers cover it: never launch a build whose
+  // per-thread count would leave that wait unsatisfiable
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsPhi) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  // persistent: exactly the CTAs that are resident at once
-  const int grid = std::max(1, std::min(a.n_units, per_sm * sms));
+  // the kernel allocates all 512 TMEM columns: exactly one CTA per SM
+  if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  const int grid = std::max(1, std::min(a.n_units, sms));
   kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv);
   return cudaGetLastError();
 }
@@ -689,23 +812,23 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
 int forward_block_n(int D, int phi, int max_kv, int debug_flags) {
   (void)D;
   (void)phi;
-  return (max_kv <= 64 && !(debug_flags & 2)) ? 64 : 128;
+  (void)max_kv;
+  (void)debug_flags;
+  return kBN;
 }
 
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream) {
+  if (block_n != kBN) return cudaErrorInvalidValue;
   const bool sm = a.phi == 1;
-#define GDPA_FWD_CASE(D_, BN_)                                                       \
-  if (D == D_ && block_n == BN_)                                                     \
-    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, sms, stream)                 \
-              : launch_one<D_, BN_, false>(a, tq, tk, tv, sms, stream);
-  GDPA_FWD_CASE(32, 64)
-  GDPA_FWD_CASE(32, 128)
-  GDPA_FWD_CASE(64, 64)
-  GDPA_FWD_CASE(64, 128)
-  GDPA_FWD_CASE(128, 64)
-  GDPA_FWD_CASE(128, 128)
+#define GDPA_FWD_CASE(D_)                                                 \
+  if (D == D_)                                                            \
+    return sm ? launch_one<D_, true>(a, tq, tk, tv, sms, stream)          \
+              : launch_one<D_, false>(a, tq, tk, tv, sms, stream);
+  GDPA_FWD_CASE(32)
+  GDPA_FWD_CASE(64)
+  GDPA_FWD_CASE(128)
 #undef GDPA_FWD_CASE
   return cudaErrorInvalidValue;
 }

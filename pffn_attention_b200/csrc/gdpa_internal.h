@@ -108,6 +108,16 @@ struct UnitStream {
     u = index(0, blockIdx.x, gridDim.x);
     nxt = u < n_units ? __ldg(info + u / H) : make_int4(0, 0, 0, 0);
   }
+  // The unit the next call of next() returns, without advancing.
+  __device__ __forceinline__ bool peek(GdpaUnit& t) const {
+    if (u >= n_units) return false;
+    t.h = u % H;
+    t.q0 = nxt.x;
+    t.Lq = nxt.y;
+    t.k0 = nxt.z;
+    t.Lk = nxt.w;
+    return true;
+  }
   __device__ __forceinline__ bool next(GdpaUnit& t) {
     if (u >= n_units) return false;
     t.h = u % H;

@@ -65,6 +65,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends), for
+// a thread that polls several barriers and acts on whichever is ready first.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // try_wait that lets the hardware suspend the thread for up to hint_ns (it
 // resumes as soon as the phase completes), so a waiting warp does not take
 // issue slots from the compute warps that share its SM sub-partition.
@@ -98,6 +110,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same call).  The increase waits until other warpgroups have released enough
+// registers, so the budgets must sum to at most the launch's registers.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register budget");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register budget");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -111,6 +137,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4, %5}], [%2], %6;"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
         "l"(policy)
+      : "memory");
+}
+
+// 3-D tile prefetch into L2 only (no shared memory, no completion): warms
+// the lines a later tma_load_3d of the same box will read.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2,
+                                                   uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;"
+      ::"l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 
@@ -276,6 +312,14 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)(layout & 7u) << 61;
   return d;
+}
+
+// desc + off, evaluated where it is used: keeps a loop's per-step descriptors
+// from being hoisted out of it as loop invariants (one register pair each).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t off16) {
+  uint64_t r;
+  asm volatile("add.s64 %0, %1, %2;" : "=l"(r) : "l"(desc), "l"((uint64_t)off16));
+  return r;
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D:

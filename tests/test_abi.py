@@ -87,9 +87,7 @@ def test_workspace_size_grows_with_problem(lib):
 
 
 def test_tile_shape_query(lib):
-    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64))
-    assert (rc, bm, bn) == (0, 128, 64)
-    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=2000))
-    assert (rc, bm, bn) == (0, 128, 128)
-    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64, debug_flags=2))
-    assert (rc, bm, bn) == (0, 128, 128)
+    # one forward tile shape: 128 query rows x 128-key blocks
+    for kv in (64, 2000):
+        rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=kv))
+        assert (rc, bm, bn) == (0, 128, 128)

@@ -45,7 +45,7 @@ def test_workload_parity(cuda_lib, cfg, B):
 # -------------------------------------------------- shapes, activations, biases
 @pytest.mark.parametrize("D", [32, 64, 128])
 @pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY])
-@pytest.mark.parametrize("kv_len", [40, 200])  # key block 64 and 128 paths
+@pytest.mark.parametrize("kv_len", [40, 200])  # one and two 128-key blocks
 def test_head_dims_and_activations(cuda_lib, D, phi, kv_len):
     ql = [1, 127, 128, 129, 300]
     kl = [kv_len, 1, kv_len - 1, kv_len, 63]
@@ -142,23 +142,20 @@ def test_full_size_sampled(cuda_lib, cfg):
     _sampled_full(cuda_lib, cfg)
 
 
-# -------------------------------------------------- 128-key blocks where 64 would be chosen
-@pytest.mark.parametrize("cfg,B", [(1, None), (2, 6)])
-def test_workload_parity_128_key_variant(cuda_lib, cfg, B):
-    w = make_workload(cfg, B=B, with_dout=False)
-    dev = torch.device("cuda")
-    p = cuda_lib.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
-                             window=(w.window_left, w.window_right), bias_kind=w.bias_kind,
-                             max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv, debug_flags=2)
-    rc, bm, bn = cuda_lib.gdpa_forward_tile_shape(p)
-    assert (rc, bm, bn) == (0, 128, 128)
-    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
-    ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
-    bias = w.bias.to(dev) if w.bias is not None else None
-    o, lse, ws = cuda_lib.forward(w.q.to(dev), w.k.to(dev), w.v.to(dev), qo, ko, bias=bias,
-                                  params=p)
-    assert cuda_lib.device_status(ws) == 0
-    ro, rlse = oracle.forward_workload(w)
-    compare("O", o, ro)
-    if w.phi == PHI_SOFTMAX:
-        compare_lse(lse, rlse)
+# -------------------------------------------------- K/V ring: resident and streamed units
+# A unit without a band keeps its key blocks in the shared K/V ring when they
+# fit (D = 128: up to 2 blocks of 128 keys) and streams them per tile otherwise;
+# tiles alternate between the two slots, so odd tile counts end a unit on
+# either slot and the next unit's loads wait for the ring stages it reuses.
+@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU])
+@pytest.mark.parametrize("kv_lens", [[256, 256, 256, 256], [257, 600, 1, 320],
+                                     [64, 256, 257, 192]])
+def test_kv_ring_resident_and_streamed(cuda_lib, phi, kv_lens):
+    ql = [385, 128, 700, 1]
+    if phi == PHI_SOFTMAX:
+        w = make_workload(3, seed=7 + sum(kv_lens), q_lens=ql, kv_lens=kv_lens, H=3, D=128,
+                          phi=phi, scale=1.0 / np.sqrt(128))
+    else:
+        w = make_workload(2, seed=7 + sum(kv_lens), q_lens=ql, kv_lens=kv_lens, H=3, D=128,
+                          phi=phi, scale=1.0, kv_std=1.0 / np.sqrt(128))
+    check_against_oracle(cuda_lib, w)
