@@ -110,11 +110,17 @@ GDPA_API gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const
 /* Backward: dq, dk, dv (bf16) from the forward's inputs, its output o, the
  * upstream gradient dout, and lse (softmax only; o and lse are unused for the
  * element-wise activations and may be NULL there).  Every row of dq, dk, dv is
- * written (zeros where nothing flows).  dbias must be NULL (the bias/gate
- * gradient is not produced).  The gradient of the definition above:
+ * written (zeros where nothing flows).  dbias (fp32 [H][total_kv], optional,
+ * only with a bias or gate, else GDPA_ERR_INVALID_ARG) receives the gradient of
+ * the bias input: the library zeroes it on the stream, then every key's sum
+ * over its sample's queries is added (keys no query sees stay 0).  The
+ * gradient of the definition above:
  *   dV_j = sum_i p_ij dO_i,  dP_ij = dO_i . V_j,
  *   dS_ij = p_ij (dP_ij - dO_i . O_i) (softmax)  or  dP_ij * phi'(s_ij),
- *   dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i.
+ *   dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i,
+ *   dbias_hj = sum_i dS_ij (additive bias),
+ *   dG_hj = sum_i dS_ij (1 - sigma(G_hj)) (gate, beta = log sigma(G); the gate
+ *   gradient Kunlun reproduction notes, "Core equations", leaves implied).
  * The pages ask that the fused backward avoid materialising large
  * intermediates (Kunlun paper review §2.3, Fig. 2 discussion). */
 GDPA_API gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k,

@@ -252,8 +252,10 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
                             void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
   gdpa_status_t st = check_params(p);
   if (st != GDPA_OK) return st;
-  if (dbias) return GDPA_ERR_UNSUPPORTED;
   if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
+  // a bias gradient needs a bias; it is fp32 [H][total_kv]
+  if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
+  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 3u)) return GDPA_ERR_INVALID_ARG;
   const bool softmax = p->phi == GDPA_PHI_SOFTMAX;
   if (p->total_q > 0 && (!q || !dout || !dq || (softmax && (!o || !lse))))
     return GDPA_ERR_INVALID_ARG;
@@ -281,6 +283,11 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
                                   p->window_right, tile_start, order, info, eff_max_q(p),
                                   eff_max_kv(p), status, s);
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  if (dbias && p->total_kv > 0) {
+    // the kernel adds each key's two column-half sums into it
+    e = cudaMemsetAsync(dbias, 0, sizeof(float) * (size_t)p->H * (size_t)p->total_kv, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
   if (p->B == 0 || (p->total_q == 0 && p->total_kv == 0)) return GDPA_OK;
   if (softmax && p->total_q > 0) {
     e = launch_bwd_preprocess(static_cast<const __nv_bfloat16*>(o),
@@ -316,6 +323,7 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   a.dq = static_cast<__nv_bfloat16*>(dq);
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dbias = dbias;
   a.dq_scratch = scratch;
   a.status = status;
   a.total_q = p->total_q;

@@ -36,8 +36,8 @@ namespace {
 
 constexpr int kBwdThreads = 384;
 constexpr int kRegsLaunch = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int kRegsControl = 96;   // warpgroup 0
-constexpr int kRegsPhi = 200;      // warpgroups 1 and 2
+constexpr int kRegsControl = 88;   // warpgroup 0
+constexpr int kRegsPhi = 208;      // warpgroups 1 and 2
 static_assert(128 * kRegsControl + 256 * kRegsPhi <= kBwdThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 constexpr float kLog2eB = 1.4426950408889634f;
@@ -362,19 +362,6 @@ __device__ __forceinline__ void tmem_row(uint32_t taddr, float (&out)[NCOL]) {
   }
 }
 
-template <int N>
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&v)[N], float mul) {
-#pragma unroll
-  for (int e = 0; e < N; e += 8) {
-    uint4 w;
-    w.x = pack_bf16x2(v[e + 0] * mul, v[e + 1] * mul);
-    w.y = pack_bf16x2(v[e + 2] * mul, v[e + 3] * mul);
-    w.z = pack_bf16x2(v[e + 4] * mul, v[e + 5] * mul);
-    w.w = pack_bf16x2(v[e + 6] * mul, v[e + 7] * mul);
-    *reinterpret_cast<uint4*>(dst + e) = w;
-  }
-}
-
 // ------------------------------------------------------------------ phi warpgroups
 template <class C, int PHI>
 __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
@@ -397,6 +384,8 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
     if (!__all_sync(0xffffffffu, ok_)) return false;                                   \
   } while (0)
 
+  int64_t pre_idx = -1;  // bias element fetched ahead (pre_val), or -1
+  float pre_val = 0.f;
   UnitStream units(a.info, a.H, a.n_units);
   BUnit t;
   while (units.next(t)) {
@@ -416,17 +405,31 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
       }
     }
     float beta = 0.f;
+    float graw = 0.f;  // this key's raw bias (gate) value
+    float dsum = 0.f;  // this key's sum of dS over this warpgroup's query columns
     bool ok = for_each_pair(
         t, a.wl, a.wr,
         [&](int kb, int mt, bool first, bool last) -> bool {
           const int key = kb * C::BN + r;   // this thread's key (S^T row)
+          if (first) dsum = 0.f;
           if (first && a.bias_kind != 0) {
+            // this key block's raw bias, fetched one key block ahead
+            float gv = 0.f;
+            const int64_t gi = key < t.Lk ? (int64_t)t.h * a.total_kv + t.k0 + key : -1;
+            if (gi >= 0) gv = gi == pre_idx ? pre_val : a.bias[gi];
             beta = 0.f;
-            if (key < t.Lk) {
-              const float gv = a.bias[(int64_t)t.h * a.total_kv + t.k0 + key];
-              beta = a.bias_kind == 2 ? fminf(gv, 0.f) - log1pf(__expf(-fabsf(gv))) : gv;
-            }
+            if (gi >= 0) beta = a.bias_kind == 2 ? fminf(gv, 0.f) - log1pf(__expf(-fabsf(gv))) : gv;
+            graw = gv;
             if (SOFTMAX) beta *= kLog2eB;
+            // the next key block of this unit, else the next unit's first
+            pre_idx = -1;
+            if ((kb + 1) * C::BN < t.Lk) {
+              if ((kb + 1) * C::BN + r < t.Lk) pre_idx = gi + C::BN;
+            } else {
+              BUnit nt;
+              if (units.peek(nt) && r < nt.Lk) pre_idx = (int64_t)nt.h * a.total_kv + nt.k0 + r;
+            }
+            if (pre_idx >= 0) pre_val = a.bias[pre_idx];
           }
           const int m0 = mt * kBlockM;
           const int rs = ri & 1;
@@ -477,6 +480,7 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
               }
               s[e] = vis ? p : 0.f;
               dp[e] = vis ? ds : 0.f;
+              dsum += dp[e];
             }
             // P^T row -> TMEM, two bf16 per column, into this warpgroup's own dP^T
             // columns that have already been read: queries 64g+32ch.. at column
@@ -597,6 +601,13 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
           }
           if (last) {
             // dK, dV of this key block: thread = key row, columns [g*D/2, (g+1)*D/2)
+            if (a.dbias && key < t.Lk) {
+              // d beta_j = sum_i dS_ij; for the gate beta = log sigma(G), whose
+              // derivative is 1 - sigma(G) = 1 / (1 + e^G).  The two warpgroups'
+              // halves meet in a zeroed element: either order gives the same sum.
+              const float fac = a.bias_kind == 2 ? 1.f / (1.f + __expf(graw)) : 1.f;
+              atomicAdd(a.dbias + (int64_t)t.h * a.total_kv + t.k0 + key, dsum * fac);
+            }
             BWD_WAIT(C::B_DKVFULL, bi & 1, 0x1400 + C::B_DKVFULL);
             ++bi;
             tc_fence_after();
@@ -605,12 +616,39 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
             tmem_row<HALF_D>(tmem + tl + C::T_DV + g * HALF_D, dvv);
             tc_fence_before();
             mbar_arrive(sm.bar(C::B_DKVEMPTY));
-            if (key < t.Lk) {
-              const int64_t row = ((int64_t)(t.k0 + key) * a.H + t.h) * C::D + g * HALF_D;
-              store_row_bf16<HALF_D>(a.dk + row, dkv, a.scale);
-              store_row_bf16<HALF_D>(a.dv + row, dvv, 1.f);
+            // Each half row goes through this warp's own dS^T rows (free: every MMA
+            // that read dS^T has completed), then out as whole row segments, so a
+            // warp's store covers full 128-byte lines instead of one 16-byte piece
+            // of 32 rows 2 KB apart.
+            constexpr int CPR = HALF_D * 2 / 16;          // 16-byte chunks per half row
+            constexpr int SWM = (CPR >= 8 ? 8 : CPR) - 1;
+            const uint32_t stage = sm.dst() + g * (128 * 128) + wq * 32 * 128;
+            const int wkey = kb * C::BN + wq * 32;        // first key of this warp
+#pragma unroll
+            for (int tsel = 0; tsel < 2; ++tsel) {
+              const float mul = tsel == 0 ? a.scale : 1.f;
+#pragma unroll
+              for (int c = 0; c < CPR; ++c) {
+                const float* v8 = (tsel == 0 ? dkv : dvv) + 8 * c;
+                st_shared_v4(stage + lane * 128 + ((c ^ (lane & SWM)) << 4),
+                             pack_bf16x2(v8[0] * mul, v8[1] * mul), pack_bf16x2(v8[2] * mul, v8[3] * mul),
+                             pack_bf16x2(v8[4] * mul, v8[5] * mul), pack_bf16x2(v8[6] * mul, v8[7] * mul));
+              }
+              __syncwarp();
+              __nv_bfloat16* dst = tsel == 0 ? a.dk : a.dv;
+#pragma unroll 1
+              for (int it = 0; it < CPR; ++it) {
+                const int lin = it * 32 + lane;
+                const int j = lin / CPR, c = lin % CPR;   // row of this warp, chunk
+                const uint4 v = ld_shared_v4(stage + j * 128 + ((c ^ (j & SWM)) << 4));
+                if (wkey + j < t.Lk)
+                  *reinterpret_cast<uint4*>(dst + ((int64_t)(t.k0 + wkey + j) * a.H + t.h) * C::D +
+                                            g * HALF_D + c * 8) = v;
+              }
+              __syncwarp();
             }
           }
+
           return true;
         },
         [&](int kb) -> bool {
@@ -683,7 +721,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   // Registers: the launch gives 384 x 168; warpgroup 0 (producer, MMA issuer,
   // allocator, row loader) needs few, the two phi warpgroups take the rest:
-  // 128 x 96 + 256 x 200 = 63488 <= 64512.  Each budget is set inside its own
+  // 128 x 88 + 256 x 208 = 64512.  Each budget is set inside its own
   // branch so the compiler allocates each role's code against it.
   if (warp < 4) {
     setmaxnreg_dec<kRegsControl>();

@@ -57,6 +57,7 @@ struct BwdArgs {
   __nv_bfloat16* dq;        // [total_q][H][D]
   __nv_bfloat16* dk;        // [total_kv][H][D]
   __nv_bfloat16* dv;        // [total_kv][H][D]
+  float* dbias;             // [H][total_kv], zeroed by the launcher, or nullptr
   float* dq_scratch;        // grid x slot_rows x D
   DeviceStatus* status;
   int64_t total_q, total_kv;

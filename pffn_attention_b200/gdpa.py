@@ -191,8 +191,9 @@ def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1
 
 def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=1.0,
              window=(-1, -1), bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0,
-             dq=None, dk=None, dv=None, workspace=None, stream=None, params=None):
-    """dQ, dK, dV on the device (bf16, shapes of q, k, v)."""
+             dq=None, dk=None, dv=None, dbias=None, workspace=None, stream=None, params=None):
+    """dQ, dK, dV on the device (bf16, shapes of q, k, v).  With a bias or gate,
+    pass dbias (fp32 [H, total_kv]) to also receive the bias gradient."""
     import torch
     total_q, H, D = q.shape
     total_kv = k.shape[0]
@@ -207,7 +208,8 @@ def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=
         workspace = workspace_for(p, True, q.device)
     rc = gdpa_backward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                        _ptr(q_offsets), _ptr(kv_offsets), _ptr(bias), _ptr(dq), _ptr(dk),
-                       _ptr(dv), None, _ptr(workspace), workspace.numel(), _stream(stream))
+                       _ptr(dv), _ptr(dbias), _ptr(workspace), workspace.numel(),
+                       _stream(stream))
     _check(rc, "gdpa_backward")
     return dq, dk, dv, workspace
 

@@ -25,7 +25,8 @@ def to_np(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def compare(name, got, ref, rel_l2=REL_L2, max_abs=MAX_ABS):
+def compare(name, got, ref, rel_l2=REL_L2, max_abs=MAX_ABS, bf16_out=True):
+    """bf16_out=False for fp32 outputs (the bias gradient): no half-ulp allowance."""
     got = to_np(got) if torch.is_tensor(got) else np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -34,7 +35,8 @@ def compare(name, got, ref, rel_l2=REL_L2, max_abs=MAX_ABS):
     nref = np.linalg.norm(ref)
     rel = np.linalg.norm(err) / nref if nref > 0 else np.linalg.norm(err)
     mx = float(np.abs(err).max()) if err.size else 0.0
-    excess = float((np.abs(err) - bf16_half_ulp(ref)).max()) if err.size else 0.0
+    allow = bf16_half_ulp(ref) if bf16_out else 0.0
+    excess = float((np.abs(err) - allow).max()) if err.size else 0.0
     assert rel <= rel_l2 and excess <= max_abs, (
         f"{name}: rel_l2={rel:.3e} max_abs={mx:.3e} beyond_half_ulp={excess:.3e}")
     return rel, mx

@@ -76,6 +76,11 @@ def test_null_and_unaligned_pointers_rejected(lib):
                              None) == 1
     assert lib.gdpa_forward(None, None, None, None, None, None, None, None, None, None, 0,
                             None) == 1
+    # a bias gradient without a bias, and an unaligned bias gradient
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert gdpa.gdpa_backward(p, *args, None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert gdpa.gdpa_backward(pb, *args, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, 1 << 20,
+                              None) == 1
 
 
 def test_workspace_size_grows_with_problem(lib):

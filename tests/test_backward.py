@@ -28,19 +28,35 @@ def gpu_fwd_bwd(gdpa, w):
     dq = torch.full_like(q, float("nan"))
     dk = torch.full_like(k, float("nan"))
     dv = torch.full_like(v, float("nan"))
-    dq, dk, dv, wsb = gdpa.backward(q, k, v, o, do, lse, qo, ko, dq=dq, dk=dk, dv=dv, **kw)
+    # with a bias or gate, its gradient too (NaN-filled: every element is written)
+    dbias = (torch.full((w.H, w.total_kv), float("nan"), dtype=torch.float32, device=dev)
+             if w.bias is not None else None)
+    dq, dk, dv, wsb = gdpa.backward(q, k, v, o, do, lse, qo, ko, dq=dq, dk=dk, dv=dv,
+                                    dbias=dbias, **kw)
     assert gdpa.device_status(wsb) == 0
     torch.cuda.synchronize()
-    return o, dq, dk, dv
+    return o, dq, dk, dv, dbias
 
 
 def check_backward(gdpa, w):
-    _, dq, dk, dv = gpu_fwd_bwd(gdpa, w)
-    rdq, rdk, rdv, _ = oracle.backward_workload(w)
+    _, dq, dk, dv, dbias = gpu_fwd_bwd(gdpa, w)
+    rdq, rdk, rdv, rdb = oracle.backward_workload(w)
     compare("dQ", dq, rdq)
     compare("dK", dk, rdk)
     compare("dV", dv, rdv)
+    if dbias is not None:
+        compare_dbias(dbias, rdb)
     return dq, dk, dv
+
+
+def compare_dbias(got, ref):
+    """The bias gradient is fp32: no output rounding, but each key sums dS over
+    up to a sample's queries, and dS uses delta = dO . O with the forward's bf16
+    O (relative error up to 2^-9 of |delta|), so the max abs bound scales with
+    the tensor's magnitude; relative L2 stays <= 1e-2."""
+    ref = np.asarray(ref, np.float64)
+    scale = max(1.0, float(np.abs(ref).max())) if ref.size else 1.0
+    compare("dbias", got, ref, max_abs=3e-2 * scale, bf16_out=False)
 
 
 def test_gated_training_step_parity(cuda_lib):
@@ -102,7 +118,7 @@ def test_repeat_calls_bit_identical(cuda_lib):
     a = gpu_fwd_bwd(cuda_lib, w)
     b = gpu_fwd_bwd(cuda_lib, w)
     for x, y in zip(a, b):
-        assert torch.equal(x, y)
+        assert torch.equal(x, y)  # dbias too: its two adds per key commute exactly
 
 
 @pytest.mark.slow
@@ -110,14 +126,14 @@ def test_full_size_gated_training_sampled(cuda_lib):
     """Full gated training workload on the GPU; a sample of it checked against
     the oracle (samples are independent, so a subset is an exact sub-problem)."""
     w = make_workload(5, device="cuda")
-    _, dq, dk, dv = gpu_fwd_bwd(cuda_lib, w)
+    _, dq, dk, dv, dbias = gpu_fwd_bwd(cuda_lib, w)
     rng = np.random.default_rng(5)
     picks = sorted({0, w.B - 1, int(np.argmax(w.q_lens)), int(np.argmin(w.q_lens)),
                     *rng.choice(w.B, 4, replace=False).tolist()})
     sub = subset(w, picks)
     for name in ("q", "k", "v", "dout", "bias"):
         setattr(sub, name, getattr(sub, name).cpu())
-    rdq, rdk, rdv, _ = oracle.backward_workload(sub)
+    rdq, rdk, rdv, rdb = oracle.backward_workload(sub)
     qrows = torch.tensor(np.concatenate([np.arange(w.q_offsets[b], w.q_offsets[b + 1])
                                          for b in picks]), device="cuda")
     krows = torch.tensor(np.concatenate([np.arange(w.kv_offsets[b], w.kv_offsets[b + 1])
@@ -125,3 +141,34 @@ def test_full_size_gated_training_sampled(cuda_lib):
     compare("dQ", dq[qrows], rdq)
     compare("dK", dk[krows], rdk)
     compare("dV", dv[krows], rdv)
+    compare_dbias(dbias[:, krows], rdb)
+
+
+# -------------------------------------------------- bias / gate gradient
+@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU])
+@pytest.mark.parametrize("bias_kind", [BIAS_ADD, BIAS_GATE])
+@pytest.mark.parametrize("window", [(-1, -1), (127, 0)])
+def test_bias_gradient(cuda_lib, phi, bias_kind, window):
+    """d bias_j = sum_i dS_ij (add) and dG_j = (1 - sigma(G_j)) sum_i dS_ij (gate),
+    over samples with one and several key blocks, ragged tails, a key block
+    beyond every query's band (its keys get exactly 0) and an empty sample."""
+    ql = [1, 130, 300, 0, 64]
+    kl = [1, 129, 300, 50, 500]
+    if phi == PHI_SOFTMAX:
+        w = make_workload(5, seed=250 + bias_kind, q_lens=ql, kv_lens=kl, H=3, bias=bias_kind,
+                          window=window)
+    else:
+        # SiLU's P is unnormalised and an N(0, 1) bias widens the scores; dO is
+        # scaled so bf16 rounding of P before the dV MMA stays inside the bound
+        ql = [1, 130, 200, 0, 64]
+        w = make_workload(2, seed=260 + bias_kind, q_lens=ql, kv_lens=kl, H=3, D=128,
+                          phi=phi, scale=1.0, kv_std=1.0 / np.sqrt(128), bias=bias_kind,
+                          window=window, with_dout=True, dout_std=0.125)
+    check_backward(cuda_lib, w)
+    if window == (127, 0):
+        # sample 4 (64 queries, 500 keys): query i sees keys [i - 127, i], so
+        # keys 64.. are outside every band (partly inside a processed key block)
+        _, _, _, _, dbias = gpu_fwd_bwd(cuda_lib, w)
+        k0 = int(w.kv_offsets[4])
+        assert torch.all(dbias[:, k0 + 64:k0 + 500] == 0)
+        assert torch.all(dbias[:, int(w.kv_offsets[3]):int(w.kv_offsets[4])] == 0)
