@@ -9,7 +9,8 @@
  *
  *     O = phi(scale * Q K^T + beta) V
  *
- * where phi is an element-wise activation (SiLU, reproducing act(X W1) W2) or
+ * where phi is an element-wise activation (SiLU, reproducing act(X W1) W2, or
+ * GELU, the element-wise example of the Kunlun paper review, §2.3 "GDPA") or
  * a row softmax (pooling, cross-attention and sliding-window self-attention),
  * and beta is an optional per-key additive bias, or the gate log sigmoid(G)
  * of the Kunlun reproduction notes ("Core equations").  The optional band
@@ -70,7 +71,7 @@ typedef enum {
   GDPA_ERR_DEVICE_CHECK = 6  /* device: a sample is longer than max_seqlen_q / _kv */
 } gdpa_status_t;
 
-enum { GDPA_PHI_SILU = 0, GDPA_PHI_SOFTMAX = 1, GDPA_PHI_IDENTITY = 2 };
+enum { GDPA_PHI_SILU = 0, GDPA_PHI_SOFTMAX = 1, GDPA_PHI_IDENTITY = 2, GDPA_PHI_GELU = 3 };
 enum { GDPA_BIAS_NONE = 0, GDPA_BIAS_ADD = 1, GDPA_BIAS_GATE = 2 };
 
 typedef struct {
@@ -81,7 +82,8 @@ typedef struct {
   int64_t total_kv;   /* kv_offsets[B] */
   int max_seqlen_q;   /* upper bound on any sample's query length; 0 = total_q */
   int max_seqlen_kv;  /* upper bound on any sample's key length;   0 = total_kv */
-  int phi;            /* GDPA_PHI_* : SiLU x*sigmoid(x), row softmax, or identity */
+  int phi;            /* GDPA_PHI_* : SiLU x*sigmoid(x), row softmax, identity, or
+                         GELU x*Phi(x) (Phi the standard normal distribution) */
   float scale;        /* multiplies QK^T before beta is added (= 1/tau) */
   int window_left;    /* -1 = unbounded */
   int window_right;   /* -1 = unbounded */

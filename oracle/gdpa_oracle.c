@@ -12,7 +12,9 @@
  *     vis(i,j) = (wl < 0 || j >= i - wl) && (wr < 0 || j <= i + wr)
  *     s_ij     = scale * sum_d Q[i,h,d] K[j,h,d] + beta_hj
  *     beta_hj  = 0 | bias[h][j] | log sigmoid(G[h][j])      (none/add/gate)
- *     p_ij     = silu(s_ij) | s_ij | softmax_j(s_ij)  over visible j, else 0
+ *     p_ij     = silu(s_ij) | s_ij | softmax_j(s_ij) | gelu(s_ij)
+ *                over visible j, else 0;  gelu(x) = x Phi(x), Phi the standard
+ *                normal distribution function, 0.5 (1 + erf(x / sqrt 2))
  *     O_i      = sum_j p_ij V_j
  *     LSE_i    = log sum_{visible j} exp(s_ij)               (softmax only)
  *
@@ -20,8 +22,8 @@
  *   - Kunlun paper review (liuzhao09.github.io), §2.3 "GDPA" and Fig. 2:
  *     the personalised FFN recast as attention with the sequence as query and
  *     context-generated K, V; step order QK^T / tau, then an activation that
- *     may be element-wise (non-softmax), then Attn x V; tau is a free
- *     temperature, passed here as scale = 1/tau.
+ *     may be element-wise (non-softmax), GELU named as the example, then
+ *     Attn x V; tau is a free temperature, passed here as scale = 1/tau.
  *   - Kunlun reproduction notes (daiwk.github.io), "Core equations":
  *     A = softmax(QK^T / sqrt(d) + log sigma(G)) -- the gate enters the scores
  *     additively as log sigma(G), after the scaling.
@@ -38,6 +40,7 @@
  *   dS_ij = p_ij (dP_ij - delta_i), delta_i = sum_j p_ij dP_ij       (softmax)
  *         = dP_ij (sigma(s) + s sigma(s)(1 - sigma(s)))              (SiLU)
  *         = dP_ij                                                    (identity)
+ *         = dP_ij (Phi(s) + s phi(s)), phi(x) = exp(-x^2/2) / sqrt(2 pi)  (GELU)
  *   dQ_i  = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i
  *   dbias_hj = sum_i dS_ij  (add)  or  sum_i dS_ij (1 - sigma(G_hj))  (gate)
  *
@@ -54,7 +57,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_PHI_SILU = 0, ORACLE_PHI_SOFTMAX = 1, ORACLE_PHI_IDENTITY = 2 };
+enum { ORACLE_PHI_SILU = 0, ORACLE_PHI_SOFTMAX = 1, ORACLE_PHI_IDENTITY = 2, ORACLE_PHI_GELU = 3 };
 enum { ORACLE_BIAS_NONE = 0, ORACLE_BIAS_ADD = 1, ORACLE_BIAS_GATE = 2 };
 
 typedef struct {
@@ -78,6 +81,12 @@ static double sigmoid(double x) {
   return e / (1.0 + e);
 }
 
+/* Standard normal distribution function and density (GELU and its derivative). */
+static double normal_cdf(double x) { return 0.5 * (1.0 + erf(x / sqrt(2.0))); }
+static double normal_pdf(double x) {
+  return exp(-0.5 * x * x) / sqrt(2.0 * 3.14159265358979323846);
+}
+
 /* log sigma(g), written so that neither branch overflows. */
 static double log_sigmoid(double g) {
   if (g >= 0.0) return -log1p(exp(-g));
@@ -94,7 +103,7 @@ static double score_bias(const oracle_params* p, const double* bias, int h,
 static int check_params(const oracle_params* p, const int32_t* qo,
                         const int32_t* ko) {
   if (!p || p->B < 0 || p->H <= 0 || p->D <= 0) return 1;
-  if (p->phi < 0 || p->phi > 2 || p->bias_kind < 0 || p->bias_kind > 2) return 1;
+  if (p->phi < 0 || p->phi > 3 || p->bias_kind < 0 || p->bias_kind > 2) return 1;
   if (qo[0] != 0 || ko[0] != 0) return 1;
   for (int b = 0; b < p->B; ++b)
     if (qo[b + 1] < qo[b] || ko[b + 1] < ko[b]) return 1;
@@ -137,7 +146,12 @@ static double row_probs(const oracle_params* p, const double* s,
   }
   for (int64_t j = 0; j < Lk; ++j) {
     if (!vis[j]) { pr[j] = 0.0; continue; }
-    pr[j] = (p->phi == ORACLE_PHI_SILU) ? s[j] * sigmoid(s[j]) : s[j];
+    if (p->phi == ORACLE_PHI_SILU)
+      pr[j] = s[j] * sigmoid(s[j]);
+    else if (p->phi == ORACLE_PHI_GELU)
+      pr[j] = s[j] * normal_cdf(s[j]);
+    else
+      pr[j] = s[j];
   }
   return 0.0;
 }
@@ -247,6 +261,8 @@ int gdpa_oracle_backward(const oracle_params* p, const double* q, const double* 
           } else if (p->phi == ORACLE_PHI_SILU) {
             double sg = sigmoid(s[j]);
             ds[j] = dp[j] * (sg + s[j] * sg * (1.0 - sg));
+          } else if (p->phi == ORACLE_PHI_GELU) {
+            ds[j] = dp[j] * (normal_cdf(s[j]) + s[j] * normal_pdf(s[j]));
           } else {
             ds[j] = dp[j];
           }

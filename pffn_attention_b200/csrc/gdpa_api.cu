@@ -63,7 +63,7 @@ gdpa_status_t check_params(const gdpa_params_t* p) {
   if (!std::isfinite(p->scale)) return GDPA_ERR_INVALID_ARG;
   if (p->wait_timeout_us < 0) return GDPA_ERR_INVALID_ARG;
   if (p->D != 32 && p->D != 64 && p->D != 128) return GDPA_ERR_UNSUPPORTED;
-  if (p->phi < 0 || p->phi > 2) return GDPA_ERR_UNSUPPORTED;
+  if (p->phi < 0 || p->phi > 3) return GDPA_ERR_UNSUPPORTED;
   if (p->bias_kind < 0 || p->bias_kind > 2) return GDPA_ERR_UNSUPPORTED;
   if (p->B > kMaxSortBatch) return GDPA_ERR_UNSUPPORTED;
   if ((int64_t)p->H * p->B >= (int64_t(1) << 31)) return GDPA_ERR_UNSUPPORTED;

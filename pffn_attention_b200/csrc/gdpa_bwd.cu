@@ -41,6 +41,7 @@ constexpr int kRegsPhi = 208;      // warpgroups 1 and 2
 static_assert(128 * kRegsControl + 256 * kRegsPhi <= kBwdThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 constexpr float kLog2eB = 1.4426950408889634f;
+constexpr float kInvSqrt2Pi = 0.3989422804014327f;  // 1 / sqrt(2 pi)
 
 template <int D_>
 struct BwdCfg {
@@ -474,6 +475,12 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
                 const float sg = fmaf(0.5f, th, 0.5f);       // sigmoid(x)
                 p = x * sg;
                 ds = dp[e] * fmaf(x * sg, 1.f - sg, sg);      // sg + x sg (1 - sg)
+              } else if (PHI == 3) {
+                // gelu(x) = x Phi(x); gelu'(x) = Phi(x) + x phi(x), phi the
+                // standard normal density exp(-x^2 / 2) / sqrt(2 pi)
+                const float cdf = normcdff(x);
+                p = x * cdf;
+                ds = dp[e] * fmaf(x, kInvSqrt2Pi * __expf(-0.5f * x * x), cdf);
               } else {
                 p = x;
                 ds = dp[e];
@@ -830,6 +837,7 @@ cudaError_t launch_backward(const BwdArgs& a, int D, const CUtensorMap& tq, cons
   if (D == D_) {                                                               \
     if (a.phi == 1) return launch_bwd_one<D_, 1>(a, tq, tk, tv, tdo, grid, stream); \
     if (a.phi == 0) return launch_bwd_one<D_, 0>(a, tq, tk, tv, tdo, grid, stream); \
+    if (a.phi == 3) return launch_bwd_one<D_, 3>(a, tq, tk, tv, tdo, grid, stream); \
     return launch_bwd_one<D_, 2>(a, tq, tk, tv, tdo, grid, stream);             \
   }
   GDPA_BWD_CASE(32)

@@ -483,6 +483,7 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
   const uint32_t tslot = tmem + ((uint32_t)(wq * 32) << 16) + s * C::TMEM_SLOT;
   const bool has_bias = a.bias_kind != 0;
   const bool identity = a.phi == 2;
+  const bool gelu = a.phi == 3;
   const float sc = SOFTMAX ? a.scale * kLog2e : a.scale;
   uint32_t nsb = 0, tq = 0, bc = 0;  // S blocks, non-empty tiles, bias blocks of the slot
 
@@ -595,6 +596,13 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
             v[e] = __float_as_uint(p0);
             v[e + 1] = __float_as_uint(p1);
             ps2[(e >> 1) & 1] = f2_add(ps2[(e >> 1) & 1], f2_pack(p0, p1));
+          }
+        } else if (gelu) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            // gelu(x) = x Phi(x) (masked columns: gelu(0) = 0)
+            const float x = __uint_as_float(v[e]);
+            v[e] = __float_as_uint(x * normcdff(x));
           }
         } else if (!identity) {
 #pragma unroll

@@ -20,7 +20,7 @@ GDPA_OK = 0
 STATUS_NAMES = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
                 3: "GDPA_ERR_WORKSPACE", 4: "GDPA_ERR_CUDA", 5: "GDPA_ERR_TIMEOUT",
                 6: "GDPA_ERR_DEVICE_CHECK"}
-PHI = {"silu": 0, "softmax": 1, "identity": 2}
+PHI = {"silu": 0, "softmax": 1, "identity": 2, "gelu": 3}
 BIAS = {"none": 0, "add": 1, "gate": 2}
 
 EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",

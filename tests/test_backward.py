@@ -9,7 +9,8 @@ import torch
 
 import oracle
 from parity import compare
-from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX,
+from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_GELU, PHI_IDENTITY, PHI_SILU,
+                       PHI_SOFTMAX,
                        make_workload, subset)
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +66,7 @@ def test_gated_training_step_parity(cuda_lib):
 
 
 @pytest.mark.parametrize("D", [32, 64, 128])
-@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU, PHI_IDENTITY])
+@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU, PHI_IDENTITY, PHI_GELU])
 def test_head_dims_and_activations(cuda_lib, D, phi):
     ql = [1, 127, 128, 129, 250]
     kl = [40, 1, 127, 200, 129]
@@ -145,7 +146,7 @@ def test_full_size_gated_training_sampled(cuda_lib):
 
 
 # -------------------------------------------------- bias / gate gradient
-@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU])
+@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU, PHI_GELU])
 @pytest.mark.parametrize("bias_kind", [BIAS_ADD, BIAS_GATE])
 @pytest.mark.parametrize("window", [(-1, -1), (127, 0)])
 def test_bias_gradient(cuda_lib, phi, bias_kind, window):

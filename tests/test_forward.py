@@ -5,7 +5,8 @@ import torch
 
 import oracle
 from parity import compare, compare_lse
-from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX,
+from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_GELU, PHI_IDENTITY, PHI_SILU,
+                       PHI_SOFTMAX,
                        make_workload, subset)
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +45,7 @@ def test_workload_parity(cuda_lib, cfg, B):
 
 # -------------------------------------------------- shapes, activations, biases
 @pytest.mark.parametrize("D", [32, 64, 128])
-@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY])
+@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY, PHI_GELU])
 @pytest.mark.parametrize("kv_len", [40, 200])  # one and two 128-key blocks
 def test_head_dims_and_activations(cuda_lib, D, phi, kv_len):
     ql = [1, 127, 128, 129, 300]

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_IDENTITY, PHI_SILU,
+from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_GELU, PHI_IDENTITY, PHI_SILU,
                        PHI_SOFTMAX, offsets_from_lengths)
 
 
@@ -53,6 +53,29 @@ def test_pffn_two_matmul_form():
             W1 = k[ko[b]:ko[b + 1], h, :].T          # D x Lk
             W2 = v[ko[b]:ko[b + 1], h, :]            # Lk x D
             ref = silu_np(scale * (S @ W1)) @ W2
+            np.testing.assert_allclose(o[qo[b]:qo[b + 1], h, :], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_gelu_two_matmul_form_matches_torch():
+    """GELU GDPA (the pages' example of an element-wise activation in place of
+    softmax, Kunlun paper review §2.3) equals gelu(scale S W1) W2 with torch's
+    exact (erf) GELU in fp64 and numpy matmuls, with a gate and a band."""
+    rng = np.random.default_rng(16)
+    q, k, v, qo, ko = rand_problem(rng, [6, 13, 1], [9, 4, 7], H=2, D=5)
+    g = rng.standard_normal((2, ko[-1]))
+    scale, (wl, wr) = 0.61, (3, 1)
+    o, _ = oracle.forward(q, k, v, qo, ko, phi=PHI_GELU, scale=scale, window=(wl, wr),
+                          bias=g, bias_kind=BIAS_GATE)
+    for b in range(3):
+        Lq, Lk = qo[b + 1] - qo[b], ko[b + 1] - ko[b]
+        vis = band_mask(Lq, Lk, wl, wr)
+        for h in range(2):
+            S = q[qo[b]:qo[b + 1], h, :]
+            W1 = k[ko[b]:ko[b + 1], h, :].T
+            W2 = v[ko[b]:ko[b + 1], h, :]
+            gate = torch.nn.functional.logsigmoid(torch.tensor(g[h, ko[b]:ko[b + 1]])).numpy()
+            x = torch.tensor(scale * (S @ W1) + gate[None, :])
+            ref = (torch.nn.functional.gelu(x, approximate="none").numpy() * vis) @ W2
             np.testing.assert_allclose(o[qo[b]:qo[b + 1], h, :], ref, rtol=1e-12, atol=1e-13)
 
 
@@ -324,7 +347,7 @@ def _loss(q, k, v, dout, qo, ko, phi, scale, window, g, bias_kind):
     return float(np.sum(o * dout))
 
 
-@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY])
+@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY, PHI_GELU])
 @pytest.mark.parametrize("bias_kind,window", [(BIAS_NONE, (-1, -1)), (BIAS_ADD, (1, 0)),
                                               (BIAS_GATE, (-1, -1)), (BIAS_GATE, (0, 2))])
 def test_finite_difference_gradients(phi, bias_kind, window):
@@ -352,7 +375,7 @@ def test_finite_difference_gradients(phi, bias_kind, window):
         np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
 
 
-@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX])
+@pytest.mark.parametrize("phi", [PHI_SILU, PHI_SOFTMAX, PHI_GELU])
 def test_backward_matches_torch_autograd(phi):
     """Gradients equal torch autograd (fp64, CPU) of the formula built from
     torch's own softmax / silu / logsigmoid / matmul, with a band and gate."""
@@ -381,6 +404,8 @@ def test_backward_matches_torch_autograd(phi):
             s = 0.45 * Q @ K.T + torch.nn.functional.logsigmoid(tg[h, ko[b]:ko[b + 1]])[None]
             if phi == PHI_SOFTMAX:
                 p = torch.softmax(s.masked_fill(~vis, -math.inf), dim=1)
+            elif phi == PHI_GELU:
+                p = torch.nn.functional.gelu(s, approximate="none") * vis
             else:
                 p = torch.nn.functional.silu(s) * vis
             rows.append(p @ V)

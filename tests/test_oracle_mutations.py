@@ -12,7 +12,8 @@ import pytest
 
 import oracle
 import test_oracle as pins
-from workloads import BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX
+from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_GELU, PHI_IDENTITY, PHI_SILU,
+                       PHI_SOFTMAX)
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdpa_oracle.c")
 
@@ -37,6 +38,11 @@ MUTATIONS = {
     "dq_uses_queries": ("dqi[d] += p->scale * ds[j] * kj[d];", "dqi[d] += p->scale * ds[j] * qi[d];"),
     "gate_grad_sign": ("1.0 - sigmoid(g);", "sigmoid(g);"),
     "dv_uses_dp": ("dvj[d] += pr[j] * doi[d];", "dvj[d] += dp[j] * doi[d];"),
+    # GELU: the tanh approximation instead of erf, and a dropped derivative term
+    "gelu_tanh_approximation": ("return 0.5 * (1.0 + erf(x / sqrt(2.0)));",
+                                "return 0.5 * (1.0 + tanh(0.7978845608 * (x + 0.044715 * x * x * x)));"),
+    "gelu_grad_term_dropped": ("ds[j] = dp[j] * (normal_cdf(s[j]) + s[j] * normal_pdf(s[j]));",
+                               "ds[j] = dp[j] * normal_cdf(s[j]);"),
 }
 
 PIN_CALLS = [
@@ -53,6 +59,8 @@ PIN_CALLS = [
     lambda: pins.test_backward_matches_torch_autograd(PHI_SILU),
     lambda: pins.test_backward_matches_torch_autograd(PHI_SOFTMAX),
     lambda: pins.test_finite_difference_gradients(PHI_IDENTITY, BIAS_NONE, (-1, -1)),
+    lambda: pins.test_gelu_two_matmul_form_matches_torch(),
+    lambda: pins.test_backward_matches_torch_autograd(PHI_GELU),
 ]
 
 

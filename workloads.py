@@ -24,7 +24,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY = 0, 1, 2
+PHI_SILU, PHI_SOFTMAX, PHI_IDENTITY, PHI_GELU = 0, 1, 2, 3
 BIAS_NONE, BIAS_ADD, BIAS_GATE = 0, 1, 2
 
 
