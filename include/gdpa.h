@@ -92,6 +92,10 @@ typedef struct {
                          the bounded-wait path can be tested (returns TIMEOUT);
                          other bits are reserved and ignored */
   int wait_timeout_us;/* bound on any single in-kernel wait; 0 = 2000000 (2 s) */
+  const int32_t* head_phi; /* optional host array of H GDPA_PHI_* values, one per
+                         head (H <= 64); NULL = every head uses phi.  Read during
+                         the call only.  LSE rows of non-softmax heads are not
+                         written. */
 } gdpa_params_t;
 
 /* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward

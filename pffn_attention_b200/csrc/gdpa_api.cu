@@ -64,11 +64,28 @@ gdpa_status_t check_params(const gdpa_params_t* p) {
   if (p->wait_timeout_us < 0) return GDPA_ERR_INVALID_ARG;
   if (p->D != 32 && p->D != 64 && p->D != 128) return GDPA_ERR_UNSUPPORTED;
   if (p->phi < 0 || p->phi > 3) return GDPA_ERR_UNSUPPORTED;
+  if (p->head_phi) {
+    if (p->H > 64) return GDPA_ERR_UNSUPPORTED;
+    for (int h = 0; h < p->H; ++h)
+      if (p->head_phi[h] < 0 || p->head_phi[h] > 3) return GDPA_ERR_UNSUPPORTED;
+  }
   if (p->bias_kind < 0 || p->bias_kind > 2) return GDPA_ERR_UNSUPPORTED;
   if (p->B > kMaxSortBatch) return GDPA_ERR_UNSUPPORTED;
   if ((int64_t)p->H * p->B >= (int64_t(1) << 31)) return GDPA_ERR_UNSUPPORTED;
   return GDPA_OK;
 }
+
+// Heads whose activation is phi (bit h), ~0 for all heads when every head
+// uses p->phi, 0 when none does.
+uint64_t phi_heads(const gdpa_params_t* p, int phi) {
+  if (!p->head_phi) return p->phi == phi ? ~0ull : 0ull;
+  uint64_t m = 0;
+  for (int h = 0; h < p->H; ++h)
+    if (p->head_phi[h] == phi) m |= 1ull << h;
+  return m;
+}
+
+bool any_softmax(const gdpa_params_t* p) { return phi_heads(p, GDPA_PHI_SOFTMAX) != 0; }
 
 int eff_max_q(const gdpa_params_t* p) {
   return p->max_seqlen_q > 0 ? p->max_seqlen_q : (int)p->total_q;
@@ -93,7 +110,7 @@ WorkspaceLayout make_layout(const gdpa_params_t* p, int backward, int sms) {
   off += align256((size_t)std::max(p->B, 1) * 16);
   if (backward) {
     L.delta = off;
-    if (p->phi == GDPA_PHI_SOFTMAX) off += align256((size_t)p->H * (size_t)p->total_q * 4);
+    if (any_softmax(p)) off += align256((size_t)p->H * (size_t)p->total_q * 4);
     L.grid = backward_grid(p, sms);
     L.dq_slot_rows = (std::min(eff_max_q(p), (int)p->total_q) + kBlockM - 1) / kBlockM * kBlockM;
     L.dq_scratch = off;
@@ -225,7 +242,6 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.info = info;
   a.bias = bias;
   a.o = static_cast<__nv_bfloat16*>(o);
-  a.lse = p->phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
   a.status = status;
   a.total_q = p->total_q;
   a.total_kv = p->total_kv;
@@ -241,8 +257,18 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.wr = p->window_right;
   a.debug_flags = p->debug_flags;
   a.timeout_ns = timeout_ns(p);
-  e = launch_forward(a, p->D, block_n, tq, tk, tv, sms, s);
-  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+  // one launch per activation present (a per-head activation vector groups
+  // the heads; each launch walks only its own heads' units)
+  for (int phi = 0; phi <= 3; ++phi) {
+    const uint64_t heads = phi_heads(p, phi);
+    if (!heads) continue;
+    a.phi = phi;
+    a.head_mask = heads;
+    a.lse = phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
+    e = launch_forward(a, p->D, block_n, tq, tk, tv, sms, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
+  return GDPA_OK;
 }
 
 gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k, const void* v,
@@ -256,7 +282,7 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   // a bias gradient needs a bias; it is fp32 [H][total_kv]
   if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
   if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 3u)) return GDPA_ERR_INVALID_ARG;
-  const bool softmax = p->phi == GDPA_PHI_SOFTMAX;
+  const bool softmax = any_softmax(p);
   if (p->total_q > 0 && (!q || !dout || !dq || (softmax && (!o || !lse))))
     return GDPA_ERR_INVALID_ARG;
   if (p->total_kv > 0 && (!k || !v || !dk || !dv)) return GDPA_ERR_INVALID_ARG;
@@ -341,8 +367,15 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   a.wr = p->window_right;
   a.debug_flags = p->debug_flags;
   a.timeout_ns = timeout_ns(p);
-  e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
-  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+  for (int phi = 0; phi <= 3; ++phi) {
+    const uint64_t heads = phi_heads(p, phi);
+    if (!heads) continue;
+    a.phi = phi;
+    a.head_mask = heads;
+    e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
+  return GDPA_OK;
 }
 
 gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {

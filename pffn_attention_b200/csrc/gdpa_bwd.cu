@@ -148,7 +148,7 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
   uint32_t kvi = 0, qi = 0;
-  UnitStream units(a.info, a.H, a.n_units);
+  UnitStream units(a.info, a.H, a.n_units, a.head_mask);
   BUnit t;
   while (units.next(t)) {
     bool ok = for_each_pair(
@@ -210,7 +210,7 @@ __device__ void bwd_mma(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
   constexpr uint32_t id_dq = make_idesc_bf16(kBlockM, C::D, 1, 1);  // dQ
   constexpr uint32_t SBO = 8 * C::PANEL_BYTES;
   uint32_t kvi = 0, qi = 0, pi = 0, dqi = 0, bi = 0;
-  UnitStream units(a.info, a.H, a.n_units);
+  UnitStream units(a.info, a.H, a.n_units, a.head_mask);
   BUnit t;
   while (units.next(t)) {
     bool ok = for_each_pair(
@@ -309,7 +309,7 @@ __device__ void bwd_rows(const BwdArgs& a, const BSmem<C>& sm) {
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
   uint32_t ri = 0;
-  UnitStream units(a.info, a.H, a.n_units);
+  UnitStream units(a.info, a.H, a.n_units, a.head_mask);
   BUnit t;
   while (units.next(t)) {
     bool ok = for_each_pair(
@@ -387,7 +387,7 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
 
   int64_t pre_idx = -1;  // bias element fetched ahead (pre_val), or -1
   float pre_val = 0.f;
-  UnitStream units(a.info, a.H, a.n_units);
+  UnitStream units(a.info, a.H, a.n_units, a.head_mask);
   BUnit t;
   while (units.next(t)) {
     // dQ rows of query tiles that no key block reaches are zero

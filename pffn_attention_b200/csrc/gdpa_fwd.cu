@@ -140,7 +140,8 @@ struct TileWalk {
   uint32_t g, kvi, unit_kv0;
   bool resident, in_unit;
   __device__ explicit TileWalk(const FwdArgs& a)
-      : units(a.info, a.H, a.n_units), t{}, wl(a.wl), wr(a.wr), ntile(0), mt(0), nkb(0), g(0),
+      : units(a.info, a.H, a.n_units, a.head_mask), t{}, wl(a.wl), wr(a.wr), ntile(0), mt(0),
+        nkb(0), g(0),
         kvi(0), unit_kv0(0), resident(false), in_unit(false) {}
   __device__ bool next(FTile& x) {
     for (;;) {

@@ -44,6 +44,7 @@ struct FwdArgs {
   int wl, wr;
   int debug_flags;
   uint64_t timeout_ns;
+  uint64_t head_mask;       // heads this launch computes (bit h), ~0 = all
 };
 
 struct BwdArgs {
@@ -71,6 +72,7 @@ struct BwdArgs {
   int wl, wr;
   int debug_flags;
   uint64_t timeout_ns;
+  uint64_t head_mask;       // heads this launch computes (bit h), ~0 = all
 };
 
 // Launchers (defined next to their kernels).
@@ -100,14 +102,26 @@ struct GdpaUnit {
 struct UnitStream {
   const int4* info;
   int H, n_units, round, u;
+  uint64_t mask;  // heads to walk (bit h); ~0 = all
   int4 nxt;
   __device__ __forceinline__ static int index(int round, int cta, int grid) {
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
   }
-  __device__ __forceinline__ UnitStream(const int4* info_, int H_, int n_units_)
-      : info(info_), H(H_), n_units(n_units_), round(0) {
-    u = index(0, blockIdx.x, gridDim.x);
+  // first unit at or after `round` whose head is walked
+  __device__ __forceinline__ void settle() {
+    for (;;) {
+      u = index(round, blockIdx.x, gridDim.x);
+      if (u >= n_units || mask == ~0ull) break;
+      const int h = u % H;
+      if (h < 64 && ((mask >> h) & 1ull)) break;
+      ++round;
+    }
     nxt = u < n_units ? __ldg(info + u / H) : make_int4(0, 0, 0, 0);
+  }
+  __device__ __forceinline__ UnitStream(const int4* info_, int H_, int n_units_,
+                                        uint64_t mask_ = ~0ull)
+      : info(info_), H(H_), n_units(n_units_), round(0), mask(mask_) {
+    settle();
   }
   // The unit the next call of next() returns, without advancing.
   __device__ __forceinline__ bool peek(GdpaUnit& t) const {
@@ -120,15 +134,9 @@ struct UnitStream {
     return true;
   }
   __device__ __forceinline__ bool next(GdpaUnit& t) {
-    if (u >= n_units) return false;
-    t.h = u % H;
-    t.q0 = nxt.x;
-    t.Lq = nxt.y;
-    t.k0 = nxt.z;
-    t.Lk = nxt.w;
+    if (!peek(t)) return false;
     ++round;
-    u = index(round, blockIdx.x, gridDim.x);
-    if (u < n_units) nxt = __ldg(info + u / H);
+    settle();
     return true;
   }
 };

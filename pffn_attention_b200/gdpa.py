@@ -35,7 +35,8 @@ class gdpa_params_t(ctypes.Structure):
                 ("phi", ctypes.c_int), ("scale", ctypes.c_float),
                 ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
                 ("bias_kind", ctypes.c_int), ("debug_flags", ctypes.c_int),
-                ("wait_timeout_us", ctypes.c_int)]
+                ("wait_timeout_us", ctypes.c_int),
+                ("head_phi", ctypes.POINTER(ctypes.c_int32))]
 
 
 class GdpaError(RuntimeError):
@@ -131,14 +132,30 @@ def gdpa_version() -> int:
 # ----------------------------------------------------------------- torch helpers
 def make_params(B, H, D, total_q, total_kv, *, phi=0, scale=1.0, window=(-1, -1),
                 bias_kind=0, max_seqlen_q=0, max_seqlen_kv=0, debug_flags=0,
-                wait_timeout_us=0) -> gdpa_params_t:
+                wait_timeout_us=0, head_phi=None) -> gdpa_params_t:
+    """head_phi: optional sequence of H activations (names or GDPA_PHI values),
+    one per head; the params object keeps the array alive."""
     if isinstance(phi, str):
         phi = PHI[phi]
     if isinstance(bias_kind, str):
         bias_kind = BIAS[bias_kind]
-    return gdpa_params_t(int(B), int(H), int(D), int(total_q), int(total_kv), int(max_seqlen_q),
-                         int(max_seqlen_kv), int(phi), float(scale), int(window[0]),
-                         int(window[1]), int(bias_kind), int(debug_flags), int(wait_timeout_us))
+    arr = None
+    if head_phi is not None:
+        vals = [PHI[x] if isinstance(x, str) else int(x) for x in head_phi]
+        arr = (ctypes.c_int32 * len(vals))(*vals)
+    p = gdpa_params_t(int(B), int(H), int(D), int(total_q), int(total_kv), int(max_seqlen_q),
+                      int(max_seqlen_kv), int(phi), float(scale), int(window[0]),
+                      int(window[1]), int(bias_kind), int(debug_flags), int(wait_timeout_us),
+                      ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)) if arr is not None
+                      else None)
+    p._head_phi = arr  # owns the array the struct points to
+    return p
+
+
+def _any_softmax(p) -> bool:
+    if p.head_phi:
+        return any(p.head_phi[h] == PHI["softmax"] for h in range(p.H))
+    return p.phi == PHI["softmax"]
 
 
 def _ptr(t) -> Optional[int]:
@@ -167,7 +184,7 @@ def _check(rc: int, where: str):
 
 def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1, -1),
             bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0, out=None, lse=None,
-            workspace=None, stream=None, params=None):
+            workspace=None, stream=None, params=None, head_phi=None):
     """O (and LSE for softmax) on the device.  Inputs are CUDA tensors:
     q [total_q,H,D] bf16, k/v [total_kv,H,D] bf16, offsets int32 [B+1]."""
     import torch
@@ -176,10 +193,10 @@ def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1
     B = q_offsets.numel() - 1
     p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
                               bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
-                              max_seqlen_kv=max_seqlen_kv)
+                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi)
     if out is None:
         out = torch.empty_like(q)
-    if lse is None and p.phi == PHI["softmax"]:
+    if lse is None and _any_softmax(p):
         lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = workspace_for(p, False, q.device)
@@ -191,7 +208,8 @@ def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1
 
 def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=1.0,
              window=(-1, -1), bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0,
-             dq=None, dk=None, dv=None, dbias=None, workspace=None, stream=None, params=None):
+             dq=None, dk=None, dv=None, dbias=None, workspace=None, stream=None, params=None,
+             head_phi=None):
     """dQ, dK, dV on the device (bf16, shapes of q, k, v).  With a bias or gate,
     pass dbias (fp32 [H, total_kv]) to also receive the bias gradient."""
     import torch
@@ -200,7 +218,7 @@ def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=
     B = q_offsets.numel() - 1
     p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
                               bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
-                              max_seqlen_kv=max_seqlen_kv)
+                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

@@ -96,3 +96,15 @@ def test_tile_shape_query(lib):
     for kv in (64, 2000):
         rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=kv))
         assert (rc, bm, bn) == (0, 128, 128)
+
+
+def test_head_phi_validation(lib):
+    """A per-head activation vector: entries must be GDPA_PHI values and H <= 64;
+    a softmax head anywhere makes the backward workspace hold delta."""
+    assert gdpa.gdpa_workspace_size(_params(H=3, head_phi=[0, 1, 9]), 0) == 0
+    assert gdpa.gdpa_workspace_size(_params(H=65, head_phi=[0] * 65), 0) == 0
+    assert gdpa.gdpa_workspace_size(_params(H=65), 0) > 0
+    plain = gdpa.gdpa_workspace_size(_params(H=3, phi=0), 1)
+    mixed = gdpa.gdpa_workspace_size(_params(H=3, phi=0, head_phi=[0, 1, 3]), 1)
+    assert mixed > plain > 0
+    assert gdpa.gdpa_workspace_size(_params(H=3, phi=0, head_phi=[3, 2, 0]), 1) == plain
