@@ -77,7 +77,7 @@ def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
     bwd = 0.0
     if backward:
         bwd = (2.0 * H * D * (tq * 4 + tk * 4)                     # Q, O, dO, dQ; K, V, dK, dV
-               + gate + lse)
+               + 2 * gate + lse)                                    # gate read, its gradient written
     return fwd, bwd
 
 
@@ -206,7 +206,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     training = cfg == 5
     # each rank owns an independent batch of the same distribution
     w = make_workload(cfg, B=args.batch, device=dev, seed=rank_seed(cfg, rank),
-                      with_dout=training)
+                      with_dout=training, **phi_override(args))
     qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
     ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
     p = gdpa.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
@@ -217,6 +217,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ws_f = gdpa.workspace_for(p, False, dev)
     if training:
         dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
+        # a training step also needs the gate's gradient (the gate is an input
+        # computed upstream)
+        dbias = (torch.empty((w.H, w.total_kv), dtype=torch.float32, device=dev)
+                 if w.bias is not None else None)
         ws_b = gdpa.workspace_for(p, True, dev)
     stream = torch.cuda.Stream(device=dev)
     sh = stream.cuda_stream
@@ -234,7 +238,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if training:
             rc = gdpa.gdpa_backward(p, ptr(w.q), ptr(w.k), ptr(w.v), ptr(o), ptr(w.dout), ptr(lse),
                                     ptr(qo), ptr(ko), ptr(w.bias), ptr(dq), ptr(dk), ptr(dv),
-                                    None, ptr(ws_b), ws_b.numel(), sh)
+                                    ptr(dbias), ptr(ws_b), ws_b.numel(), sh)
             if rc:
                 raise gdpa.GdpaError(rc, "gdpa_backward")
         if ev is not None:
@@ -286,7 +290,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     else:
         dom_name, dom_ms, dom_bytes, dom_flops = "gdpa_forward", fwd_ms, b_fwd, f_fwd
     achieved_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = measured_traffic(dom_name, w.B)
+    # the committed capture is of the default workload; other runs report none
+    traffic = (measured_traffic(dom_name, w.B)
+               if args.workload == DEFAULT_WORKLOAD and not args.phi else None)
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
                 "traffic": None if traffic is None else round(traffic / 1e9, 3),
@@ -309,7 +315,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "B": w.B, "H": w.H, "D": w.D,
                    "global_batch": w.B * world, "seq_len": f"q U[256,1024] / kv 256"
                    if cfg == 5 else "see workload", "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (no flush)"},
+                   "l2": "inputs larger than L2 (no flush)",
+                   "phi": {v: k for k, v in PHI_NAMES.items()}[w.phi],
+                   "gate_grad": bool(training and w.bias is not None)},
         "pct_of_peak": {"measured_burst": round(value / world / peaks["bf16_tflops"], 4),
                         "measured_sustained": round(value / world
                                                     / peaks["bf16_tflops_sustained"], 4),
@@ -350,6 +358,8 @@ def run_e2e(args, w, p, qo, ko, training, dev, world):
     if training:
         outs.update(dq=torch.empty_like(dev_in["q"]), dk=torch.empty_like(dev_in["k"]),
                     dv=torch.empty_like(dev_in["v"]))
+        if w.bias is not None:
+            outs["dbias"] = torch.empty((w.H, w.total_kv), dtype=torch.float32, device=dev)
     host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
     ws_f = gdpa.workspace_for(p, False, dev)
     ws_b = gdpa.workspace_for(p, True, dev) if training else None
@@ -374,7 +384,8 @@ def run_e2e(args, w, p, qo, ko, training, dev, world):
             rc = gdpa.gdpa_backward(p, ptr(dev_in["q"]), ptr(dev_in["k"]), ptr(dev_in["v"]), ptr(o),
                                     ptr(dev_in["dout"]), ptr(lse), ptr(dqo), ptr(dko),
                                     ptr(dev_in.get("bias")), ptr(outs["dq"]), ptr(outs["dk"]),
-                                    ptr(outs["dv"]), None, ptr(ws_b), ws_b.numel(), sh)
+                                    ptr(outs["dv"]), ptr(outs.get("dbias")), ptr(ws_b),
+                                    ws_b.numel(), sh)
             assert rc == 0, rc
         with torch.cuda.stream(stream):
             for n, t in outs.items():
@@ -398,9 +409,17 @@ def run_e2e(args, w, p, qo, ko, training, dev, world):
 
 
 # ----------------------------------------------------------------- the oracle
-def oracle_sample(cfg: int, n_samples: int, seed: int, training: bool):
+def oracle_sample(cfg: int, n_samples: int, seed: int, training: bool, **kw):
     """A fresh batch of n_samples drawn from the workload's distributions."""
-    return make_workload(cfg, B=n_samples, seed=seed, device="cpu", with_dout=training)
+    return make_workload(cfg, B=n_samples, seed=seed, device="cpu", with_dout=training, **kw)
+
+
+PHI_NAMES = {"silu": 0, "softmax": 1, "identity": 2, "gelu": 3}
+
+
+def phi_override(args) -> dict:
+    """--phi replaces the workload's activation (diagnostic runs)."""
+    return {"phi": PHI_NAMES[args.phi]} if getattr(args, "phi", None) else {}
 
 
 def time_oracle(sub, training: bool) -> float:
@@ -417,9 +436,9 @@ def cpu_baseline(args, w, training: bool, target_s: float = 16.0) -> dict:
     import oracle
     cfg = WORKLOADS[args.workload]
     n = 2
-    dt = time_oracle(oracle_sample(cfg, n, 7000, training), training)
+    dt = time_oracle(oracle_sample(cfg, n, 7000, training, **phi_override(args)), training)
     n = int(min(w.B, max(2, n * target_s / max(dt, 1e-3))))
-    sub = oracle_sample(cfg, n, 7001, training)
+    sub = oracle_sample(cfg, n, 7001, training, **phi_override(args))
     dt = time_oracle(sub, training)
     f_fwd, f_bwd = useful_flops(sub, training)
     return {"value": round((f_fwd + f_bwd) / dt / 1e12, 6), "unit": "TFLOP/s",
@@ -437,10 +456,10 @@ def run_reference(args, rank: int, world: int):
     training = cfg == 5
     per_step = 6 if training else 64
     for i in range(args.warmup):
-        time_oracle(oracle_sample(cfg, 2, 100 + i, training), training)
+        time_oracle(oracle_sample(cfg, 2, 100 + i, training, **phi_override(args)), training)
     times, flops = [], 0.0
     for i in range(args.steps):
-        sub = oracle_sample(cfg, per_step, 200 + i, training)
+        sub = oracle_sample(cfg, per_step, 200 + i, training, **phi_override(args))
         times.append(time_oracle(sub, training))
         f, b = useful_flops(sub, training)
         flops += f + b
@@ -479,6 +498,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None,
                     help="samples per rank (default: the workload's full batch); smaller "
                          "batches are for profiling captures")
+    ap.add_argument("--phi", choices=sorted(PHI_NAMES), default=None,
+                    help="replace the workload's activation (diagnostics)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

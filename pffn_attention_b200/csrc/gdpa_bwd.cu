@@ -42,6 +42,7 @@ static_assert(128 * kRegsControl + 256 * kRegsPhi <= kBwdThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 constexpr float kLog2eB = 1.4426950408889634f;
 constexpr float kInvSqrt2Pi = 0.3989422804014327f;  // 1 / sqrt(2 pi)
+constexpr float kInvSqrt2 = 0.7071067811865476f;    // Phi(x) = (1 + erf(x / sqrt 2)) / 2
 
 template <int D_>
 struct BwdCfg {
@@ -478,7 +479,7 @@ __device__ void bwd_phi(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
               } else if (PHI == 3) {
                 // gelu(x) = x Phi(x); gelu'(x) = Phi(x) + x phi(x), phi the
                 // standard normal density exp(-x^2 / 2) / sqrt(2 pi)
-                const float cdf = normcdff(x);
+                const float cdf = fmaf(0.5f, erff(x * kInvSqrt2), 0.5f);
                 p = x * cdf;
                 ds = dp[e] * fmaf(x, kInvSqrt2Pi * __expf(-0.5f * x * x), cdf);
               } else {

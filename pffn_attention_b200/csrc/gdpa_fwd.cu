@@ -42,7 +42,8 @@ namespace gdpa {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kBN = 128;  // keys per block
+// keys per block: 128, or 64 when no sample has more than 64 keys (a 128-key
+// block would then be half masked, in the MMAs and in phi)
 constexpr int kRegsLaunch = 168;   // 65536 / 384 rounded down to a multiple of 8
 constexpr int kRegsControl = 104;  // warpgroup 0: producer, MMA issuer, allocator, bias
 constexpr int kRegsPhi = 200;      // the two phi warpgroups
@@ -50,12 +51,13 @@ static_assert(128 * kRegsControl + 256 * kRegsPhi <= kThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kInvSqrt2 = 0.7071067811865476f;  // Phi(x) = (1 + erf(x / sqrt 2)) / 2
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
-template <int D_>
+template <int D_, int BN_>
 struct FwdCfg {
   static constexpr int D = D_;
-  static constexpr int BN = kBN;
+  static constexpr int BN = BN_;
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
   // (64 B, 64-byte swizzle) when D = 32.
@@ -65,8 +67,8 @@ struct FwdCfg {
   static constexpr uint32_t LAYOUT = D >= 64 ? LAYOUT_SW128 : LAYOUT_SW64;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;  // one K (or V) block
-  // K/V ring: 128 KB of stages (2 for D = 128, 4 for D = 64, 8 for D = 32)
-  static constexpr int NKV = (64 * 1024) / KV_BYTES;
+  // K/V ring: up to 128 KB of stages (D = 128: 2 of 128 keys or 4 of 64), at most 8
+  static constexpr int NKV = (64 * 1024) / KV_BYTES > 8 ? 8 : (64 * 1024) / KV_BYTES;
   static constexpr int STAGE_WARP = 32 * 128;  // O staging: 32 rows x 128 B per phi warp
   static constexpr int OFF_Q = 0;                                // [2 slots]
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;              // [NKV]
@@ -601,9 +603,9 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
         } else if (gelu) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            // gelu(x) = x Phi(x) (masked columns: gelu(0) = 0)
+            // gelu(x) = x Phi(x), Phi from erf (masked columns: gelu(0) = 0)
             const float x = __uint_as_float(v[e]);
-            v[e] = __float_as_uint(x * normcdff(x));
+            v[e] = __float_as_uint(x * fmaf(0.5f, erff(x * kInvSqrt2), 0.5f));
           }
         } else if (!identity) {
 #pragma unroll
@@ -709,11 +711,11 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
 #undef PHI_WAIT
 }
 
-template <int D, bool SOFTMAX>
+template <int D, int BN, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
   sm.base = smem_u32(smem_raw);
@@ -792,11 +794,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool SOFTMAX>
+template <int D, int BN, bool SOFTMAX>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, int sms, cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  auto kern = gdpa_fwd_kernel<D, SOFTMAX>;
+  using C = FwdCfg<D, BN>;
+  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX>;
   // the phi warpgroups raise their register budget with setmaxnreg, which waits
   // until the block's launch registers cover it: never launch a build whose
   // per-thread count would leave that wait unsatisfiable
@@ -821,23 +823,24 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
 int forward_block_n(int D, int phi, int max_kv, int debug_flags) {
   (void)D;
   (void)phi;
-  (void)max_kv;
   (void)debug_flags;
-  return kBN;
+  return max_kv <= 64 ? 64 : 128;
 }
 
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream) {
-  if (block_n != kBN) return cudaErrorInvalidValue;
   const bool sm = a.phi == 1;
-#define GDPA_FWD_CASE(D_)                                                 \
-  if (D == D_)                                                            \
-    return sm ? launch_one<D_, true>(a, tq, tk, tv, sms, stream)          \
-              : launch_one<D_, false>(a, tq, tk, tv, sms, stream);
-  GDPA_FWD_CASE(32)
-  GDPA_FWD_CASE(64)
-  GDPA_FWD_CASE(128)
+#define GDPA_FWD_CASE(D_, BN_)                                                   \
+  if (D == D_ && block_n == BN_)                                                 \
+    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, sms, stream)             \
+              : launch_one<D_, BN_, false>(a, tq, tk, tv, sms, stream);
+  GDPA_FWD_CASE(32, 64)
+  GDPA_FWD_CASE(32, 128)
+  GDPA_FWD_CASE(64, 64)
+  GDPA_FWD_CASE(64, 128)
+  GDPA_FWD_CASE(128, 64)
+  GDPA_FWD_CASE(128, 128)
 #undef GDPA_FWD_CASE
   return cudaErrorInvalidValue;
 }

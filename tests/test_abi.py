@@ -92,10 +92,11 @@ def test_workspace_size_grows_with_problem(lib):
 
 
 def test_tile_shape_query(lib):
-    # one forward tile shape: 128 query rows x 128-key blocks
-    for kv in (64, 2000):
-        rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=kv))
-        assert (rc, bm, bn) == (0, 128, 128)
+    # 128 query rows; 64-key blocks when no sample has more than 64 keys
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=64))
+    assert (rc, bm, bn) == (0, 128, 64)
+    rc, bm, bn = gdpa.gdpa_forward_tile_shape(_params(max_seqlen_kv=65))
+    assert (rc, bm, bn) == (0, 128, 128)
 
 
 def test_head_phi_validation(lib):
