@@ -488,6 +488,91 @@ def dist_env():
     return rank, world, local
 
 
+# ----------------------------------------------------------------- grouped
+# Event-level personalisation: each event type runs its own small GDPA problem
+# with its own heads, width, activation and window.  A synthetic set of eight
+# event types (shapes chosen across the workloads' ranges) timed as one
+# gdpa_forward_grouped call against the same problems as separate calls.
+EVENT_TYPES = [  # (H, D, phi, window, B, q lengths, kv lengths ("same" = q), bias)
+    (8, 128, 1, (255, 0), 64, (200, 1000), "same", 0),
+    (4, 128, 1, (127, 0), 128, (100, 500), "same", 0),
+    (4, 64, 1, (63, 0), 256, (50, 300), "same", 0),
+    (2, 64, 0, (-1, -1), 512, (20, 200), (64, 64), 0),
+    (2, 32, 1, (31, 0), 512, (10, 100), "same", 0),
+    (8, 128, 1, (-1, -1), 128, (100, 600), (256, 256), 2),
+    (4, 64, 3, (-1, -1), 256, (50, 400), (64, 64), 0),
+    (2, 32, 0, (-1, -1), 1024, (1, 64), (16, 16), 0),
+]
+
+
+def run_grouped(args):
+    import torch
+
+    from pffn_attention_b200 import gdpa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    names = {v: k for k, v in PHI_NAMES.items()}
+    rng = np.random.default_rng(600)
+    ws_, probs, flops, byts = [], [], 0.0, 0.0
+    for i, (H, D, phi, win, B, ql, kl, bias) in enumerate(EVENT_TYPES):
+        q_lens = rng.integers(ql[0], ql[1] + 1, B)
+        kv_lens = q_lens if kl == "same" else rng.integers(kl[0], kl[1] + 1, B)
+        base = 3 if phi == 1 else 2
+        extra = {} if phi == 1 else dict(scale=1.0, kv_std=1.0 / np.sqrt(D))
+        w = make_workload(base, seed=610 + i, q_lens=q_lens, kv_lens=kv_lens, H=H, D=D, phi=phi,
+                          window=win, bias=bias, device=dev, with_dout=False, **extra)
+        ws_.append(w)
+        probs.append(dict(q=w.q, k=w.k, v=w.v,
+                          q_offsets=torch.tensor(w.q_offsets, dtype=torch.int32, device=dev),
+                          kv_offsets=torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev),
+                          bias=w.bias, phi=names[phi], scale=w.scale, window=win,
+                          bias_kind=bias, max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv))
+        flops += useful_flops(w, False)[0]
+        byts += algorithmic_bytes(w, False)[0]
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    outs, wsg = gdpa.forward_grouped(probs, stream=stream)  # allocates outputs, workspace
+    single = []
+    for d, (o, lse) in zip(probs, outs):
+        kw = {k: d[k] for k in ("phi", "scale", "window", "bias", "bias_kind", "max_seqlen_q",
+                                "max_seqlen_kv")}
+        _, _, ws1 = gdpa.forward(d["q"], d["k"], d["v"], d["q_offsets"], d["kv_offsets"], out=o,
+                                 lse=lse, stream=stream, **kw)  # its workspace, reused below
+        single.append((d, kw, o, lse, ws1))
+
+    def grouped_step():
+        gdpa.forward_grouped(probs, workspace=wsg, stream=stream)
+
+    def separate_step():
+        for d, kw, o, lse, ws1 in single:
+            gdpa.forward(d["q"], d["k"], d["v"], d["q_offsets"], d["kv_offsets"], out=o,
+                         lse=lse, workspace=ws1, stream=stream, **kw)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    g_ms = timed(grouped_step)
+    s_ms = timed(separate_step)
+    assert gdpa.device_status(wsg, stream) == 0
+    return {"metric": "GDPA grouped forward, event-type problems per call (useful TFLOP/s)",
+            "value": round(flops / (g_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(g_ms, 4),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "event_groups", "problems": len(EVENT_TYPES),
+                       "samples": int(sum(w.B for w in ws_))},
+            "separate_calls_ms": round(s_ms, 4), "grouped_speedup": round(s_ms / g_ms, 3),
+            "achieved_gbs": round(byts / (g_ms * 1e-3) / 1e9, 1)}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,12 +587,20 @@ def main(argv=None):
                     help="replace the workload's activation (diagnostics)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grouped", action="store_true",
+                    help="time the event-type problems as one grouped call vs separate calls")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
     rank, world, local = dist_env()
     if world != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.grouped:
+        if world != 1 or args.impl != "ours":
+            ap.error("--grouped runs on one GPU, our implementation")
+        print(json.dumps(run_grouped(args)), flush=True)
+        return 0
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)

@@ -136,6 +136,40 @@ GDPA_API gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, cons
                             void* dk, void* dv, float* dbias, void* workspace,
                             size_t workspace_bytes, gdpa_stream_t stream);
 
+/* Grouped forward: several independent GDPA problems in one call, each with
+ * its own shapes (B, H, D), activation(s), scale, band, bias and tensors --
+ * the many small problems of event-level personalisation, where each event
+ * type has its own model width, head count and window (Kunlun paper review,
+ * §2.5, "Event-level Personalization").  Problems that share the head dim,
+ * the key-block size (64 keys when no sample has more than 64, else 128) and
+ * softmax-or-not run in ONE persistent launch whose CTAs take the
+ * (problem, sample, head) units of all of them, longest sample first; a call
+ * makes one such launch per distinct combination.  Each problem's outputs
+ * equal those of gdpa_forward on it alone.  Limits per launch group: at most
+ * 256 problems and 16384 samples in total.  Every problem is validated as by
+ * gdpa_forward before anything is launched; the workspace is for the whole
+ * call (gdpa_forward_grouped_workspace_size) and gdpa_get_device_status
+ * reads its status. */
+typedef struct {
+  gdpa_params_t params;
+  const void* q;                /* [total_q][H][D] bf16 */
+  const void* k;                /* [total_kv][H][D] bf16 */
+  const void* v;                /* [total_kv][H][D] bf16 */
+  const int32_t* q_offsets;     /* [B+1] */
+  const int32_t* kv_offsets;    /* [B+1] */
+  const float* bias;            /* [H][total_kv] fp32, or NULL (bias_kind NONE) */
+  void* o;                      /* [total_q][H][D] bf16 */
+  float* lse;                   /* [H][total_q] fp32 or NULL (softmax heads only) */
+} gdpa_forward_problem_t;
+
+/* Workspace bytes of gdpa_forward_grouped for these problems; 0 when they are
+ * invalid or exceed the limits above. */
+GDPA_API size_t gdpa_forward_grouped_workspace_size(const gdpa_forward_problem_t* problems,
+                                                    int n_problems);
+GDPA_API gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems,
+                                            int n_problems, void* workspace,
+                                            size_t workspace_bytes, gdpa_stream_t stream);
+
 /* Forward for callers that cannot allocate device memory.  (The Kunlun pages
  * have no counterpart to this entry point; it exists for this library's users.)
  * Some callers have no way to give the library a workspace: a plugin inside a

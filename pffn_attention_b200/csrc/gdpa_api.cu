@@ -6,6 +6,8 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
+#include <algorithm>
 
 #include "gdpa.h"
 #include "gdpa_internal.h"
@@ -137,9 +139,114 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H, int D, int 
   return r == CUDA_SUCCESS;
 }
 
+// Everything gdpa_forward checks about one problem before any launch.
+gdpa_status_t check_forward_args(const gdpa_params_t* p, const void* q, const void* k,
+                                 const void* v, const int32_t* q_offsets,
+                                 const int32_t* kv_offsets, const float* bias, const void* o,
+                                 const float* lse) {
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
+  if (p->total_q > 0 && (!q || !o)) return GDPA_ERR_INVALID_ARG;
+  if (p->total_kv > 0 && (!k || !v)) return GDPA_ERR_INVALID_ARG;
+  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GDPA_ERR_INVALID_ARG;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
+  return GDPA_OK;
+}
+
 uint64_t timeout_ns(const gdpa_params_t* p) {
   const int us = p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000;
   return (uint64_t)us * 1000ull;
+}
+
+
+// ---- grouped forward
+// One activation's heads of one caller problem.
+struct VProblem {
+  int src;          // index into the caller's problems
+  int phi;
+  uint64_t heads;
+};
+
+// Problems that share a launch: head dim, key-block size, softmax or not.
+struct LaunchGroup {
+  int D, block_n;
+  bool softmax;
+  std::vector<VProblem> vp;
+  int entries = 0, hmax = 0;
+  size_t off_probs = 0, off_maps = 0, off_sched = 0, off_info = 0, off_eprob = 0;
+};
+
+// Workspace of a grouped call: status block and the tables the host fills
+// (schedule jobs; per group: problem table, tensor maps, schedule table) as
+// one contiguous range copied in one transfer (the status copied as zeros),
+// then per group the sorted entries and their problems, which the schedule
+// kernel writes.
+struct GroupedLayout {
+  size_t off_jobs = 0, tables_end = 0, total = 0;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Validates every problem, forms the launch groups and lays out the workspace.
+// Nothing touches the device.
+gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
+                           std::vector<LaunchGroup>& groups, GroupedLayout& lay) {
+  if (!probs || n < 1) return GDPA_ERR_INVALID_ARG;
+  groups.clear();
+  for (int i = 0; i < n; ++i) {
+    const gdpa_forward_problem_t& f = probs[i];
+    const gdpa_params_t* p = &f.params;
+    gdpa_status_t st = check_forward_args(p, f.q, f.k, f.v, f.q_offsets, f.kv_offsets, f.bias,
+                                          f.o, f.lse);
+    if (st != GDPA_OK) return st;
+    const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p), p->debug_flags);
+    for (int phi = 0; phi <= 3; ++phi) {
+      const uint64_t heads = phi_heads(p, phi);
+      if (!heads) continue;
+      const bool sm = phi == GDPA_PHI_SOFTMAX;
+      LaunchGroup* g = nullptr;
+      for (LaunchGroup& x : groups)
+        if (x.D == p->D && x.block_n == block_n && x.softmax == sm) g = &x;
+      if (!g) {
+        groups.push_back(LaunchGroup{});
+        g = &groups.back();
+        g->D = p->D;
+        g->block_n = block_n;
+        g->softmax = sm;
+      }
+      g->vp.push_back(VProblem{i, phi, heads});
+    }
+  }
+  size_t total = align256(sizeof(DeviceStatus));
+  lay.off_jobs = total;
+  total = align256(total + groups.size() * sizeof(GroupSchedJob));
+  for (LaunchGroup& g : groups) {
+    if ((int)g.vp.size() > kMaxGroupProblems) return GDPA_ERR_UNSUPPORTED;
+    int64_t entries = 0;
+    for (const VProblem& v : g.vp) {
+      entries += probs[v.src].params.B;
+      g.hmax = std::max(g.hmax, probs[v.src].params.H);
+    }
+    if (entries > kMaxSortBatch) return GDPA_ERR_UNSUPPORTED;
+    if (entries * (int64_t)g.hmax >= (int64_t(1) << 31)) return GDPA_ERR_UNSUPPORTED;
+    g.entries = (int)entries;
+    const size_t nv = g.vp.size();
+    g.off_probs = total;
+    g.off_maps = align256(g.off_probs + nv * sizeof(FwdProblem));
+    g.off_sched = align256(g.off_maps + 3 * nv * sizeof(CUtensorMap));
+    total = align256(g.off_sched + nv * sizeof(GroupSchedProblem));
+  }
+  lay.tables_end = total;
+  for (LaunchGroup& g : groups) {
+    g.off_info = total;
+    g.off_eprob = align256(g.off_info + (size_t)g.entries * sizeof(int4));
+    total = align256(g.off_eprob + (size_t)g.entries * sizeof(int32_t));
+  }
+  lay.total = total;
+  return GDPA_OK;
 }
 
 }  // namespace
@@ -198,16 +305,9 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
                            const int32_t* q_offsets, const int32_t* kv_offsets,
                            const float* bias, void* o, float* lse, void* workspace,
                            size_t workspace_bytes, gdpa_stream_t stream) {
-  gdpa_status_t st = check_params(p);
+  gdpa_status_t st = check_forward_args(p, q, k, v, q_offsets, kv_offsets, bias, o, lse);
   if (st != GDPA_OK) return st;
-  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
-  if (p->total_q > 0 && (!q || !o)) return GDPA_ERR_INVALID_ARG;
-  if (p->total_kv > 0 && (!k || !v)) return GDPA_ERR_INVALID_ARG;
-  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(workspace))
-    return GDPA_ERR_INVALID_ARG;
-  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return GDPA_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
   const WorkspaceLayout L = make_layout(p, 0, sms);
@@ -236,27 +336,21 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
     tv = tq;
   }
   FwdArgs a{};
-  a.q_offsets = q_offsets;
-  a.kv_offsets = kv_offsets;
-  a.order = order;
   a.info = info;
-  a.bias = bias;
-  a.o = static_cast<__nv_bfloat16*>(o);
   a.status = status;
-  a.total_q = p->total_q;
-  a.total_kv = p->total_kv;
-  a.B = p->B;
   a.H = p->H;
   a.n_units = p->B * p->H;
-  a.max_q = eff_max_q(p);
-  a.max_kv = eff_max_kv(p);
-  a.scale = p->scale;
-  a.phi = p->phi;
-  a.bias_kind = p->bias_kind;
-  a.wl = p->window_left;
-  a.wr = p->window_right;
   a.debug_flags = p->debug_flags;
   a.timeout_ns = timeout_ns(p);
+  a.p0.bias = bias;
+  a.p0.o = static_cast<__nv_bfloat16*>(o);
+  a.p0.total_q = p->total_q;
+  a.p0.total_kv = p->total_kv;
+  a.p0.H = p->H;
+  a.p0.bias_kind = p->bias_kind;
+  a.p0.wl = p->window_left;
+  a.p0.wr = p->window_right;
+  a.p0.scale = p->scale;
   // one launch per activation present (a per-head activation vector groups
   // the heads; each launch walks only its own heads' units)
   for (int phi = 0; phi <= 3; ++phi) {
@@ -264,7 +358,9 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
     if (!heads) continue;
     a.phi = phi;
     a.head_mask = heads;
-    a.lse = phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
+    a.p0.phi = phi;
+    a.p0.head_mask = heads;
+    a.p0.lse = phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
     e = launch_forward(a, p->D, block_n, tq, tk, tv, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
@@ -373,6 +469,128 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
     a.phi = phi;
     a.head_mask = heads;
     e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
+  return GDPA_OK;
+}
+
+size_t gdpa_forward_grouped_workspace_size(const gdpa_forward_problem_t* problems,
+                                           int n_problems) {
+  std::vector<LaunchGroup> groups;
+  GroupedLayout lay;
+  if (plan_grouped(problems, n_problems, groups, lay) != GDPA_OK) return 0;
+  return lay.total;
+}
+
+gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n_problems,
+                                   void* workspace, size_t workspace_bytes,
+                                   gdpa_stream_t stream) {
+  std::vector<LaunchGroup> groups;
+  GroupedLayout lay;
+  gdpa_status_t st = plan_grouped(problems, n_problems, groups, lay);
+  if (st != GDPA_OK) return st;
+  // tensor maps in the workspace must be 64-byte aligned
+  if (reinterpret_cast<uintptr_t>(workspace) & 63u) return GDPA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < lay.total) return GDPA_ERR_WORKSPACE;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  cudaStream_t s = (cudaStream_t)stream;
+
+  // the cleared status and every table staged on the host, copied in one transfer
+  std::vector<uint8_t> host(lay.tables_end, 0);
+  auto at = [&](size_t off) { return host.data() + off; };
+  GroupSchedJob* jobs = reinterpret_cast<GroupSchedJob*>(at(lay.off_jobs));
+  std::vector<int> q_map(groups.size(), -1);
+  std::vector<uint64_t> timeouts(groups.size(), 0);
+  int max_entries = 1;
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    const LaunchGroup& g = groups[gi];
+    const size_t nv = g.vp.size();
+    FwdProblem* fp = reinterpret_cast<FwdProblem*>(at(g.off_probs));
+    CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(at(g.off_maps));
+    GroupSchedProblem* sp = reinterpret_cast<GroupSchedProblem*>(at(g.off_sched));
+    int ebase = 0;
+    for (size_t j = 0; j < nv; ++j) {
+      const VProblem& vp = g.vp[j];
+      const gdpa_forward_problem_t& f = problems[vp.src];
+      const gdpa_params_t* p = &f.params;
+      fp[j].bias = f.bias;
+      fp[j].o = static_cast<__nv_bfloat16*>(f.o);
+      fp[j].lse = vp.phi == GDPA_PHI_SOFTMAX ? f.lse : nullptr;
+      fp[j].total_q = p->total_q;
+      fp[j].total_kv = p->total_kv;
+      fp[j].H = p->H;
+      fp[j].phi = vp.phi;
+      fp[j].bias_kind = p->bias_kind;
+      fp[j].wl = p->window_left;
+      fp[j].wr = p->window_right;
+      fp[j].scale = p->scale;
+      fp[j].head_mask = vp.heads;
+      // encoded into an aligned local object, then copied into the staging bytes
+      CUtensorMap m;
+      if (p->total_q > 0) {
+        if (!make_map(&m, f.q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+        std::memcpy(&maps[3 * j], &m, sizeof(m));
+        if (q_map[gi] < 0) q_map[gi] = (int)j;
+      }
+      if (p->total_kv > 0) {
+        if (!make_map(&m, f.k, p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
+        std::memcpy(&maps[3 * j + 1], &m, sizeof(m));
+        if (!make_map(&m, f.v, p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
+        std::memcpy(&maps[3 * j + 2], &m, sizeof(m));
+      }
+      sp[j].q_offsets = f.q_offsets;
+      sp[j].kv_offsets = f.kv_offsets;
+      sp[j].B = p->B;
+      sp[j].ebase = ebase;
+      sp[j].wl = p->window_left;
+      sp[j].wr = p->window_right;
+      sp[j].max_q = eff_max_q(p);
+      sp[j].max_kv = eff_max_kv(p);
+      ebase += p->B;
+      timeouts[gi] = std::max(timeouts[gi], timeout_ns(p));
+    }
+    // maps of empty tensors are never read; keep every slot a valid map
+    if (q_map[gi] >= 0)
+      for (size_t j = 0; j < nv; ++j)
+        for (int w = 0; w < 3; ++w)
+          if (problems[g.vp[j].src].params.total_q == 0 ||
+              (w > 0 && problems[g.vp[j].src].params.total_kv == 0))
+            std::memcpy(&maps[3 * j + w], &maps[3 * q_map[gi]], sizeof(CUtensorMap));
+    jobs[gi].probs = reinterpret_cast<const GroupSchedProblem*>(ws + g.off_sched);
+    jobs[gi].n_probs = (int)nv;
+    jobs[gi].n_entries = g.entries;
+    jobs[gi].block_n = g.block_n;
+    jobs[gi].info = reinterpret_cast<int4*>(ws + g.off_info);
+    jobs[gi].eprob = reinterpret_cast<int32_t*>(ws + g.off_eprob);
+    max_entries = std::max(max_entries, g.entries);
+  }
+  if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return GDPA_ERR_CUDA;
+  cudaError_t e = launch_group_schedule(reinterpret_cast<const GroupSchedJob*>(ws + lay.off_jobs),
+                                        (int)groups.size(), max_entries, kBlockM, status, s);
+  if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    const LaunchGroup& g = groups[gi];
+    if (g.entries == 0 || q_map[gi] < 0) continue;  // no query row in the group
+    FwdArgs a{};
+    a.info = reinterpret_cast<const int4*>(ws + g.off_info);
+    a.status = status;
+    a.H = g.hmax;
+    a.n_units = g.entries * g.hmax;
+    a.phi = g.softmax ? GDPA_PHI_SOFTMAX : GDPA_PHI_SILU;  // launch class only
+    a.debug_flags = 0;
+    a.timeout_ns = timeouts[gi];
+    a.head_mask = ~0ull;
+    a.eprob = reinterpret_cast<const int32_t*>(ws + g.off_eprob);
+    a.probs = reinterpret_cast<const FwdProblem*>(ws + g.off_probs);
+    a.maps = reinterpret_cast<const CUtensorMap*>(ws + g.off_maps);
+    CUtensorMap m0;  // kernel parameters, unused when grouped
+    std::memcpy(&m0, at(g.off_maps) + 3 * q_map[gi] * sizeof(CUtensorMap), sizeof(m0));
+    e = launch_forward(a, g.D, g.block_n, m0, m0, m0, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;

@@ -54,10 +54,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kInvSqrt2 = 0.7071067811865476f;  // Phi(x) = (1 + erf(x / sqrt 2)) / 2
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
-template <int D_, int BN_>
+template <int D_, int BN_, bool GROUPED_>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;
+  static constexpr bool GROUPED = GROUPED_;  // units of several problems
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
   // (64 B, 64-byte swizzle) when D = 32.
@@ -106,6 +107,15 @@ struct FwdCfg {
 
 using Unit = GdpaUnit;
 
+// A unit's problem: the table's in a grouped launch, else the inline one of a
+// single-problem call (read from the kernel parameters).  Returned by value
+// so only the fields a caller uses are loaded.
+template <class C>
+__device__ __forceinline__ FwdProblem fwd_problem(const FwdArgs& a, int p) {
+  if constexpr (C::GROUPED) return a.probs[p];
+  return a.p0;
+}
+
 // Key-block range [kb0, kb1) a tile starting at local row m0 may touch.
 template <int BN>
 __device__ __forceinline__ void kv_range(int m0, int Lk, int wl, int wr, int& kb0, int& kb1) {
@@ -128,6 +138,7 @@ struct FTile {
   bool resident;        // the unit's blocks are loaded once, at its first tile
   bool unit_first;      // first tile of its unit
   int slot;             // 0 or 1: tiles alternate between the two slots
+  int prob;             // its problem (grouped launch; 0 otherwise)
 };
 
 // The CTA's tiles in the order every role uses.  Units come from UnitStream
@@ -136,19 +147,24 @@ struct FTile {
 // block count at every tile of a streamed unit.
 template <class C>
 struct TileWalk {
-  UnitStream units;
+  const FwdArgs* args;
+  UnitStreamT<C::GROUPED> units;
   Unit t;
   int wl, wr, ntile, mt, nkb;
   uint32_t g, kvi, unit_kv0;
   bool resident, in_unit;
   __device__ explicit TileWalk(const FwdArgs& a)
-      : units(a.info, a.H, a.n_units, a.head_mask), t{}, wl(a.wl), wr(a.wr), ntile(0), mt(0),
-        nkb(0), g(0),
-        kvi(0), unit_kv0(0), resident(false), in_unit(false) {}
+      : args(&a), units(a.info, a.H, a.n_units, a.head_mask, a.eprob, a.probs), t{},
+        wl(a.p0.wl), wr(a.p0.wr), ntile(0), mt(0), nkb(0), g(0), kvi(0), unit_kv0(0),
+        resident(false), in_unit(false) {}
   __device__ bool next(FTile& x) {
     for (;;) {
       if (!in_unit) {
         if (!units.next(t)) return false;
+        if constexpr (C::GROUPED) {  // the band of this unit's problem
+          wl = args->probs[t.prob].wl;
+          wr = args->probs[t.prob].wr;
+        }
         ntile = (t.Lq + kBlockM - 1) / kBlockM;
         nkb = (t.Lk + C::BN - 1) / C::BN;
         resident = wl < 0 && wr < 0 && nkb > 0 && nkb <= C::NKV;
@@ -178,6 +194,7 @@ struct TileWalk {
         if (x.kb1 > x.kb0) kvi += x.kb1 - x.kb0;
       }
       x.slot = (int)(g & 1);
+      x.prob = t.prob;
       ++g;
       ++mt;
       return true;
@@ -236,7 +253,12 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   uint32_t nq[2] = {0u, 0u};
   bool dropped = false;
   TileWalk<C> walk(a);
-  FTile x;
+  FTile x{};
+  // a grouped launch keeps each problem's Q, K, V maps in device memory
+  auto map_of = [&](int prob, int which) -> const CUtensorMap* {
+    if constexpr (C::GROUPED) return a.maps + 3 * prob + which;
+    return which == 0 ? tq : which == 1 ? tk : tv;
+  };
   auto load_kv = [&](uint32_t ring, int kb) -> bool {
     const int st = (int)(ring % C::NKV);
     if (!mbar_wait(sm.bar(C::B_KVEMPTY + st), ((ring / C::NKV) & 1) ^ 1, abort, a.status,
@@ -244,10 +266,12 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
       return false;
     sm.kv_tag()[st] = (int)ring;  // published by the arrive below (release)
     mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + st), 2 * C::KV_BYTES);
+    const CUtensorMap* mk = map_of(x.prob, 1);
+    const CUtensorMap* mv = map_of(x.prob, 2);
     for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
-      tma_load_3d(sm.k(st) + pnl * C::BN * C::PANEL_BYTES, tk, sm.bar(C::B_KVFULL + st),
+      tma_load_3d(sm.k(st) + pnl * C::BN * C::PANEL_BYTES, mk, sm.bar(C::B_KVFULL + st),
                   pnl * C::PANEL_ELEMS, x.h, x.k0 + kb * C::BN, pol_keep);
-      tma_load_3d(sm.v(st) + pnl * C::BN * C::PANEL_BYTES, tv, sm.bar(C::B_KVFULL + st),
+      tma_load_3d(sm.v(st) + pnl * C::BN * C::PANEL_BYTES, mv, sm.bar(C::B_KVFULL + st),
                   pnl * C::PANEL_ELEMS, x.h, x.k0 + kb * C::BN, pol_keep);
     }
     return true;
@@ -262,8 +286,9 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
       dropped = true;  // test hook: this Q tile is never loaded
     } else {
       mbar_arrive_expect_tx(sm.bar(C::B_QFULL + s), C::Q_BYTES);
+      const CUtensorMap* mq = map_of(x.prob, 0);
       for (int pnl = 0; pnl < C::NPANEL; ++pnl)
-        tma_load_3d(sm.q(s) + pnl * kBlockM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + s),
+        tma_load_3d(sm.q(s) + pnl * kBlockM * C::PANEL_BYTES, mq, sm.bar(C::B_QFULL + s),
                     pnl * C::PANEL_ELEMS, x.h, x.q0 + x.m0, pol_stream);
     }
     ++nq[s];
@@ -273,10 +298,12 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
       Unit nt;
       if (walk.units.peek(nt)) {
         const int nb = min((nt.Lk + C::BN - 1) / C::BN, 2);
+        const CUtensorMap* mk = map_of(nt.prob, 1);
+        const CUtensorMap* mv = map_of(nt.prob, 2);
         for (int j = 0; j < nb; ++j)
           for (int pnl = 0; pnl < C::NPANEL; ++pnl) {
-            tma_prefetch_l2_3d(tk, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
-            tma_prefetch_l2_3d(tv, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
+            tma_prefetch_l2_3d(mk, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
+            tma_prefetch_l2_3d(mv, pnl * C::PANEL_ELEMS, nt.h, nt.k0 + j * C::BN, pol_keep);
           }
       }
     }
@@ -445,21 +472,23 @@ __device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, int s, bool softm
   const int lane = threadIdx.x & 31;
   uint32_t bc = 0;
   TileWalk<C> walk(a);
-  FTile x;
+  FTile x{};
   while (walk.next_slot(x, s)) {
+    const FwdProblem P = fwd_problem<C>(a, x.prob);
+    if (P.bias_kind == 0) continue;  // the phi warpgroup adds no bias for this tile
     for (int j = x.kb0; j < x.kb1; ++j) {
       const int bb = bc & 1;
       bool ok = mbar_wait(sm.bar(C::B_BEMPTY + 2 * s + bb), ((bc >> 1) & 1) ^ 1, abort, a.status,
                           a.timeout_ns, 0x300 + C::B_BEMPTY + 2 * s + bb);
       if (!__all_sync(0xffffffffu, ok)) return;
       float* dst = sm.bias(s, bb);
-      const float* src = a.bias + (int64_t)x.h * a.total_kv + x.k0;
+      const float* src = P.bias + (int64_t)x.h * P.total_kv + x.k0;
       for (int c = lane; c < C::BN; c += 32) {
         const int key = j * C::BN + c;
         float beta = 0.f;
         if (key < x.Lk) {
           const float g = src[key];
-          if (a.bias_kind == 2) {
+          if (P.bias_kind == 2) {
             // log sigma(g) = min(g, 0) - log(1 + exp(-|g|))
             beta = fminf(g, 0.f) - log1pf(__expf(-fabsf(g)));
           } else {
@@ -484,10 +513,6 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
   const int lane = threadIdx.x & 31;
   const int r = wq * 32 + lane;             // row of the tile owned by this thread
   const uint32_t tslot = tmem + ((uint32_t)(wq * 32) << 16) + s * C::TMEM_SLOT;
-  const bool has_bias = a.bias_kind != 0;
-  const bool identity = a.phi == 2;
-  const bool gelu = a.phi == 3;
-  const float sc = SOFTMAX ? a.scale * kLog2e : a.scale;
   uint32_t nsb = 0, tq = 0, bc = 0;  // S blocks, non-empty tiles, bias blocks of the slot
 
 #define PHI_WAIT(bar_, par_, where_)                                                   \
@@ -497,23 +522,34 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
   } while (0)
 
   TileWalk<C> walk(a);
-  FTile x;
+  FTile x{};
   while (walk.next_slot(x, s)) {
+    // this tile's problem: its outputs, scale, activation, bias and band
+    const FwdProblem P = fwd_problem<C>(a, x.prob);
+    __nv_bfloat16* const out = P.o;
+    float* const lse_out = P.lse;
+    const int Hp = P.H;
+    const int64_t tqp = P.total_q;
+    const int wl = P.wl, wr = P.wr;
+    const bool has_bias = P.bias_kind != 0;
+    const bool identity = P.phi == 2;
+    const bool gelu = P.phi == 3;
+    const float sc = SOFTMAX ? P.scale * kLog2e : P.scale;
     const int row = x.m0 + r;
     const bool row_ok = row < x.Lq;
     const int nkv = x.kb1 - x.kb0;
     if (nkv <= 0) {
       if (row_ok) {
-        __nv_bfloat16* orow = a.o + ((int64_t)(x.q0 + row) * a.H + x.h) * C::D;
+        __nv_bfloat16* orow = out + ((int64_t)(x.q0 + row) * Hp + x.h) * C::D;
         const uint4 z = make_uint4(0, 0, 0, 0);
         for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
-        if (SOFTMAX && a.lse) a.lse[(int64_t)x.h * a.total_q + x.q0 + row] = -INFINITY;
+        if (SOFTMAX && lse_out) lse_out[(int64_t)x.h * tqp + x.q0 + row] = -INFINITY;
       }
       continue;
     }
     // visible keys of this row: [lo, hi]
-    const int lo = a.wl >= 0 ? row - a.wl : INT_MIN;
-    const int hi = min(x.Lk - 1, a.wr >= 0 ? row + a.wr : INT_MAX);
+    const int lo = wl >= 0 ? row - wl : INT_MIN;
+    const int hi = min(x.Lk - 1, wr >= 0 ? row + wr : INT_MAX);
     float m_run = -INFINITY, l_run = 0.f;
     for (int idx = 0; idx < nkv; ++idx) {
       const int kbase = (x.kb0 + idx) * C::BN;
@@ -523,7 +559,7 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
       tc_fence_after();
       const float2* bias2 = reinterpret_cast<const float2*>(sm.bias(s, bb));
       // visible columns of this block: [clo, chi] (no shift of an unbounded side)
-      const int clo = a.wl >= 0 ? lo - kbase : INT_MIN;
+      const int clo = wl >= 0 ? lo - kbase : INT_MIN;
       const int chi = hi - kbase;  // hi <= Lk - 1 always
       const bool full = clo <= 0 && chi >= C::BN - 1;
       const uint64_t sc2 = f2_pack(sc, sc);
@@ -697,25 +733,25 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
         const int grow = x.m0 + wq * 32 + j;
         const uint4 v = ld_shared_v4(sm.stage(pw, j, cc, SWM));
         if (grow < x.Lq)
-          *reinterpret_cast<uint4*>(a.o + ((int64_t)(x.q0 + grow) * a.H + x.h) * C::D +
+          *reinterpret_cast<uint4*>(out + ((int64_t)(x.q0 + grow) * Hp + x.h) * C::D +
                                     ps * PW + cc * 8) = v;
       }
       __syncwarp();
     }
     ++tq;
-    if (SOFTMAX && row_ok && a.lse) {
-      a.lse[(int64_t)x.h * a.total_q + x.q0 + row] =
+    if (SOFTMAX && row_ok && lse_out) {
+      lse_out[(int64_t)x.h * tqp + x.q0 + row] =
           l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 #undef PHI_WAIT
 }
 
-template <int D, int BN, bool SOFTMAX>
+template <int D, int BN, bool SOFTMAX, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
-  using C = FwdCfg<D, BN>;
+  using C = FwdCfg<D, BN, GROUPED>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
   sm.base = smem_u32(smem_raw);
@@ -770,7 +806,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       if (lane == 0) role_mma<C>(a, sm, tmem);
     } else {
-      if (a.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
+      // a grouped launch may mix problems with and without a bias
+      if (C::GROUPED || a.p0.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
     }
   } else {
     setmaxnreg_inc<kRegsPhi>();
@@ -794,11 +831,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BN, bool SOFTMAX>
+template <int D, int BN, bool SOFTMAX, bool GROUPED>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, int sms, cudaStream_t stream) {
-  using C = FwdCfg<D, BN>;
-  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX>;
+  using C = FwdCfg<D, BN, GROUPED>;
+  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED>;
   // the phi warpgroups raise their register budget with setmaxnreg, which waits
   // until the block's launch registers cover it: never launch a build whose
   // per-thread count would leave that wait unsatisfiable
@@ -831,10 +868,15 @@ cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorM
                            const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream) {
   const bool sm = a.phi == 1;
-#define GDPA_FWD_CASE(D_, BN_)                                                   \
-  if (D == D_ && block_n == BN_)                                                 \
-    return sm ? launch_one<D_, BN_, true>(a, tq, tk, tv, sms, stream)             \
-              : launch_one<D_, BN_, false>(a, tq, tk, tv, sms, stream);
+  const bool grouped = a.probs != nullptr;
+#define GDPA_FWD_CASE(D_, BN_)                                                         \
+  if (D == D_ && block_n == BN_) {                                                     \
+    if (grouped)                                                                       \
+      return sm ? launch_one<D_, BN_, true, true>(a, tq, tk, tv, sms, stream)          \
+                : launch_one<D_, BN_, false, true>(a, tq, tk, tv, sms, stream);        \
+    return sm ? launch_one<D_, BN_, true, false>(a, tq, tk, tv, sms, stream)           \
+              : launch_one<D_, BN_, false, false>(a, tq, tk, tv, sms, stream);         \
+  }
   GDPA_FWD_CASE(32, 64)
   GDPA_FWD_CASE(32, 128)
   GDPA_FWD_CASE(64, 64)

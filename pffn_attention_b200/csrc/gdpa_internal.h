@@ -25,26 +25,39 @@ struct WorkspaceLayout {
   int grid;
 };
 
-struct FwdArgs {
-  const int32_t* q_offsets;
-  const int32_t* kv_offsets;
-  const int32_t* order;
-  const int4* info;         // per sorted sample {q0, Lq, k0, Lk}
+// One forward problem's own data: every field a kernel role reads per unit.
+// A single-problem call carries it inline (FwdArgs::p0); a grouped call keeps
+// one per problem in device memory (FwdArgs::probs).
+struct FwdProblem {
   const float* bias;        // [H][total_kv] or nullptr
   __nv_bfloat16* o;         // [total_q][H][D]
   float* lse;               // [H][total_q] or nullptr
-  DeviceStatus* status;
   int64_t total_q, total_kv;
-  int B, H;
-  int n_units;              // B * H
-  int max_q, max_kv;
-  float scale;
+  int H;
   int phi;
   int bias_kind;
   int wl, wr;
+  float scale;
+  uint64_t head_mask;       // heads computed (bit h); ~0 = all
+};
+
+struct FwdArgs {
+  const int4* info;         // per sorted entry {q0, Lq, k0, Lk}
+  DeviceStatus* status;
+  int H;                    // head stride of the unit index (the group's largest H)
+  int n_units;              // entries * H
+  int phi;                  // activation class of the launch (1 = softmax, else element-wise)
   int debug_flags;
   uint64_t timeout_ns;
-  uint64_t head_mask;       // heads this launch computes (bit h), ~0 = all
+  uint64_t head_mask;       // single problem: heads computed (bit h), ~0 = all
+  // Grouped launch: problem of sorted entry e is eprob[e]; units are
+  // (entry, head) with head stride H (the group's largest), units a problem
+  // lacks are skipped; per-problem data and Q/K/V maps in device memory.
+  // All nullptr for a single problem (p0 and the kernel's map parameters).
+  const int32_t* eprob;
+  const FwdProblem* probs;
+  const CUtensorMap* maps;  // [problem][Q, K, V]
+  FwdProblem p0;
 };
 
 struct BwdArgs {
@@ -75,11 +88,32 @@ struct BwdArgs {
   uint64_t head_mask;       // heads this launch computes (bit h), ~0 = all
 };
 
+// Per problem of a grouped forward launch, for its schedule: the problem's
+// entries are ebase .. ebase + B - 1 of the group's entry list.
+struct GroupSchedProblem {
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  int B, ebase;
+  int wl, wr;
+  int max_q, max_kv;
+};
+constexpr int kMaxGroupProblems = 256;  // per launch group
+
+// One launch group's schedule job (the schedule kernel runs one CTA per group).
+struct GroupSchedJob {
+  const GroupSchedProblem* probs;
+  int n_probs, n_entries, block_n;
+  int4* info;
+  int32_t* eprob;
+};
+
 // Launchers (defined next to their kernels).
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
                             int32_t* order, int4* info, int max_q, int max_kv,
                             DeviceStatus* status, cudaStream_t stream);
+cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
+                                  int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, int sms,
                            cudaStream_t stream);
@@ -97,30 +131,47 @@ cudaError_t launch_backward(const BwdArgs& a, int D, const CUtensorMap& tq,
 // so its latency hides behind the current unit.
 struct GdpaUnit {
   int h, q0, Lq, k0, Lk;
+  int prob;  // problem of a grouped launch (0 for a single problem)
 };
 
-struct UnitStream {
+// GROUPED: units of several problems (per-entry problem index, per-problem
+// head counts and masks); otherwise one problem with an optional head mask.
+template <bool GROUPED>
+struct UnitStreamT {
   const int4* info;
+  const int32_t* eprob;      // problem of each sorted entry (GROUPED)
+  const FwdProblem* probs;   // per-problem heads and head masks (GROUPED)
   int H, n_units, round, u;
-  uint64_t mask;  // heads to walk (bit h); ~0 = all
+  uint64_t mask;  // heads to walk (bit h); ~0 = all (single problem)
   int4 nxt;
+  int nprob;      // problem of the unit next() returns
   __device__ __forceinline__ static int index(int round, int cta, int grid) {
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
   }
-  // first unit at or after `round` whose head is walked
+  __device__ __forceinline__ static bool head_on(uint64_t m, int h) {
+    return m == ~0ull || (h < 64 && ((m >> h) & 1ull));
+  }
+  // first unit at or after `round` this walk computes
   __device__ __forceinline__ void settle() {
     for (;;) {
       u = index(round, blockIdx.x, gridDim.x);
-      if (u >= n_units || mask == ~0ull) break;
-      const int h = u % H;
-      if (h < 64 && ((mask >> h) & 1ull)) break;
+      if (u >= n_units) break;
+      if constexpr (GROUPED) {
+        const int h = u % H;
+        nprob = __ldg(eprob + u / H);
+        if (h < probs[nprob].H && head_on(probs[nprob].head_mask, h)) break;
+      } else {
+        if (mask == ~0ull || head_on(mask, u % H)) break;
+      }
       ++round;
     }
     nxt = u < n_units ? __ldg(info + u / H) : make_int4(0, 0, 0, 0);
   }
-  __device__ __forceinline__ UnitStream(const int4* info_, int H_, int n_units_,
-                                        uint64_t mask_ = ~0ull)
-      : info(info_), H(H_), n_units(n_units_), round(0), mask(mask_) {
+  __device__ __forceinline__ UnitStreamT(const int4* info_, int H_, int n_units_,
+                                         uint64_t mask_ = ~0ull, const int32_t* eprob_ = nullptr,
+                                         const FwdProblem* probs_ = nullptr)
+      : info(info_), eprob(eprob_), probs(probs_), H(H_), n_units(n_units_), round(0),
+        mask(mask_), nprob(0) {
     settle();
   }
   // The unit the next call of next() returns, without advancing.
@@ -131,6 +182,7 @@ struct UnitStream {
     t.Lq = nxt.y;
     t.k0 = nxt.z;
     t.Lk = nxt.w;
+    t.prob = GROUPED ? nprob : 0;
     return true;
   }
   __device__ __forceinline__ bool next(GdpaUnit& t) {
@@ -140,5 +192,6 @@ struct UnitStream {
     return true;
   }
 };
+using UnitStream = UnitStreamT<false>;
 
 }  // namespace gdpa

@@ -129,7 +129,94 @@ __global__ void __launch_bounds__(kSchedThreads)
   if (B == 0 && tid == 0) tile_start[0] = 0;
 }
 
+// Grouped forward: per launch group (one CTA each), the entries (problem,
+// sample) of every problem in the group, sorted by the same cost (each
+// problem's own band), longest first, ties by ascending entry; info[i] is the
+// sorted entry's sample descriptor and eprob[i] its problem.  Problem tables in
+// shared memory.  The caller clears the workspace status beforehand.
+__global__ void __launch_bounds__(kSchedThreads)
+    gdpa_group_schedule_kernel(const GroupSchedJob* __restrict__ jobs, int BM,
+                               DeviceStatus* status) {
+  extern __shared__ unsigned long long keys[];
+  __shared__ GroupSchedProblem sp[kMaxGroupProblems];
+  const int tid = threadIdx.x;
+  const GroupSchedJob job = jobs[blockIdx.x];
+  const GroupSchedProblem* __restrict__ probs = job.probs;
+  const int n_probs = job.n_probs, n_entries = job.n_entries, BN = job.block_n;
+  int4* __restrict__ info = job.info;
+  int32_t* __restrict__ eprob = job.eprob;
+  for (int i = tid; i < n_probs; i += kSchedThreads) sp[i] = probs[i];
+  __syncthreads();
+  auto problem_of = [&](int e) {  // last problem whose first entry is <= e
+    int lo = 0, hi = n_probs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sp[mid].ebase <= e) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  int n = 1;
+  while (n < n_entries) n <<= 1;
+  for (int i = tid; i < n; i += kSchedThreads) {
+    unsigned long long key = ~0ull;
+    if (i < n_entries) {
+      const GroupSchedProblem& P = sp[problem_of(i)];
+      const int b = i - P.ebase;
+      const int Lq = P.q_offsets[b + 1] - P.q_offsets[b];
+      const int Lk = P.kv_offsets[b + 1] - P.kv_offsets[b];
+      unsigned long long c = sample_cost(Lq, Lk, BM, BN, P.wl, P.wr);
+      if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
+      key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < n; i += kSchedThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          const bool ascending = (i & k) == 0;
+          if ((x > y) == ascending) {
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int pos = tid; pos < n_entries; pos += kSchedThreads) {
+    const int e = (int)(keys[pos] & 0xFFFFFFFFull);
+    const int p = problem_of(e);
+    const GroupSchedProblem& P = sp[p];
+    const int b = e - P.ebase;
+    const int q0 = P.q_offsets[b], Lq = P.q_offsets[b + 1] - q0;
+    const int k0 = P.kv_offsets[b], Lk = P.kv_offsets[b + 1] - k0;
+    // a sample longer than its problem's declared bound is reported and skipped
+    const bool bad = Lq > P.max_q || Lk > P.max_kv;
+    if (bad && status) record_error(status, 6, e);
+    info[pos] = make_int4(q0, bad ? 0 : Lq, k0, bad ? 0 : Lk);
+    eprob[pos] = p;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
+                                  int block_m, DeviceStatus* status, cudaStream_t stream) {
+  if (n_jobs < 1 || max_entries > kMaxSortBatch) return cudaErrorInvalidValue;
+  int n = 1;
+  while (n < max_entries) n <<= 1;
+  const size_t smem = (size_t)n * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(gdpa_group_schedule_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(kMaxSortBatch * sizeof(unsigned long long)));
+  if (e != cudaSuccess) return e;
+  gdpa_group_schedule_kernel<<<n_jobs, kSchedThreads, smem, stream>>>(jobs, block_m, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,

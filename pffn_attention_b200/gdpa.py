@@ -25,7 +25,8 @@ BIAS = {"none": 0, "add": 1, "gate": 2}
 
 EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
-            "gdpa_version", "gdpa_forward_no_alloc")
+            "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
+            "gdpa_forward_grouped")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -37,6 +38,13 @@ class gdpa_params_t(ctypes.Structure):
                 ("bias_kind", ctypes.c_int), ("debug_flags", ctypes.c_int),
                 ("wait_timeout_us", ctypes.c_int),
                 ("head_phi", ctypes.POINTER(ctypes.c_int32))]
+
+
+class gdpa_forward_problem_t(ctypes.Structure):
+    _fields_ = [("params", gdpa_params_t), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("q_offsets", ctypes.c_void_p),
+                ("kv_offsets", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
 
 class GdpaError(RuntimeError):
@@ -78,6 +86,11 @@ def load(path: str = LIB_PATH):
     lib.gdpa_forward_no_alloc.restype = ctypes.c_int
     lib.gdpa_version.argtypes = []
     lib.gdpa_version.restype = ctypes.c_int
+    FP = ctypes.POINTER(gdpa_forward_problem_t)
+    lib.gdpa_forward_grouped_workspace_size.argtypes = [FP, ctypes.c_int]
+    lib.gdpa_forward_grouped_workspace_size.restype = sz
+    lib.gdpa_forward_grouped.argtypes = [FP, ctypes.c_int, vp, sz, st]
+    lib.gdpa_forward_grouped.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -91,6 +104,17 @@ def gdpa_forward(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, workspace, wor
                  stream) -> int:
     return int(load().gdpa_forward(ctypes.byref(p), q, k, v, q_offsets, kv_offsets, bias, o, lse,
                                    workspace, workspace_bytes, stream))
+
+
+def gdpa_forward_grouped_workspace_size(problems) -> int:
+    """problems: a ctypes array of gdpa_forward_problem_t (or None)."""
+    n = 0 if problems is None else len(problems)
+    return int(load().gdpa_forward_grouped_workspace_size(problems, n))
+
+
+def gdpa_forward_grouped(problems, workspace, workspace_bytes, stream) -> int:
+    n = 0 if problems is None else len(problems)
+    return int(load().gdpa_forward_grouped(problems, n, workspace, workspace_bytes, stream))
 
 
 def gdpa_forward_no_alloc(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, stream) -> int:
@@ -204,6 +228,43 @@ def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1
                       _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "gdpa_forward")
     return out, lse, workspace
+
+
+def forward_grouped(problems, *, workspace=None, stream=None):
+    """Several GDPA problems in one call.  problems: a list of dicts with the
+    tensors q, k, v, q_offsets, kv_offsets (and optional bias, out, lse) and the
+    keyword arguments of forward() (phi, scale, window, bias_kind,
+    max_seqlen_q, max_seqlen_kv, head_phi).  Returns ([(o, lse), ...], workspace)."""
+    import torch
+    arr = (gdpa_forward_problem_t * len(problems))()
+    outs, keep = [], []
+    for i, d in enumerate(problems):
+        q, k, v = d["q"], d["k"], d["v"]
+        total_q, H, D = q.shape
+        p = make_params(d["q_offsets"].numel() - 1, H, D, total_q, k.shape[0],
+                        phi=d.get("phi", "silu"), scale=d.get("scale", 1.0),
+                        window=d.get("window", (-1, -1)), bias_kind=d.get("bias_kind", "none"),
+                        max_seqlen_q=d.get("max_seqlen_q", 0),
+                        max_seqlen_kv=d.get("max_seqlen_kv", 0), head_phi=d.get("head_phi"))
+        o = d.get("out") if d.get("out") is not None else torch.empty_like(q)
+        lse = d.get("lse")
+        if lse is None and _any_softmax(p):
+            lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+        keep.append(p)
+        arr[i].params = p
+        for name, t in (("q", q), ("k", k), ("v", v), ("q_offsets", d["q_offsets"]),
+                        ("kv_offsets", d["kv_offsets"]), ("bias", d.get("bias")), ("o", o),
+                        ("lse", lse)):
+            setattr(arr[i], name, _ptr(t))
+        outs.append((o, lse))
+    if workspace is None:
+        n = gdpa_forward_grouped_workspace_size(arr)
+        if n == 0:
+            raise GdpaError(1, "gdpa_forward_grouped_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=problems[0]["q"].device)
+    rc = gdpa_forward_grouped(arr, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "gdpa_forward_grouped")
+    return outs, workspace
 
 
 def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=1.0,

@@ -109,3 +109,24 @@ def test_head_phi_validation(lib):
     mixed = gdpa.gdpa_workspace_size(_params(H=3, phi=0, head_phi=[0, 1, 3]), 1)
     assert mixed > plain > 0
     assert gdpa.gdpa_workspace_size(_params(H=3, phi=0, head_phi=[3, 2, 0]), 1) == plain
+
+
+def test_grouped_forward_validation(lib):
+    """Grouped calls are validated on the host before any launch: no problems,
+    a problem with bad parameters or pointers, or an unaligned workspace."""
+    def arr(*params):
+        a = (gdpa.gdpa_forward_problem_t * len(params))()
+        for i, p in enumerate(params):
+            a[i].params = p
+            for name in ("q", "k", "v", "q_offsets", "kv_offsets", "o"):
+                setattr(a[i], name, FAKE)
+        return a
+    assert gdpa.gdpa_forward_grouped_workspace_size(None) == 0
+    good = arr(_params(), _params(H=3, D=128, phi=1))
+    assert gdpa.gdpa_forward_grouped_workspace_size(good) > 0
+    assert gdpa.gdpa_forward_grouped_workspace_size(arr(_params(), _params(D=48))) == 0
+    nobias = arr(_params(bias_kind=2))  # a gate without its tensor
+    assert gdpa.gdpa_forward_grouped(nobias, FAKE, 1 << 20, None) == 1
+    assert gdpa.gdpa_forward_grouped(None, FAKE, 1 << 20, None) == 1
+    # tensor maps live in the workspace: it must be 64-byte aligned
+    assert gdpa.gdpa_forward_grouped(good, FAKE + 16, 1 << 20, None) == 1

@@ -1,0 +1,117 @@
+"""Grouped forward: several problems with their own shapes, activations,
+bands and biases in one call, as event-level personalisation runs them.
+
+Each problem's output must equal gdpa_forward on that problem alone (the same
+per-unit arithmetic, so bit for bit) and match the oracle.
+"""
+import copy
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import compare, compare_lse
+from workloads import (BIAS_ADD, BIAS_GATE, BIAS_NONE, PHI_GELU, PHI_IDENTITY, PHI_SILU,
+                       PHI_SOFTMAX, make_workload)
+
+pytestmark = pytest.mark.gpu
+
+NAMES = {PHI_SILU: "silu", PHI_SOFTMAX: "softmax", PHI_IDENTITY: "identity", PHI_GELU: "gelu"}
+
+
+def _problems():
+    """(workload, head_phi or None) per problem."""
+    out = []
+    # D = 128, softmax, gate, causal band (the sliding-window shape)
+    out.append((make_workload(4, seed=400, q_lens=[300, 1, 129], kv_lens=[300, 1, 129], H=3,
+                              window=(127, 0), bias=BIAS_GATE), None))
+    # D = 128, SiLU, at most 64 keys (64-key blocks)
+    out.append((make_workload(2, seed=401, q_lens=[200, 64, 7, 130], kv_lens=[64, 1, 33, 64],
+                              H=2, D=128, phi=PHI_SILU, scale=1.0,
+                              kv_std=1.0 / np.sqrt(128)), None))
+    # D = 64, one activation per head, additive bias
+    out.append((make_workload(2, seed=402, q_lens=[150, 90, 1], kv_lens=[200, 64, 300], H=4,
+                              D=64, scale=1.0, kv_std=1.0 / np.sqrt(64), bias=BIAS_ADD),
+                [PHI_SOFTMAX, PHI_SILU, PHI_GELU, PHI_IDENTITY]))
+    # D = 128, softmax, no bias: shares a launch with the first problem
+    out.append((make_workload(3, seed=403, q_lens=[32, 32, 32, 5, 250], kv_lens=[700, 128, 9, 1,
+                                                                                   256], H=5),
+                None))
+    # a problem whose samples have no queries
+    out.append((make_workload(2, seed=404, q_lens=[0, 0], kv_lens=[10, 3], H=2, D=64, scale=1.0,
+                              kv_std=1.0 / np.sqrt(64)), None))
+    return out
+
+
+def _to_dev(w, head_phi):
+    dev = torch.device("cuda")
+    d = dict(q=w.q.to(dev), k=w.k.to(dev), v=w.v.to(dev),
+             q_offsets=torch.tensor(w.q_offsets, dtype=torch.int32, device=dev),
+             kv_offsets=torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev),
+             bias=None if w.bias is None else w.bias.to(dev), phi=NAMES[w.phi], scale=w.scale,
+             window=(w.window_left, w.window_right), bias_kind=w.bias_kind,
+             max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv)
+    if head_phi is not None:
+        d["head_phi"] = [NAMES[x] for x in head_phi]
+    return d
+
+
+def test_grouped_equals_separate_calls_and_oracle(cuda_lib):
+    probs = _problems()
+    dev_probs = [_to_dev(w, hp) for w, hp in probs]
+    outs, ws = cuda_lib.forward_grouped(dev_probs)
+    assert cuda_lib.device_status(ws) == 0
+    torch.cuda.synchronize()
+    for (w, hp), d, (o, lse) in zip(probs, dev_probs, outs):
+        # the same problem alone
+        kw = {k: d[k] for k in ("phi", "scale", "window", "bias", "bias_kind", "max_seqlen_q",
+                                "max_seqlen_kv")}
+        if hp is not None:
+            kw["head_phi"] = d["head_phi"]
+        o1, lse1, ws1 = cuda_lib.forward(d["q"], d["k"], d["v"], d["q_offsets"],
+                                         d["kv_offsets"], **kw)
+        assert cuda_lib.device_status(ws1) == 0
+        assert torch.equal(o, o1)
+        heads = hp if hp is not None else [w.phi] * w.H
+        for h, phi in enumerate(heads):
+            if phi == PHI_SOFTMAX:
+                assert torch.equal(lse[h], lse1[h])
+        # and the oracle, head by head with that head's activation
+        for phi in sorted(set(heads)):
+            wp = copy.copy(w)
+            wp.phi = phi
+            ro, rlse = oracle.forward_workload(wp)
+            for h in [i for i, x in enumerate(heads) if x == phi]:
+                compare(f"O[h{h}]", o[:, h], ro[:, h])
+                if phi == PHI_SOFTMAX:
+                    compare_lse(lse[h], rlse[h])
+
+
+def test_grouped_many_small_problems(cuda_lib):
+    """Forty event-type problems of mixed shapes in one call."""
+    rng = np.random.default_rng(405)
+    probs = []
+    for i in range(40):
+        H = int(rng.integers(1, 5))
+        D = int(rng.choice([32, 64, 128]))
+        B = int(rng.integers(1, 4))
+        ql = rng.integers(1, 200, B).tolist()
+        kl = rng.integers(1, 150, B).tolist()
+        phi = int(rng.choice([PHI_SOFTMAX, PHI_SILU]))
+        if phi == PHI_SOFTMAX:
+            w = make_workload(3, seed=500 + i, q_lens=ql, kv_lens=kl, H=H, D=D,
+                              scale=1.0 / np.sqrt(D))
+        else:
+            w = make_workload(2, seed=500 + i, q_lens=ql, kv_lens=kl, H=H, D=D, phi=phi,
+                              scale=1.0, kv_std=1.0 / np.sqrt(D))
+        probs.append((w, None))
+    dev_probs = [_to_dev(w, None) for w, _ in probs]
+    outs, ws = cuda_lib.forward_grouped(dev_probs)
+    assert cuda_lib.device_status(ws) == 0
+    torch.cuda.synchronize()
+    for (w, _), (o, lse) in zip(probs, outs):
+        ro, rlse = oracle.forward_workload(w)
+        compare("O", o, ro)
+        if w.phi == PHI_SOFTMAX:
+            compare_lse(lse, rlse)
