@@ -96,7 +96,49 @@ typedef struct {
                          head (H <= 64); NULL = every head uses phi.  Read during
                          the call only.  LSE rows of non-softmax heads are not
                          written. */
+  /* Rotary temporal embedding of Q and K (gdpa_rotary_table below): device
+   * tables of rotations, [total_q][D/2] for the queries and [total_kv][D/2] for
+   * the keys, 16-byte aligned; both NULL = no rotation.  Give both or neither
+   * (self-attention passes the same table twice).  The forward turns each Q
+   * tile and K block as it arrives in shared memory, before QK^T; V is not
+   * rotated.  Not accepted by gdpa_backward or the grouped forward yet
+   * (GDPA_ERR_UNSUPPORTED). */
+  const void* rope_q;
+  const void* rope_kv;
 } gdpa_params_t;
+
+/* ---- Rotary temporal embedding (Kunlun paper review §2.2: RoPE extended from
+ * positions to log-scaled time gaps, with position frequencies theta_i and time
+ * frequencies phi_i; the page's formulas were lost, this is the reading used).
+ *
+ * Token t (0-based within its sample) of a jagged sequence has the gap
+ * dt_t = time[t] - time[t-1] to the previous event of its sample (0 for the
+ * first token; a negative gap counts as 0) and the scaled gap
+ * tau_t = ln(1 + dt_t / time_scale).  Pair i = (2i, 2i+1) of every head vector
+ * of that token turns by alpha_{t,i} = t * theta_i + tau_t * phi_i:
+ *   x'_2i = x_2i cos(alpha) - x_2i+1 sin(alpha),
+ *   x'_2i+1 = x_2i sin(alpha) + x_2i+1 cos(alpha). */
+typedef struct {
+  int D;               /* head dim: 32, 64 or 128 */
+  float time_scale;    /* tau_scale, > 0, in the unit of time[] */
+  const float* theta;  /* optional host [D/2] position frequencies; NULL = 10000^(-2i/D) */
+  const float* phi;    /* optional host [D/2] time frequencies; NULL = theta */
+} gdpa_rotary_params_t;
+
+/* Bytes of a rotation table for `total` tokens: total * D/2 * 4
+ * ((cos, sin) of each angle as two fp16 values, cos first). */
+GDPA_API size_t gdpa_rotary_table_bytes(int D, int64_t total);
+
+/* Fills table [total][D/2] (device, 16-byte aligned, the caller's) for the
+ * jagged sequence given by offsets [B+1] (device int32, as elsewhere) and
+ * time [total] (device int64 event times, non-decreasing within a sample for
+ * the gaps to mean anything).  The angle is formed and reduced modulo 2 pi in
+ * fp64, then its cosine and sine are taken in fp32 and rounded to fp16.  One
+ * table serves every head, the forward and the backward, and every layer that
+ * sees the same sequence.  Asynchronous on stream. */
+GDPA_API gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, int64_t total,
+                                         const int32_t* offsets, const int64_t* time,
+                                         void* table, gdpa_stream_t stream);
 
 /* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward
  * (backward = 1) needs for these parameters.  0 on invalid parameters. */

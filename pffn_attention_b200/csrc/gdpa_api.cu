@@ -74,6 +74,10 @@ gdpa_status_t check_params(const gdpa_params_t* p) {
   if (p->bias_kind < 0 || p->bias_kind > 2) return GDPA_ERR_UNSUPPORTED;
   if (p->B > kMaxSortBatch) return GDPA_ERR_UNSUPPORTED;
   if ((int64_t)p->H * p->B >= (int64_t(1) << 31)) return GDPA_ERR_UNSUPPORTED;
+  // rotation tables: both or neither, 16-byte aligned (one 16-byte load per
+  // four pairs)
+  if ((p->rope_q == nullptr) != (p->rope_kv == nullptr)) return GDPA_ERR_INVALID_ARG;
+  if (p->rope_q && (!aligned16(p->rope_q) || !aligned16(p->rope_kv))) return GDPA_ERR_INVALID_ARG;
   return GDPA_OK;
 }
 
@@ -188,8 +192,6 @@ struct GroupedLayout {
   size_t off_jobs = 0, tables_end = 0, total = 0;
 };
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 // Validates every problem, forms the launch groups and lays out the workspace.
 // Nothing touches the device.
 gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
@@ -202,6 +204,7 @@ gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
     gdpa_status_t st = check_forward_args(p, f.q, f.k, f.v, f.q_offsets, f.kv_offsets, f.bias,
                                           f.o, f.lse);
     if (st != GDPA_OK) return st;
+    if (p->rope_q) return GDPA_ERR_UNSUPPORTED;  // rotation: single-problem calls only
     const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p), p->debug_flags);
     for (int phi = 0; phi <= 3; ++phi) {
       const uint64_t heads = phi_heads(p, phi);
@@ -351,6 +354,8 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.p0.wl = p->window_left;
   a.p0.wr = p->window_right;
   a.p0.scale = p->scale;
+  a.rope_q = static_cast<const uint32_t*>(p->rope_q);
+  a.rope_kv = static_cast<const uint32_t*>(p->rope_kv);
   // one launch per activation present (a per-head activation vector groups
   // the heads; each launch walks only its own heads' units)
   for (int phi = 0; phi <= 3; ++phi) {
@@ -374,6 +379,7 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
                             void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
   gdpa_status_t st = check_params(p);
   if (st != GDPA_OK) return st;
+  if (p->rope_q) return GDPA_ERR_UNSUPPORTED;  // rotary backward: not built yet
   if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
   // a bias gradient needs a bias; it is fp32 [H][total_kv]
   if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
@@ -594,6 +600,38 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;
+}
+
+size_t gdpa_rotary_table_bytes(int D, int64_t total) {
+  if ((D != 32 && D != 64 && D != 128) || total < 0) return 0;
+  return (size_t)total * (size_t)(D / 2) * 4u;
+}
+
+gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, int64_t total,
+                                const int32_t* offsets, const int64_t* time, void* table,
+                                gdpa_stream_t stream) {
+  if (!r) return GDPA_ERR_INVALID_ARG;
+  if (r->D != 32 && r->D != 64 && r->D != 128) return GDPA_ERR_UNSUPPORTED;
+  if (!(r->time_scale > 0.f) || !std::isfinite(r->time_scale)) return GDPA_ERR_INVALID_ARG;
+  if (B < 0 || B > kMaxSortBatch || total < 0 || total >= (int64_t(1) << 31))
+    return GDPA_ERR_INVALID_ARG;
+  if (B == 0 || total == 0) return GDPA_OK;
+  if (!offsets || !time || !table || !aligned16(table)) return GDPA_ERR_INVALID_ARG;
+  RotaryArgs a{};
+  a.D = r->D;
+  a.B = B;
+  a.total = total;
+  a.time_scale = r->time_scale;
+  for (int i = 0; i < r->D / 2; ++i) {
+    const float th = r->theta ? r->theta[i] : (float)std::pow(10000.0, -2.0 * i / r->D);
+    const float ph = r->phi ? r->phi[i] : th;
+    if (!std::isfinite(th) || !std::isfinite(ph)) return GDPA_ERR_INVALID_ARG;
+    a.theta[i] = th;
+    a.phi[i] = ph;
+  }
+  cudaError_t e = launch_rotary_table(a, offsets, time, static_cast<uint32_t*>(table),
+                                      (cudaStream_t)stream);
+  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 
 gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {

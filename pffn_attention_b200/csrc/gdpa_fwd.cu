@@ -36,6 +36,8 @@
 #include <cfloat>
 #include <climits>
 
+#include <cuda_fp16.h>
+
 #include "gdpa_internal.h"
 
 namespace gdpa {
@@ -54,11 +56,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kInvSqrt2 = 0.7071067811865476f;  // Phi(x) = (1 + erf(x / sqrt 2)) / 2
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
-template <int D_, int BN_, bool GROUPED_>
+template <int D_, int BN_, bool GROUPED_, bool ROPE_ = false>
 struct FwdCfg {
   static constexpr int D = D_;
   static constexpr int BN = BN_;
   static constexpr bool GROUPED = GROUPED_;  // units of several problems
+  static constexpr bool ROPE = ROPE_;        // Q and K turned by the rotation tables
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
   // (64 B, 64-byte swizzle) when D = 32.
@@ -90,7 +93,10 @@ struct FwdCfg {
   static constexpr int B_OEMPTY = B_OFULL + 2;
   static constexpr int B_BFULL = B_OEMPTY + 2;
   static constexpr int B_BEMPTY = B_BFULL + 4;
-  static constexpr int NBARS = B_BEMPTY + 4;
+  // rotary: Q of slot s, K of ring stage i turned and ready for the MMA
+  static constexpr int B_QROT = B_BEMPTY + 4;
+  static constexpr int B_KROT = B_QROT + 2;
+  static constexpr int NBARS = B_KROT + NKV;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem addr, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES;  // base is 1024-aligned (checked at entry)
@@ -384,12 +390,15 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
       if (z.ns < z.nkv && z.ns == z.npv) {
         const uint32_t ring = z.kv0 + (uint32_t)z.ns;
         const int st = (int)(ring % C::NKV);
-        bool ok = z.ns > 0 || mbar_test_wait(sm.bar(C::B_QFULL + s), z.tq & 1);
+        // Q and K are ready once loaded, or once turned when rotary
+        constexpr int QREADY = C::ROPE ? C::B_QROT : C::B_QFULL;
+        constexpr int KREADY = C::ROPE ? C::B_KROT : C::B_KVFULL;
+        bool ok = z.ns > 0 || mbar_test_wait(sm.bar(QREADY + s), z.tq & 1);
         // The other slot may be far ahead or behind in the ring: the stage's
         // full barrier identifies this ring index's phase only once the
         // producer has started loading it (the previous content's phase done).
         ok = ok && sm.kv_tag()[st] == (int)ring;
-        ok = ok && mbar_test_wait(sm.bar(C::B_KVFULL + st), (ring / C::NKV) & 1);
+        ok = ok && mbar_test_wait(sm.bar(KREADY + st), (ring / C::NKV) & 1);
         ok = ok && (z.pc == 0 || mbar_test_wait(sm.bar(C::B_PVDONE + s), (z.pc - 1) & 1));
         if (ok) {
           tc_fence_after();
@@ -501,6 +510,116 @@ __device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, int s, bool softm
       ++bc;
     }
   }
+}
+
+// ------------------------------------------------------------------ rotation warps
+// Pair (x0, x1) of bf16 values turned by the angle whose (cos, sin) is the
+// fp16 pair cs.
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t x, uint32_t cs) {
+  const float x0 = __uint_as_float(x << 16), x1 = __uint_as_float(x & 0xffff0000u);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cs));
+  return pack_bf16x2(fmaf(x0, f.x, -x1 * f.y), fmaf(x0, f.y, x1 * f.x));
+}
+
+// Rows [r0, min(r1, nvalid)) of a swizzled tile of `rows` rows turned in place
+// by the table rows of tokens tok0 + row.  A lane takes 16-byte chunks (four
+// pairs), two at a time (four spill under the control warps' register budget).
+template <class C>
+__device__ __forceinline__ void rotate_tile(uint32_t tile, int rows, int r0, int r1, int nvalid,
+                                            const uint32_t* __restrict__ tab, int64_t tok0,
+                                            int lane) {
+  constexpr int CH = C::D / 8;              // chunks per row
+  constexpr int CPP = C::PANEL_BYTES / 16;  // chunks per panel row
+  const int n = (min(r1, nvalid) - r0) * CH;
+  auto addr_of = [&](int it, int& row, int& ch) {
+    row = r0 + it / CH;
+    ch = it % CH;
+    const int pnl = ch / CPP, cw = ch % CPP;
+    const int swz = C::PANEL_BYTES == 128 ? (row & 7) : ((row >> 1) & 3);
+    return tile + (uint32_t)(pnl * rows * C::PANEL_BYTES + row * C::PANEL_BYTES + ((cw ^ swz) << 4));
+  };
+  for (int base = 0; base < n; base += 64) {
+    uint4 cs[2], x[2];
+    uint32_t ad[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int it = base + u * 32 + lane;
+      if (it < n) {
+        int row, ch;
+        ad[u] = addr_of(it, row, ch);
+        cs[u] = __ldg(reinterpret_cast<const uint4*>(tab + (tok0 + row) * (C::D / 2) + ch * 4));
+        x[u] = ld_shared_v4(ad[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (base + u * 32 + lane < n)
+        st_shared_v4(ad[u], rotate_pair(x[u].x, cs[u].x), rotate_pair(x[u].y, cs[u].y),
+                     rotate_pair(x[u].z, cs[u].z), rotate_pair(x[u].w, cs[u].w));
+    }
+  }
+}
+
+// Rotary temporal embedding (Kunlun paper review §2.2): warps 2 and 3 turn
+// each Q tile, and each K block as it is loaded, in shared memory between the
+// TMA load and the S MMA, in the producer's order; each warp takes half the
+// rows.  The issuer waits for the turned tiles.  With a bias the same warps
+// also write beta (both slots, in tile order, one block after its K block, so
+// every wait depends only on work already done).
+template <class C>
+__device__ void role_rotary(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
+  volatile int* abort = sm.abort_flag();
+  const int w = (threadIdx.x >> 5) - 2;  // 0 or 1
+  const int lane = threadIdx.x & 31;
+  const bool has_bias = a.p0.bias_kind != 0;
+  uint32_t nq[2] = {0u, 0u}, bc[2] = {0u, 0u};
+  TileWalk<C> walk(a);
+  FTile x{};
+#define ROT_WAIT(bar_, par_, where_)                                                   \
+  do {                                                                               \
+    bool ok_ = mbar_wait(sm.bar(bar_), (par_), abort, a.status, a.timeout_ns, where_); \
+    if (!__all_sync(0xffffffffu, ok_)) return;                                       \
+  } while (0)
+  while (walk.next(x)) {
+    if (x.kb1 <= x.kb0) continue;  // nothing loaded: the phi warpgroup writes zeros
+    const int s = x.slot;
+    ROT_WAIT(C::B_QFULL + s, nq[s] & 1, 0x500 + C::B_QFULL + s);
+    rotate_tile<C>(sm.q(s), kBlockM, w * (kBlockM / 2), (w + 1) * (kBlockM / 2), x.Lq - x.m0,
+                   a.rope_q, (int64_t)x.q0 + x.m0, lane);
+    fence_proxy_async_smem();  // the MMA reads the turned tile through the async proxy
+    mbar_arrive(sm.bar(C::B_QROT + s));
+    ++nq[s];
+    const bool loads = !(x.resident && !x.unit_first);
+    for (int kb = x.kb0; kb < x.kb1; ++kb) {
+      if (loads) {
+        const uint32_t ring = x.kv0 + (uint32_t)(kb - x.kb0);
+        const int st = (int)(ring % C::NKV);
+        ROT_WAIT(C::B_KVFULL + st, (ring / C::NKV) & 1, 0x500 + C::B_KVFULL + st);
+        rotate_tile<C>(sm.k(st), C::BN, w * (C::BN / 2), (w + 1) * (C::BN / 2),
+                       x.Lk - kb * C::BN, a.rope_kv, (int64_t)x.k0 + kb * C::BN, lane);
+        fence_proxy_async_smem();
+        mbar_arrive(sm.bar(C::B_KROT + st));
+      }
+      if (has_bias) {
+        const int bb = bc[s] & 1;
+        ROT_WAIT(C::B_BEMPTY + 2 * s + bb, ((bc[s] >> 1) & 1) ^ 1, 0x500 + C::B_BEMPTY + 2 * s + bb);
+        float* dst = sm.bias(s, bb);
+        const float* src = a.p0.bias + (int64_t)x.h * a.p0.total_kv + x.k0;
+        for (int c = w * 32 + lane; c < C::BN; c += 64) {
+          const int key = kb * C::BN + c;
+          float beta = 0.f;
+          if (key < x.Lk) {
+            const float g = src[key];
+            beta = a.p0.bias_kind == 2 ? fminf(g, 0.f) - log1pf(__expf(-fabsf(g))) : g;
+          }
+          dst[c] = softmax ? beta * kLog2e : beta;
+        }
+        mbar_arrive(sm.bar(C::B_BFULL + 2 * s + bb));
+        ++bc[s];
+      }
+    }
+  }
+#undef ROT_WAIT
 }
 
 // ------------------------------------------------------------------ phi warpgroups
@@ -747,11 +866,11 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
 #undef PHI_WAIT
 }
 
-template <int D, int BN, bool SOFTMAX, bool GROUPED>
+template <int D, int BN, bool SOFTMAX, bool GROUPED, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
-  using C = FwdCfg<D, BN, GROUPED>;
+  using C = FwdCfg<D, BN, GROUPED, ROPE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
   sm.base = smem_u32(smem_raw);
@@ -776,8 +895,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sm.bar(C::B_KVEMPTY + i), 1);
     }
     for (int i = 0; i < 4; ++i) {
-      mbar_init(sm.bar(C::B_BFULL + i), 32);
+      mbar_init(sm.bar(C::B_BFULL + i), C::ROPE ? 64 : 32);  // rotary: both warps write beta
       mbar_init(sm.bar(C::B_BEMPTY + i), 128);
+    }
+    if (C::ROPE) {
+      for (int s = 0; s < 2; ++s) mbar_init(sm.bar(C::B_QROT + s), 64);
+      for (int i = 0; i < C::NKV; ++i) mbar_init(sm.bar(C::B_KROT + i), 64);
     }
     for (int i = 0; i < 8; ++i) sm.kv_tag()[i] = -1;
     *sm.abort_flag() = 0;
@@ -805,6 +928,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
     } else if (warp == 1) {
       if (lane == 0) role_mma<C>(a, sm, tmem);
+    } else if constexpr (C::ROPE) {
+      role_rotary<C>(a, sm, SOFTMAX);
     } else {
       // a grouped launch may mix problems with and without a bias
       if (C::GROUPED || a.p0.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
@@ -831,11 +956,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BN, bool SOFTMAX, bool GROUPED>
+template <int D, int BN, bool SOFTMAX, bool GROUPED, bool ROPE = false>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                        const CUtensorMap& tv, int sms, cudaStream_t stream) {
-  using C = FwdCfg<D, BN, GROUPED>;
-  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED>;
+  using C = FwdCfg<D, BN, GROUPED, ROPE>;
+  auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED, ROPE>;
   // the phi warpgroups raise their register budget with setmaxnreg, which waits
   // until the block's launch registers cover it: never launch a build whose
   // per-thread count would leave that wait unsatisfiable
@@ -869,11 +994,16 @@ cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorM
                            cudaStream_t stream) {
   const bool sm = a.phi == 1;
   const bool grouped = a.probs != nullptr;
+  const bool rope = a.rope_q != nullptr;
+  if (grouped && rope) return cudaErrorInvalidValue;
 #define GDPA_FWD_CASE(D_, BN_)                                                         \
   if (D == D_ && block_n == BN_) {                                                     \
     if (grouped)                                                                       \
       return sm ? launch_one<D_, BN_, true, true>(a, tq, tk, tv, sms, stream)          \
                 : launch_one<D_, BN_, false, true>(a, tq, tk, tv, sms, stream);        \
+    if (rope)                                                                          \
+      return sm ? launch_one<D_, BN_, true, false, true>(a, tq, tk, tv, sms, stream)   \
+                : launch_one<D_, BN_, false, false, true>(a, tq, tk, tv, sms, stream); \
     return sm ? launch_one<D_, BN_, true, false>(a, tq, tk, tv, sms, stream)           \
               : launch_one<D_, BN_, false, false>(a, tq, tk, tv, sms, stream);         \
   }

@@ -58,6 +58,10 @@ struct FwdArgs {
   const FwdProblem* probs;
   const CUtensorMap* maps;  // [problem][Q, K, V]
   FwdProblem p0;
+  // rotary temporal embedding (single problem): per-token (cos, sin) fp16
+  // pairs, [total_q][D/2] and [total_kv][D/2]; nullptr = no rotation
+  const uint32_t* rope_q;
+  const uint32_t* rope_kv;
 };
 
 struct BwdArgs {
@@ -112,6 +116,16 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
                             int32_t* order, int4* info, int max_q, int max_kv,
                             DeviceStatus* status, cudaStream_t stream);
+// Rotary temporal embedding table: angles t theta_i + tau_t phi_i per token.
+struct RotaryArgs {
+  float theta[64], phi[64];
+  double time_scale;
+  int D, B;
+  int64_t total;
+};
+cudaError_t launch_rotary_table(const RotaryArgs& r, const int32_t* offsets,
+                                const int64_t* time, uint32_t* table, cudaStream_t stream);
+
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,

@@ -26,7 +26,7 @@ BIAS = {"none": 0, "add": 1, "gate": 2}
 EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
             "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
-            "gdpa_forward_grouped")
+            "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -37,7 +37,13 @@ class gdpa_params_t(ctypes.Structure):
                 ("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
                 ("bias_kind", ctypes.c_int), ("debug_flags", ctypes.c_int),
                 ("wait_timeout_us", ctypes.c_int),
-                ("head_phi", ctypes.POINTER(ctypes.c_int32))]
+                ("head_phi", ctypes.POINTER(ctypes.c_int32)),
+                ("rope_q", ctypes.c_void_p), ("rope_kv", ctypes.c_void_p)]
+
+
+class gdpa_rotary_params_t(ctypes.Structure):
+    _fields_ = [("D", ctypes.c_int), ("time_scale", ctypes.c_float),
+                ("theta", ctypes.POINTER(ctypes.c_float)), ("phi", ctypes.POINTER(ctypes.c_float))]
 
 
 class gdpa_forward_problem_t(ctypes.Structure):
@@ -91,6 +97,11 @@ def load(path: str = LIB_PATH):
     lib.gdpa_forward_grouped_workspace_size.restype = sz
     lib.gdpa_forward_grouped.argtypes = [FP, ctypes.c_int, vp, sz, st]
     lib.gdpa_forward_grouped.restype = ctypes.c_int
+    lib.gdpa_rotary_table_bytes.argtypes = [ctypes.c_int, ctypes.c_int64]
+    lib.gdpa_rotary_table_bytes.restype = sz
+    lib.gdpa_rotary_table.argtypes = [ctypes.POINTER(gdpa_rotary_params_t), ctypes.c_int,
+                                      ctypes.c_int64, vp, vp, vp, st]
+    lib.gdpa_rotary_table.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -104,6 +115,15 @@ def gdpa_forward(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, workspace, wor
                  stream) -> int:
     return int(load().gdpa_forward(ctypes.byref(p), q, k, v, q_offsets, kv_offsets, bias, o, lse,
                                    workspace, workspace_bytes, stream))
+
+
+def gdpa_rotary_table_bytes(D: int, total: int) -> int:
+    return int(load().gdpa_rotary_table_bytes(int(D), int(total)))
+
+
+def gdpa_rotary_table(r: gdpa_rotary_params_t, B, total, offsets, time, table, stream) -> int:
+    return load().gdpa_rotary_table(ctypes.byref(r), int(B), int(total), offsets, time, table,
+                                    stream)
 
 
 def gdpa_forward_grouped_workspace_size(problems) -> int:
@@ -156,9 +176,10 @@ def gdpa_version() -> int:
 # ----------------------------------------------------------------- torch helpers
 def make_params(B, H, D, total_q, total_kv, *, phi=0, scale=1.0, window=(-1, -1),
                 bias_kind=0, max_seqlen_q=0, max_seqlen_kv=0, debug_flags=0,
-                wait_timeout_us=0, head_phi=None) -> gdpa_params_t:
+                wait_timeout_us=0, head_phi=None, rope=None) -> gdpa_params_t:
     """head_phi: optional sequence of H activations (names or GDPA_PHI values),
-    one per head; the params object keeps the array alive."""
+    one per head; the params object keeps the array alive.  rope: optional
+    (q table, kv table) pair of device tensors from rotary_table."""
     if isinstance(phi, str):
         phi = PHI[phi]
     if isinstance(bias_kind, str):
@@ -173,6 +194,9 @@ def make_params(B, H, D, total_q, total_kv, *, phi=0, scale=1.0, window=(-1, -1)
                       ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)) if arr is not None
                       else None)
     p._head_phi = arr  # owns the array the struct points to
+    if rope is not None:
+        p.rope_q, p.rope_kv = _ptr(rope[0]), _ptr(rope[1])
+        p._rope = rope  # keeps the tables alive with the params
     return p
 
 
@@ -206,18 +230,41 @@ def _check(rc: int, where: str):
         raise GdpaError(rc, where)
 
 
+def rotary_table(offsets, time, D, time_scale, *, theta=None, phi=None, out=None,
+                 stream=None):
+    """Rotation table [total, D/2] (int32 view of the fp16 (cos, sin) pairs) of
+    the rotary temporal embedding for the jagged sequence of offsets (int32
+    [B+1]) and time (int64 [total]) on the device.  theta / phi: optional
+    sequences of D/2 position / time frequencies."""
+    import torch
+    total = time.numel()
+    B = offsets.numel() - 1
+    if out is None:
+        out = torch.empty((total, D // 2), dtype=torch.int32, device=time.device)
+    def arr(x):
+        return None if x is None else (ctypes.c_float * len(x))(*[float(v) for v in x])
+    th, ph = arr(theta), arr(phi)
+    r = gdpa_rotary_params_t(int(D), float(time_scale),
+                             ctypes.cast(th, ctypes.POINTER(ctypes.c_float)) if th else None,
+                             ctypes.cast(ph, ctypes.POINTER(ctypes.c_float)) if ph else None)
+    rc = gdpa_rotary_table(r, B, total, _ptr(offsets), _ptr(time), _ptr(out), _stream(stream))
+    _check(rc, "gdpa_rotary_table")
+    return out
+
+
 def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1, -1),
             bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0, out=None, lse=None,
-            workspace=None, stream=None, params=None, head_phi=None):
+            workspace=None, stream=None, params=None, head_phi=None, rope=None):
     """O (and LSE for softmax) on the device.  Inputs are CUDA tensors:
-    q [total_q,H,D] bf16, k/v [total_kv,H,D] bf16, offsets int32 [B+1]."""
+    q [total_q,H,D] bf16, k/v [total_kv,H,D] bf16, offsets int32 [B+1];
+    rope: optional (q table, kv table) from rotary_table."""
     import torch
     total_q, H, D = q.shape
     total_kv = k.shape[0]
     B = q_offsets.numel() - 1
     p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
                               bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
-                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi)
+                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi, rope=rope)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and _any_softmax(p):

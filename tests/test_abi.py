@@ -130,3 +130,62 @@ def test_grouped_forward_validation(lib):
     assert gdpa.gdpa_forward_grouped(None, FAKE, 1 << 20, None) == 1
     # tensor maps live in the workspace: it must be 64-byte aligned
     assert gdpa.gdpa_forward_grouped(good, FAKE + 16, 1 << 20, None) == 1
+
+
+def test_rotary_validation(lib):
+    """Rotary tables: D, time scale, jagged sizes and alignment are checked on
+    the host; the tables must come as a pair; the backward and grouped forward
+    refuse them (not built)."""
+    def rp(D=64, scale=60.0):
+        return gdpa.gdpa_rotary_params_t(D, scale, None, None)
+    assert gdpa.gdpa_rotary_table_bytes(64, 10) == 10 * 32 * 4
+    assert gdpa.gdpa_rotary_table_bytes(48, 10) == 0
+    assert gdpa.gdpa_rotary_table(rp(D=48), 2, 10, FAKE, FAKE, FAKE, None) == 2
+    assert gdpa.gdpa_rotary_table(rp(scale=0.0), 2, 10, FAKE, FAKE, FAKE, None) == 1
+    assert gdpa.gdpa_rotary_table(rp(scale=float("inf")), 2, 10, FAKE, FAKE, FAKE, None) == 1
+    assert gdpa.gdpa_rotary_table(rp(), 2, 10, FAKE, FAKE, FAKE + 4, None) == 1
+    assert gdpa.gdpa_rotary_table(rp(), 2, 10, None, FAKE, FAKE, None) == 1
+    assert gdpa.gdpa_rotary_table(rp(), 0, 0, None, None, None, None) == 0  # nothing to do
+    bad_freq = (ctypes.c_float * 32)(*([1.0] * 31 + [float("nan")]))
+    r = gdpa.gdpa_rotary_params_t(64, 60.0, ctypes.cast(bad_freq, ctypes.POINTER(ctypes.c_float)),
+                                  None)
+    assert gdpa.gdpa_rotary_table(r, 2, 10, FAKE, FAKE, FAKE, None) == 1
+    p = _params()
+    p.rope_q = FAKE
+    assert gdpa.gdpa_workspace_size(p, 0) == 0  # one table without the other
+    p.rope_kv = FAKE + 8
+    assert gdpa.gdpa_workspace_size(p, 0) == 0  # unaligned
+    p.rope_kv = FAKE
+    assert gdpa.gdpa_workspace_size(p, 0) > 0
+    args = (FAKE,) * 8 + (None,) + (FAKE,) * 3 + (None, FAKE)  # no bias, no bias gradient
+    assert gdpa.gdpa_backward(p, *args, 1 << 20, None) == 2
+    a = (gdpa.gdpa_forward_problem_t * 1)()
+    a[0].params = p
+    for name in ("q", "k", "v", "q_offsets", "kv_offsets", "o"):
+        setattr(a[0], name, FAKE)
+    assert gdpa.gdpa_forward_grouped_workspace_size(a) == 0
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors have the C structs' sizes and field offsets."""
+    import subprocess
+    structs = {"gdpa_params_t": gdpa.gdpa_params_t,
+               "gdpa_forward_problem_t": gdpa.gdpa_forward_problem_t,
+               "gdpa_rotary_params_t": gdpa.gdpa_rotary_params_t}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "gdpa.h"', 'int main(void) {']
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{name}.{field} %zu\\n", offsetof({name}, {field}));')
+    lines.append('  return 0; }')
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe)])
+    got = dict(line.rsplit(" ", 1) for line in subprocess.check_output([str(exe)]).decode().split("\n")
+               if line)
+    for name, cls in structs.items():
+        assert int(got[name]) == ctypes.sizeof(cls), name
+        for field, _ in cls._fields_:
+            assert int(got[f"{name}.{field}"]) == getattr(cls, field).offset, (name, field)

@@ -1,0 +1,172 @@
+"""Rotary temporal embedding on the GPU vs the fp64 oracle (``oracle.rotary``):
+the rotation table, and the forward with Q and K turned in shared memory."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import rotary
+from parity import LSE_ABS, compare
+from workloads import (BIAS_GATE, BIAS_NONE, EVENT_TIME_SCALE, PHI_GELU, PHI_SILU, PHI_SOFTMAX,
+                       event_times, make_workload)
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(x, dtype=None):
+    return torch.as_tensor(x, dtype=dtype).cuda()
+
+
+def gpu_table(gdpa, offsets, times, D, **kw):
+    t = gdpa.rotary_table(_dev(offsets, torch.int32), _dev(times, torch.int64), D,
+                          EVENT_TIME_SCALE, **kw)
+    torch.cuda.synchronize()
+    return t
+
+
+def table_cos_sin(t):
+    h = t.view(torch.float16).float().cpu().numpy()  # [total, D] as (cos, sin) pairs
+    return h[:, 0::2], h[:, 1::2]
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_table_matches_oracle_angles(cuda_lib, D):
+    lens = [1, 5, 0, 300, 2048]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    times = event_times(lens, seed=D)
+    c, s = table_cos_sin(gpu_table(cuda_lib, off, times, D))
+    a = rotary.angles(off, times, D, EVENT_TIME_SCALE)
+    # fp16 rounding of values in [-1, 1] (half an ulp <= 2^-12) plus the fp32
+    # cosine and sine of the reduced angle
+    np.testing.assert_allclose(c, np.cos(a), rtol=0, atol=5e-4)
+    np.testing.assert_allclose(s, np.sin(a), rtol=0, atol=5e-4)
+
+
+def test_table_custom_frequencies(cuda_lib):
+    D = 64
+    lens = [7, 130]
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    times = event_times(lens, seed=3)
+    rng = np.random.default_rng(9)
+    th = rng.uniform(0, 1, D // 2).astype(np.float32)
+    ph = rng.uniform(0, 2, D // 2).astype(np.float32)
+    c, s = table_cos_sin(gpu_table(cuda_lib, off, times, D, theta=th, phi=ph))
+    a = rotary.angles(off, times, D, EVENT_TIME_SCALE, th.astype(np.float64), ph.astype(np.float64))
+    np.testing.assert_allclose(c, np.cos(a), atol=5e-4)
+    np.testing.assert_allclose(s, np.sin(a), atol=5e-4)
+
+
+def check_lse(lse, rlse, w, aq, ak):
+    """LSE against the oracle with a bound derived from the rotated operands.
+
+    The MMA takes the turned Q and K as bf16, so each turned element carries a
+    relative error of up to 2^-8 (bf16 rounding) plus about 2^-10 (the fp16
+    cosine and sine).  A score then moves by at most
+    scale * 2 * (2^-8 + 2^-10) * sum_d |q'_d k'_d| (used here with 2^-6), and
+    an LSE by at most the largest move of its row's scores; fp32 accumulation
+    keeps the plain bound of 2e-3 on top.
+    """
+    got = lse.detach().cpu().double().numpy()
+    ref = np.asarray(rlse)
+    neg = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(got), neg), "LSE -inf pattern differs"
+    qr = np.abs(rotary.rotate(w.q.double().numpy(), aq))
+    kr = np.abs(rotary.rotate(w.k.double().numpy(), ak))
+    bound = np.full(ref.shape, LSE_ABS)
+    for b in range(w.B):
+        qs = slice(int(w.q_offsets[b]), int(w.q_offsets[b + 1]))
+        ks = slice(int(w.kv_offsets[b]), int(w.kv_offsets[b + 1]))
+        if qs.stop == qs.start or ks.stop == ks.start:
+            continue
+        for h in range(w.H):
+            m = (qr[qs, h] @ kr[ks, h].T).max(axis=1)
+            bound[h, qs] += abs(w.scale) * 2.0 ** -6 * m
+    err = np.where(neg, 0.0, np.abs(np.where(neg, 0.0, got) - np.where(neg, 0.0, ref)))
+    assert (err <= bound).all(), f"LSE err {err.max():.3e} beyond bound (worst excess " \
+        f"{(err - bound).max():.3e})"
+
+
+def run(gdpa, w, tq, tk, **kw):
+    qo, ko = _dev(w.q_offsets, torch.int32), _dev(w.kv_offsets, torch.int32)
+    bias = w.bias.cuda() if w.bias is not None else None
+    o, lse, ws = gdpa.forward(w.q.cuda(), w.k.cuda(), w.v.cuda(), qo, ko, phi=w.phi,
+                              scale=w.scale, window=(w.window_left, w.window_right), bias=bias,
+                              bias_kind=w.bias_kind, max_seqlen_q=w.max_q,
+                              max_seqlen_kv=w.max_kv, rope=(tq, tk), **kw)
+    assert gdpa.device_status(ws) == 0
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def check(gdpa, w, seed, same_sequence):
+    """Self-attention (same_sequence) shares one table; otherwise queries and
+    keys have their own times."""
+    tq_np = event_times(w.q_lens, seed)
+    tk_np = tq_np if same_sequence else event_times(w.kv_lens, seed + 1)
+    tq = gpu_table(gdpa, w.q_offsets, tq_np, w.D)
+    tk = tq if same_sequence else gpu_table(gdpa, w.kv_offsets, tk_np, w.D)
+    o, lse = run(gdpa, w, tq, tk)
+    aq = rotary.angles(w.q_offsets, tq_np, w.D, EVENT_TIME_SCALE)
+    ak = rotary.angles(w.kv_offsets, tk_np, w.D, EVENT_TIME_SCALE)
+    ro, rlse = rotary.forward(w.q, w.k, w.v, w.q_offsets, w.kv_offsets, aq, ak, phi=w.phi,
+                              scale=w.scale, window=(w.window_left, w.window_right),
+                              bias=w.bias, bias_kind=w.bias_kind)
+    compare("O", o, ro)
+    if w.phi == PHI_SOFTMAX:
+        check_lse(lse, rlse, w, aq, ak)
+    return o
+
+
+# sliding-window self-attention is where the pages use temporal rotary; the
+# band keeps every key block streamed through the ring
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("window", [(127, 0), (40, 40), (-1, -1)])
+def test_self_attention(cuda_lib, D, window):
+    ql = [1, 60, 200, 333, 520, 129]
+    w = make_workload(4, seed=70 + D, q_lens=ql, kv_lens=ql, D=D, window=window,
+                      scale=1.0 / np.sqrt(D))
+    check(cuda_lib, w, seed=D, same_sequence=True)
+
+
+@pytest.mark.parametrize("phi", [PHI_SILU, PHI_GELU, PHI_SOFTMAX])
+@pytest.mark.parametrize("bias", [BIAS_NONE, BIAS_GATE])
+def test_activations_and_gate(cuda_lib, phi, bias):
+    ql = [300, 17, 256, 129]
+    kl = [200, 64, 256, 1]
+    extra = {} if phi == PHI_SOFTMAX else dict(scale=1.0, kv_std=1.0 / np.sqrt(128))
+    w = make_workload(5, seed=80 + phi + bias, q_lens=ql, kv_lens=kl, phi=phi, bias=bias,
+                      with_dout=False, **extra)
+    check(cuda_lib, w, seed=5, same_sequence=False)
+
+
+@pytest.mark.parametrize("kv_len", [64, 256, 700])  # 64-key blocks; resident ring; streamed
+def test_resident_and_streamed_keys(cuda_lib, kv_len):
+    """A unit whose key blocks stay in the ring for all its query tiles turns
+    them once; streamed blocks are turned at every load."""
+    ql = [600, 130, 5]
+    kl = [kv_len, kv_len, kv_len]
+    w = make_workload(3, seed=90, q_lens=ql, kv_lens=kl, H=2, D=128)
+    check(cuda_lib, w, seed=11, same_sequence=False)
+
+
+def test_zero_frequencies_give_the_plain_forward(cuda_lib):
+    """theta = phi = 0: every angle is 0, the turn is exact, and the result is
+    bit-identical to the forward without rotation."""
+    ql = [50, 300]
+    w = make_workload(4, seed=12, q_lens=ql, kv_lens=ql, window=(127, 0))
+    z = np.zeros(64, np.float32)
+    tq = gpu_table(cuda_lib, w.q_offsets, event_times(ql, 4), 128, theta=z, phi=z)
+    o, lse = run(cuda_lib, w, tq, tq)
+    qo, ko = _dev(w.q_offsets, torch.int32), _dev(w.kv_offsets, torch.int32)
+    o2, lse2, _ = cuda_lib.forward(w.q.cuda(), w.k.cuda(), w.v.cuda(), qo, ko, phi=w.phi,
+                                   scale=w.scale, window=(127, 0), max_seqlen_q=w.max_q,
+                                   max_seqlen_kv=w.max_kv)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
+def test_empty_samples(cuda_lib):
+    ql = [0, 3, 0, 140]
+    kl = [5, 0, 0, 140]
+    w = make_workload(4, seed=13, q_lens=ql, kv_lens=kl, window=(-1, -1))
+    check(cuda_lib, w, seed=13, same_sequence=False)

@@ -196,3 +196,30 @@ def subset(w: Workload, samples) -> Workload:
     if w.dout is not None:
         out.dout = cat(w.dout, qsl)
     return out
+
+
+# Event times for the rotary temporal embedding: behaviour logs hold events
+# from seconds to months apart, often several in the same second.  Per sample:
+# a start time in 2024 (Unix seconds), then gaps that are 0 with probability
+# 0.1 and otherwise log-uniform between 1 s and 10^7 s (about four months),
+# rounded to whole seconds.  int64 [total], non-decreasing within a sample.
+EVENT_TIME_SCALE = 3600.0  # tau_scale of the rotary workloads: one hour
+
+
+def event_times(lens, seed: int) -> np.ndarray:
+    lens = np.asarray(lens, np.int64)
+    rng = np.random.default_rng(seed)
+    total = int(lens.sum())
+    gaps = np.rint(np.exp(rng.uniform(0.0, math.log(1e7), total))).astype(np.int64)
+    gaps[rng.uniform(size=total) < 0.1] = 0
+    starts = rng.integers(1_704_067_200, 1_735_689_600, len(lens))
+    out = np.empty(total, np.int64)
+    pos = 0
+    for b, L in enumerate(lens):
+        L = int(L)
+        if L:
+            g = gaps[pos:pos + L].copy()
+            g[0] = 0
+            out[pos:pos + L] = starts[b] + np.cumsum(g)
+        pos += L
+    return out
