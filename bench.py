@@ -573,6 +573,58 @@ def run_grouped(args):
             "achieved_gbs": round(byts / (g_ms * 1e-3) / 1e9, 1)}
 
 
+def run_rotary(args):
+    """Forward of the sliding-window self-attention workload with the rotary
+    temporal embedding (Q and K turned in shared memory) against the same
+    forward without it; the table build is timed on its own."""
+    import torch
+
+    from pffn_attention_b200 import gdpa
+    from workloads import EVENT_TIME_SCALE, event_times
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = make_workload(4, device=dev, with_dout=False)
+    stream = torch.cuda.Stream(device=dev)
+    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+    times = torch.tensor(event_times(w.q_lens, 4), dtype=torch.int64, device=dev)
+    kw = dict(phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+              max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv, stream=stream)
+    table = gdpa.rotary_table(qo, times, w.D, EVENT_TIME_SCALE, stream=stream)
+    o, lse, ws = gdpa.forward(w.q, w.k, w.v, qo, qo, rope=(table, table), **kw)
+    o2, lse2, ws2 = gdpa.forward(w.q, w.k, w.v, qo, qo, **kw)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    r_ms = timed(lambda: gdpa.forward(w.q, w.k, w.v, qo, qo, rope=(table, table), out=o, lse=lse,
+                                      workspace=ws, **kw))
+    p_ms = timed(lambda: gdpa.forward(w.q, w.k, w.v, qo, qo, out=o2, lse=lse2, workspace=ws2,
+                                      **kw))
+    t_ms = timed(lambda: gdpa.rotary_table(qo, times, w.D, EVENT_TIME_SCALE, out=table,
+                                           stream=stream))
+    assert gdpa.device_status(ws, stream) == 0
+    flops = useful_flops(w, False)[0]
+    byts = algorithmic_bytes(w, False)[0] + table.numel() * 4  # + one read of the table
+    return {"metric": "GDPA forward with rotary temporal embedding, sliding-window "
+                      "self-attention (useful TFLOP/s)",
+            "value": round(flops / (r_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r_ms, 4),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D,
+                       "window": [w.window_left, w.window_right], "l2": "inputs > L2"},
+            "plain_forward_ms": round(p_ms, 4), "rotary_overhead": round(r_ms / p_ms, 3),
+            "table_ms": round(t_ms, 4), "achieved_gbs": round(byts / (r_ms * 1e-3) / 1e9, 1)}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -589,6 +641,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grouped", action="store_true",
                     help="time the event-type problems as one grouped call vs separate calls")
+    ap.add_argument("--rotary", action="store_true",
+                    help="time the sliding-window forward with the rotary temporal embedding")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -600,6 +654,11 @@ def main(argv=None):
         if world != 1 or args.impl != "ours":
             ap.error("--grouped runs on one GPU, our implementation")
         print(json.dumps(run_grouped(args)), flush=True)
+        return 0
+    if args.rotary:
+        if world != 1 or args.impl != "ours":
+            ap.error("--rotary runs on one GPU, our implementation")
+        print(json.dumps(run_rotary(args)), flush=True)
         return 0
 
     if args.impl == "reference":

@@ -90,7 +90,8 @@ typedef struct {
   int bias_kind;      /* GDPA_BIAS_*: none, beta = bias, or beta = log sigmoid(bias) */
   int debug_flags;    /* 0 in normal use.  Bit 0 drops one producer arrival so that
                          the bounded-wait path can be tested (returns TIMEOUT);
-                         other bits are reserved and ignored */
+                         bit 2 selects the in-kernel rotary turn (forward; see
+                         rope_q); other bits are reserved and ignored */
   int wait_timeout_us;/* bound on any single in-kernel wait; 0 = 2000000 (2 s) */
   const int32_t* head_phi; /* optional host array of H GDPA_PHI_* values, one per
                          head (H <= 64); NULL = every head uses phi.  Read during
@@ -99,10 +100,15 @@ typedef struct {
   /* Rotary temporal embedding of Q and K (gdpa_rotary_table below): device
    * tables of rotations, [total_q][D/2] for the queries and [total_kv][D/2] for
    * the keys, 16-byte aligned; both NULL = no rotation.  Give both or neither
-   * (self-attention passes the same table twice).  The forward turns each Q
-   * tile and K block as it arrives in shared memory, before QK^T; V is not
-   * rotated.  Not accepted by gdpa_backward or the grouped forward yet
-   * (GDPA_ERR_UNSUPPORTED). */
+   * (self-attention passes the same table twice).  The attention then uses
+   * turned Q and K (V is not turned); the backward returns dQ and dK with
+   * respect to the unturned inputs.  Both calls turn Q and K in one streaming
+   * pass into the workspace (which grows by (total_q + total_kv) * H * D * 2
+   * bytes) and run the attention kernels on the copies; the backward turns dQ
+   * and dK back in place at the end.  debug_flags bit 2 makes the forward turn
+   * each Q tile and K block in shared memory inside the attention kernel
+   * instead (no copies; measured slower).  Not accepted by the grouped
+   * forward (GDPA_ERR_UNSUPPORTED). */
   const void* rope_q;
   const void* rope_kv;
 } gdpa_params_t;
@@ -132,13 +138,23 @@ GDPA_API size_t gdpa_rotary_table_bytes(int D, int64_t total);
 /* Fills table [total][D/2] (device, 16-byte aligned, the caller's) for the
  * jagged sequence given by offsets [B+1] (device int32, as elsewhere) and
  * time [total] (device int64 event times, non-decreasing within a sample for
- * the gaps to mean anything).  The angle is formed and reduced modulo 2 pi in
- * fp64, then its cosine and sine are taken in fp32 and rounded to fp16.  One
+ * the gaps to mean anything).  The position part t * theta_i is reduced
+ * modulo 2 pi without rounding error (positions below 2^24; the default
+ * frequencies are taken in fp64), then the cosine and sine are taken in fp32
+ * and rounded to fp16.  One
  * table serves every head, the forward and the backward, and every layer that
  * sees the same sequence.  Asynchronous on stream. */
 GDPA_API gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, int64_t total,
                                          const int32_t* offsets, const int64_t* time,
                                          void* table, gdpa_stream_t stream);
+
+/* y = x turned by the table's angles (inverse = 0) or turned back (inverse
+ * != 0: the transpose, which maps dL/dx' to dL/dx), for x, y bf16
+ * [total][H][D] (device, 16-byte aligned; y may be x) and a table from
+ * gdpa_rotary_table for the same tokens.  Asynchronous on stream. */
+GDPA_API gdpa_status_t gdpa_rotary_apply(int64_t total, int H, int D, const void* x,
+                                         const void* table, void* y, int inverse,
+                                         gdpa_stream_t stream);
 
 /* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward
  * (backward = 1) needs for these parameters.  0 on invalid parameters. */

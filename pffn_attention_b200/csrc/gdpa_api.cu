@@ -122,8 +122,29 @@ WorkspaceLayout make_layout(const gdpa_params_t* p, int backward, int sms) {
     L.dq_scratch = off;
     off += align256((size_t)L.grid * (size_t)L.dq_slot_rows * (size_t)p->D * 4);
   }
+  // rotary: the turned Q and K the attention kernels read (the backward's
+  // input turn, and the forward's unless it turns them in the kernel)
+  if (p->rope_q && (backward || rotary_streamed(p->rope_q, p->debug_flags))) {
+    L.rope_q = off;
+    off += align256((size_t)p->total_q * (size_t)p->H * (size_t)p->D * 2);
+    L.rope_k = off;
+    off += align256((size_t)p->total_kv * (size_t)p->H * (size_t)p->D * 2);
+  }
   L.total = off;
   return L;
+}
+
+// One streaming launch: Q and K turned by their tables into rq, rk (inverse:
+// turned back), bf16 [total][H][D].
+cudaError_t turn_qk(const gdpa_params_t* p, const void* q, const void* k, void* rq, void* rk,
+                    int inverse, int sms, cudaStream_t s) {
+  RotaryApplyArgs r{};
+  r.H = p->H;
+  r.D = p->D;
+  r.inverse = inverse;
+  r.job[0] = RotaryJob{q, rq, static_cast<const uint32_t*>(p->rope_q), p->total_q};
+  r.job[1] = RotaryJob{k, rk, static_cast<const uint32_t*>(p->rope_kv), p->total_kv};
+  return launch_rotary_apply(r, sms, s);
 }
 
 // [rows][H][D] bf16 tensor, boxes of box_rows rows x one head x panel columns.
@@ -329,6 +350,15 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
   if (p->B == 0 || p->total_q == 0) return GDPA_OK;
 
+  const bool streamed = rotary_streamed(p->rope_q, p->debug_flags);
+  if (streamed) {  // the kernel reads turned copies of Q and K
+    void* rq = ws + L.rope_q;
+    void* rk = ws + L.rope_k;
+    e = turn_qk(p, q, k, rq, rk, 0, sms, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+    q = rq;
+    k = rk;
+  }
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
   if (p->total_kv > 0) {
@@ -354,8 +384,10 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   a.p0.wl = p->window_left;
   a.p0.wr = p->window_right;
   a.p0.scale = p->scale;
-  a.rope_q = static_cast<const uint32_t*>(p->rope_q);
-  a.rope_kv = static_cast<const uint32_t*>(p->rope_kv);
+  if (p->rope_q && !streamed) {  // turned inside the attention kernel
+    a.rope_q = static_cast<const uint32_t*>(p->rope_q);
+    a.rope_kv = static_cast<const uint32_t*>(p->rope_kv);
+  }
   // one launch per activation present (a per-head activation vector groups
   // the heads; each launch walks only its own heads' units)
   for (int phi = 0; phi <= 3; ++phi) {
@@ -379,7 +411,6 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
                             void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
   gdpa_status_t st = check_params(p);
   if (st != GDPA_OK) return st;
-  if (p->rope_q) return GDPA_ERR_UNSUPPORTED;  // rotary backward: not built yet
   if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
   // a bias gradient needs a bias; it is fp32 [H][total_kv]
   if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
@@ -417,6 +448,14 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   if (p->B == 0 || (p->total_q == 0 && p->total_kv == 0)) return GDPA_OK;
+  if (p->rope_q) {  // the attention gradient is taken at the turned Q and K
+    void* rq = ws + L.rope_q;
+    void* rk = ws + L.rope_k;
+    e = turn_qk(p, q, k, rq, rk, 0, sms, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+    q = rq;
+    k = rk;
+  }
   if (softmax && p->total_q > 0) {
     e = launch_bwd_preprocess(static_cast<const __nv_bfloat16*>(o),
                               static_cast<const __nv_bfloat16*>(dout), delta, p->total_q, p->H,
@@ -475,6 +514,10 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
     a.phi = phi;
     a.head_mask = heads;
     e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
+    if (e != cudaSuccess) return GDPA_ERR_CUDA;
+  }
+  if (p->rope_q) {  // dQ = R^T dQ', dK = R^T dK' (the turn is orthogonal), in place
+    e = turn_qk(p, dq, dk, dq, dk, 1, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;
@@ -622,15 +665,36 @@ gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, int64_t to
   a.B = B;
   a.total = total;
   a.time_scale = r->time_scale;
+  const double pi = 3.141592653589793;
   for (int i = 0; i < r->D / 2; ++i) {
-    const float th = r->theta ? r->theta[i] : (float)std::pow(10000.0, -2.0 * i / r->D);
-    const float ph = r->phi ? r->phi[i] : th;
+    // the default frequencies in fp64; given ones exactly as the caller's floats
+    const double th = r->theta ? (double)r->theta[i] : std::pow(10000.0, -2.0 * i / r->D);
+    const double ph = r->phi ? (double)r->phi[i] : th;
     if (!std::isfinite(th) || !std::isfinite(ph)) return GDPA_ERR_INVALID_ARG;
-    a.theta[i] = th;
-    a.phi[i] = ph;
+    a.theta_hi[i] = (float)(th / pi);
+    a.theta_lo[i] = (float)(th / pi - (double)a.theta_hi[i]);
+    a.phi_pi[i] = (float)(ph / pi);
   }
   cudaError_t e = launch_rotary_table(a, offsets, time, static_cast<uint32_t*>(table),
                                       (cudaStream_t)stream);
+  return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}
+
+gdpa_status_t gdpa_rotary_apply(int64_t total, int H, int D, const void* x, const void* table,
+                                void* y, int inverse, gdpa_stream_t stream) {
+  if (D != 32 && D != 64 && D != 128) return GDPA_ERR_UNSUPPORTED;
+  if (total < 0 || total >= (int64_t(1) << 31) || H <= 0) return GDPA_ERR_INVALID_ARG;
+  if (total == 0) return GDPA_OK;
+  if (!x || !table || !y || !aligned16(x) || !aligned16(table) || !aligned16(y))
+    return GDPA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  RotaryApplyArgs r{};
+  r.H = H;
+  r.D = D;
+  r.inverse = inverse ? 1 : 0;
+  r.job[0] = RotaryJob{x, y, static_cast<const uint32_t*>(table), total};
+  cudaError_t e = launch_rotary_apply(r, sms, (cudaStream_t)stream);
   return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 

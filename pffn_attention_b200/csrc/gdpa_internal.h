@@ -19,8 +19,9 @@ constexpr int kMaxSortBatch = 16384;  // batch limit of the single-CTA LPT sort
 //   then                      info[B]       int4    {q0, Lq, k0, Lk} of order[p]
 //   backward only, then       delta[H][total_q] fp32 (softmax rowsum(dO * O))
 //   backward only, then       dQ scratch: grid x slot_rows x D fp32
+//   rotary (streamed), then   turned Q [total_q][H][D], turned K [total_kv][H][D] bf16
 struct WorkspaceLayout {
-  size_t order, tile_start, info, delta, dq_scratch, total;
+  size_t order, tile_start, info, delta, dq_scratch, rope_q, rope_k, total;
   int dq_slot_rows;
   int grid;
 };
@@ -116,15 +117,36 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
                             int32_t* order, int4* info, int max_q, int max_kv,
                             DeviceStatus* status, cudaStream_t stream);
+// debug_flags bit 2: the forward turns Q and K inside the attention kernel
+// (warps 2-3, in shared memory) instead of in a streaming pass first.
+constexpr int kDebugFusedRotary = 4;
+inline bool rotary_streamed(const void* rope_q, int debug_flags) {
+  return rope_q != nullptr && !(debug_flags & kDebugFusedRotary);
+}
+
 // Rotary temporal embedding table: angles t theta_i + tau_t phi_i per token.
 struct RotaryArgs {
-  float theta[64], phi[64];
+  // theta_i / pi as hi + lo, and phi_i / pi: angles in half-turns
+  float theta_hi[64], theta_lo[64], phi_pi[64];
   double time_scale;
   int D, B;
   int64_t total;
 };
 cudaError_t launch_rotary_table(const RotaryArgs& r, const int32_t* offsets,
                                 const int64_t* time, uint32_t* table, cudaStream_t stream);
+// y = x turned by the table's angles (or back, when inverse), bf16 [total][H][D].
+struct RotaryJob {
+  const void* x;
+  void* y;
+  const uint32_t* table;
+  int64_t total;
+};
+struct RotaryApplyArgs {
+  RotaryJob job[2];  // an unused job has total 0
+  int H, D;
+  int inverse;
+};
+cudaError_t launch_rotary_apply(const RotaryApplyArgs& a, int sms, cudaStream_t stream);
 
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);

@@ -26,7 +26,8 @@ BIAS = {"none": 0, "add": 1, "gate": 2}
 EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_schedule",
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
             "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
-            "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table")
+            "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table",
+            "gdpa_rotary_apply")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -102,6 +103,9 @@ def load(path: str = LIB_PATH):
     lib.gdpa_rotary_table.argtypes = [ctypes.POINTER(gdpa_rotary_params_t), ctypes.c_int,
                                       ctypes.c_int64, vp, vp, vp, st]
     lib.gdpa_rotary_table.restype = ctypes.c_int
+    lib.gdpa_rotary_apply.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                      ctypes.c_int, st]
+    lib.gdpa_rotary_apply.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -124,6 +128,11 @@ def gdpa_rotary_table_bytes(D: int, total: int) -> int:
 def gdpa_rotary_table(r: gdpa_rotary_params_t, B, total, offsets, time, table, stream) -> int:
     return load().gdpa_rotary_table(ctypes.byref(r), int(B), int(total), offsets, time, table,
                                     stream)
+
+
+def gdpa_rotary_apply(total, H, D, x, table, y, inverse, stream) -> int:
+    return int(load().gdpa_rotary_apply(int(total), int(H), int(D), x, table, y, int(inverse),
+                                        stream))
 
 
 def gdpa_forward_grouped_workspace_size(problems) -> int:
@@ -252,6 +261,17 @@ def rotary_table(offsets, time, D, time_scale, *, theta=None, phi=None, out=None
     return out
 
 
+def rotary_apply(x, table, *, inverse=False, out=None, stream=None):
+    """x [total,H,D] bf16 turned by the table (or back); out may be x."""
+    import torch
+    total, H, D = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check(gdpa_rotary_apply(total, H, D, _ptr(x), _ptr(table), _ptr(out), int(inverse),
+                             _stream(stream)), "gdpa_rotary_apply")
+    return out
+
+
 def forward(q, k, v, q_offsets, kv_offsets, *, phi="silu", scale=1.0, window=(-1, -1),
             bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0, out=None, lse=None,
             workspace=None, stream=None, params=None, head_phi=None, rope=None):
@@ -317,16 +337,17 @@ def forward_grouped(problems, *, workspace=None, stream=None):
 def backward(q, k, v, o, dout, lse, q_offsets, kv_offsets, *, phi="silu", scale=1.0,
              window=(-1, -1), bias=None, bias_kind="none", max_seqlen_q=0, max_seqlen_kv=0,
              dq=None, dk=None, dv=None, dbias=None, workspace=None, stream=None, params=None,
-             head_phi=None):
+             head_phi=None, rope=None):
     """dQ, dK, dV on the device (bf16, shapes of q, k, v).  With a bias or gate,
-    pass dbias (fp32 [H, total_kv]) to also receive the bias gradient."""
+    pass dbias (fp32 [H, total_kv]) to also receive the bias gradient.  rope:
+    the forward's (q table, kv table); q and k stay the unturned inputs."""
     import torch
     total_q, H, D = q.shape
     total_kv = k.shape[0]
     B = q_offsets.numel() - 1
     p = params or make_params(B, H, D, total_q, total_kv, phi=phi, scale=scale, window=window,
                               bias_kind=bias_kind, max_seqlen_q=max_seqlen_q,
-                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi)
+                              max_seqlen_kv=max_seqlen_kv, head_phi=head_phi, rope=rope)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

@@ -134,8 +134,8 @@ def test_grouped_forward_validation(lib):
 
 def test_rotary_validation(lib):
     """Rotary tables: D, time scale, jagged sizes and alignment are checked on
-    the host; the tables must come as a pair; the backward and grouped forward
-    refuse them (not built)."""
+    the host; the tables must come as a pair; the grouped forward refuses them
+    (not built); the streamed turn adds the turned copies to the workspace."""
     def rp(D=64, scale=60.0):
         return gdpa.gdpa_rotary_params_t(D, scale, None, None)
     assert gdpa.gdpa_rotary_table_bytes(64, 10) == 10 * 32 * 4
@@ -157,8 +157,17 @@ def test_rotary_validation(lib):
     assert gdpa.gdpa_workspace_size(p, 0) == 0  # unaligned
     p.rope_kv = FAKE
     assert gdpa.gdpa_workspace_size(p, 0) > 0
-    args = (FAKE,) * 8 + (None,) + (FAKE,) * 3 + (None, FAKE)  # no bias, no bias gradient
-    assert gdpa.gdpa_backward(p, *args, 1 << 20, None) == 2
+    # the turned copies of Q and K live in the workspace
+    # (total_q = 10, total_kv = 8, H = 2, D = 64: 2560 + 2048 bytes, both 256-aligned)
+    for backward in (0, 1):
+        plain = gdpa.gdpa_workspace_size(_params(), backward)
+        assert gdpa.gdpa_workspace_size(p, backward) == plain + 2560 + 2048
+    p.debug_flags = 4  # turned inside the forward kernel: no copies
+    assert gdpa.gdpa_workspace_size(p, 0) == gdpa.gdpa_workspace_size(_params(), 0)
+    assert gdpa.gdpa_rotary_apply(10, 2, 48, FAKE, FAKE, FAKE, 0, None) == 2
+    assert gdpa.gdpa_rotary_apply(10, 0, 64, FAKE, FAKE, FAKE, 0, None) == 1
+    assert gdpa.gdpa_rotary_apply(10, 2, 64, FAKE + 2, FAKE, FAKE, 0, None) == 1
+    assert gdpa.gdpa_rotary_apply(0, 2, 64, None, None, None, 0, None) == 0
     a = (gdpa.gdpa_forward_problem_t * 1)()
     a[0].params = p
     for name in ("q", "k", "v", "q_offsets", "kv_offsets", "o"):

@@ -86,28 +86,41 @@ def check_lse(lse, rlse, w, aq, ak):
         f"{(err - bound).max():.3e})"
 
 
-def run(gdpa, w, tq, tk, **kw):
+FUSED = 4  # debug_flags bit 2: turn Q and K inside the attention kernel
+
+
+def params(gdpa, w, tq, tk, debug_flags=0):
+    return gdpa.make_params(w.B, w.H, w.D, int(w.q_offsets[-1]), int(w.kv_offsets[-1]),
+                            phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+                            bias_kind=w.bias_kind, max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv,
+                            debug_flags=debug_flags, rope=(tq, tk))
+
+
+def run(gdpa, w, tq, tk, mode="streamed"):
     qo, ko = _dev(w.q_offsets, torch.int32), _dev(w.kv_offsets, torch.int32)
     bias = w.bias.cuda() if w.bias is not None else None
-    o, lse, ws = gdpa.forward(w.q.cuda(), w.k.cuda(), w.v.cuda(), qo, ko, phi=w.phi,
-                              scale=w.scale, window=(w.window_left, w.window_right), bias=bias,
-                              bias_kind=w.bias_kind, max_seqlen_q=w.max_q,
-                              max_seqlen_kv=w.max_kv, rope=(tq, tk), **kw)
+    p = params(gdpa, w, tq, tk, FUSED if mode == "fused" else 0)
+    o, lse, ws = gdpa.forward(w.q.cuda(), w.k.cuda(), w.v.cuda(), qo, ko, bias=bias, params=p)
     assert gdpa.device_status(ws) == 0
     torch.cuda.synchronize()
     return o, lse
 
 
-def check(gdpa, w, seed, same_sequence):
+def tables(gdpa, w, seed, same_sequence):
     """Self-attention (same_sequence) shares one table; otherwise queries and
-    keys have their own times."""
+    keys have their own times.  Returns the device tables and oracle angles."""
     tq_np = event_times(w.q_lens, seed)
     tk_np = tq_np if same_sequence else event_times(w.kv_lens, seed + 1)
     tq = gpu_table(gdpa, w.q_offsets, tq_np, w.D)
     tk = tq if same_sequence else gpu_table(gdpa, w.kv_offsets, tk_np, w.D)
-    o, lse = run(gdpa, w, tq, tk)
     aq = rotary.angles(w.q_offsets, tq_np, w.D, EVENT_TIME_SCALE)
     ak = rotary.angles(w.kv_offsets, tk_np, w.D, EVENT_TIME_SCALE)
+    return tq, tk, aq, ak
+
+
+def check(gdpa, w, seed, same_sequence, mode="streamed"):
+    tq, tk, aq, ak = tables(gdpa, w, seed, same_sequence)
+    o, lse = run(gdpa, w, tq, tk, mode)
     ro, rlse = rotary.forward(w.q, w.k, w.v, w.q_offsets, w.kv_offsets, aq, ak, phi=w.phi,
                               scale=w.scale, window=(w.window_left, w.window_right),
                               bias=w.bias, bias_kind=w.bias_kind)
@@ -119,34 +132,117 @@ def check(gdpa, w, seed, same_sequence):
 
 # sliding-window self-attention is where the pages use temporal rotary; the
 # band keeps every key block streamed through the ring
+MODES = ["streamed", "fused"]
+
+
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("D", [32, 64, 128])
 @pytest.mark.parametrize("window", [(127, 0), (40, 40), (-1, -1)])
-def test_self_attention(cuda_lib, D, window):
+def test_self_attention(cuda_lib, D, window, mode):
     ql = [1, 60, 200, 333, 520, 129]
     w = make_workload(4, seed=70 + D, q_lens=ql, kv_lens=ql, D=D, window=window,
                       scale=1.0 / np.sqrt(D))
-    check(cuda_lib, w, seed=D, same_sequence=True)
+    check(cuda_lib, w, seed=D, same_sequence=True, mode=mode)
 
 
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("phi", [PHI_SILU, PHI_GELU, PHI_SOFTMAX])
 @pytest.mark.parametrize("bias", [BIAS_NONE, BIAS_GATE])
-def test_activations_and_gate(cuda_lib, phi, bias):
+def test_activations_and_gate(cuda_lib, phi, bias, mode):
     ql = [300, 17, 256, 129]
     kl = [200, 64, 256, 1]
     extra = {} if phi == PHI_SOFTMAX else dict(scale=1.0, kv_std=1.0 / np.sqrt(128))
     w = make_workload(5, seed=80 + phi + bias, q_lens=ql, kv_lens=kl, phi=phi, bias=bias,
                       with_dout=False, **extra)
-    check(cuda_lib, w, seed=5, same_sequence=False)
+    check(cuda_lib, w, seed=5, same_sequence=False, mode=mode)
 
 
 @pytest.mark.parametrize("kv_len", [64, 256, 700])  # 64-key blocks; resident ring; streamed
 def test_resident_and_streamed_keys(cuda_lib, kv_len):
-    """A unit whose key blocks stay in the ring for all its query tiles turns
-    them once; streamed blocks are turned at every load."""
+    """In the kernel, a unit whose key blocks stay in the ring for all its query
+    tiles turns them once; streamed blocks are turned at every load."""
     ql = [600, 130, 5]
     kl = [kv_len, kv_len, kv_len]
     w = make_workload(3, seed=90, q_lens=ql, kv_lens=kl, H=2, D=128)
-    check(cuda_lib, w, seed=11, same_sequence=False)
+    check(cuda_lib, w, seed=11, same_sequence=False, mode="fused")
+
+
+def test_streamed_and_fused_agree(cuda_lib):
+    """Both turn the same bf16 inputs with the same table and round the turned
+    values to bf16 the same way, so the attention sees identical operands."""
+    ql = [200, 513, 64]
+    w = make_workload(4, seed=14, q_lens=ql, kv_lens=ql)
+    tq, tk, _, _ = tables(cuda_lib, w, 14, True)
+    o1, l1 = run(cuda_lib, w, tq, tk, "streamed")
+    o2, l2 = run(cuda_lib, w, tq, tk, "fused")
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_apply_and_inverse(cuda_lib, D):
+    lens = [3, 400, 129]
+    w = make_workload(4, seed=15 + D, q_lens=lens, kv_lens=lens, H=3, D=D)
+    tq, _, aq, _ = tables(cuda_lib, w, 15, True)
+    x = w.q.cuda()
+    y = cuda_lib.rotary_apply(x, tq)
+    compare("turned", y, rotary.rotate(w.q.double().numpy(), aq))
+    back = cuda_lib.rotary_apply(y, tq, inverse=True)
+    compare("turned back", back, w.q.double().numpy())
+    z = x.clone()
+    cuda_lib.rotary_apply(z, tq, out=z)  # in place
+    torch.cuda.synchronize()
+    assert torch.equal(z, y)
+
+
+# -------------------------------------------------- backward
+def gpu_backward(gdpa, w, tq, tk):
+    dev = torch.device("cuda")
+    qo, ko = _dev(w.q_offsets, torch.int32), _dev(w.kv_offsets, torch.int32)
+    bias = w.bias.cuda() if w.bias is not None else None
+    p = params(gdpa, w, tq, tk)
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    o, lse, _ = gdpa.forward(q, k, v, qo, ko, bias=bias, params=p)
+    dbias = (torch.empty((w.H, int(w.kv_offsets[-1])), dtype=torch.float32, device=dev)
+             if bias is not None else None)
+    dq, dk, dv, ws = gdpa.backward(q, k, v, o, w.dout.cuda(), lse, qo, ko, bias=bias,
+                                   dbias=dbias, params=p)
+    assert gdpa.device_status(ws) == 0
+    torch.cuda.synchronize()
+    return dq, dk, dv, dbias
+
+
+@pytest.mark.parametrize("phi", [PHI_SOFTMAX, PHI_SILU])
+@pytest.mark.parametrize("window", [(127, 0), (-1, -1)])
+def test_backward_self_attention(cuda_lib, phi, window):
+    ql = [1, 60, 200, 333, 129]
+    extra = dict(dout_std=0.125) if phi == PHI_SOFTMAX else dict(
+        scale=1.0, kv_std=1.0 / np.sqrt(128), dout_std=0.125)
+    w = make_workload(4, seed=16, q_lens=ql, kv_lens=ql, phi=phi, window=window, with_dout=True,
+                      **extra)
+    tq, tk, aq, ak = tables(cuda_lib, w, 16, True)
+    dq, dk, dv, _ = gpu_backward(cuda_lib, w, tq, tk)
+    rdq, rdk, rdv, _ = rotary.backward(w.q, w.k, w.v, w.dout, w.q_offsets, w.kv_offsets, aq, ak,
+                                       phi=w.phi, scale=w.scale,
+                                       window=(w.window_left, w.window_right))
+    compare("dQ", dq, rdq)
+    compare("dK", dk, rdk)
+    compare("dV", dv, rdv)
+
+
+def test_backward_gate_cross_sequences(cuda_lib):
+    ql = [300, 17, 256]
+    kl = [200, 64, 256]
+    w = make_workload(5, seed=17, q_lens=ql, kv_lens=kl, bias=BIAS_GATE, with_dout=True,
+                      dout_std=0.125)
+    tq, tk, aq, ak = tables(cuda_lib, w, 17, False)
+    dq, dk, dv, dg = gpu_backward(cuda_lib, w, tq, tk)
+    rdq, rdk, rdv, rdg = rotary.backward(w.q, w.k, w.v, w.dout, w.q_offsets, w.kv_offsets, aq,
+                                         ak, phi=w.phi, scale=w.scale, bias=w.bias,
+                                         bias_kind=w.bias_kind)
+    compare("dQ", dq, rdq)
+    compare("dK", dk, rdk)
+    compare("dV", dv, rdv)
+    compare("dG", dg, rdg, max_abs=3e-2 * max(1.0, float(np.abs(rdg).max())), bf16_out=False)
 
 
 def test_zero_frequencies_give_the_plain_forward(cuda_lib):
