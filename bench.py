@@ -625,6 +625,48 @@ def run_rotary(args):
             "table_ms": round(t_ms, 4), "achieved_gbs": round(byts / (r_ms * 1e-3) / 1e9, 1)}
 
 
+def run_sumkron(args):
+    """SumKronLinear forward on the page's typical configuration (seed
+    summaries of the seed-pooling batch): useful FLOPs of the cheaper
+    association, 2 k T S D + 2 k T D^2 per sample."""
+    import torch
+
+    from pffn_attention_b200 import gdpa
+    from workloads import SUMKRON_CONFIG, make_sumkron
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    c = SUMKRON_CONFIG
+    B, S, T, D, k = c["B"], c["S"], c["T"], c["D"], c["k"]
+    x, a, w = make_sumkron(B, S, T, D, k, seed=1, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    y, ws = gdpa.sumkron_forward(x, a, w, stream=stream)
+    for _ in range(args.warmup):
+        gdpa.sumkron_forward(x, a, w, out=y, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        gdpa.sumkron_forward(x, a, w, out=y, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert gdpa.device_status(ws, stream) == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = B * (2.0 * k * T * S * D + 2.0 * k * T * D * D)
+    byts = 2.0 * (x.numel() + y.numel() + a.numel() + w.numel())
+    peaks, src = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"metric": "SumKronLinear forward, HSP second stage (useful TFLOP/s)",
+            "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "sumkron_hsp", **c, "l2": "inputs > L2"},
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                         "peak_source": src},
+            "achieved_gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -643,6 +685,8 @@ def main(argv=None):
                     help="time the event-type problems as one grouped call vs separate calls")
     ap.add_argument("--rotary", action="store_true",
                     help="time the sliding-window forward with the rotary temporal embedding")
+    ap.add_argument("--sumkron", action="store_true",
+                    help="time the fused SumKronLinear forward (HSP second stage)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -654,6 +698,11 @@ def main(argv=None):
         if world != 1 or args.impl != "ours":
             ap.error("--grouped runs on one GPU, our implementation")
         print(json.dumps(run_grouped(args)), flush=True)
+        return 0
+    if args.sumkron:
+        if world != 1 or args.impl != "ours":
+            ap.error("--sumkron runs on one GPU, our implementation")
+        print(json.dumps(run_sumkron(args)), flush=True)
         return 0
     if args.rotary:
         if world != 1 or args.impl != "ours":

@@ -156,6 +156,35 @@ GDPA_API gdpa_status_t gdpa_rotary_apply(int64_t total, int H, int D, const void
                                          const void* table, void* y, int inverse,
                                          gdpa_stream_t stream);
 
+/* ---- SumKronLinear (Kunlun paper review §2.4: the second stage of
+ * Hierarchical Seed Pooling compresses the seed summaries X [B, S, D] to
+ * Y [B, T, D] with a rank-k sum of Kronecker products, k (S T + D^2)
+ * parameters; the page's formula was lost, this is the reading used):
+ *   vec(Y_b) = sum_r (A_r kron W_r^T) vec(X_b),  i.e.  Y_b = sum_r A_r X_b W_r,
+ * A_r [T x S], W_r [D x D], no bias.  One fused kernel: Z_b = A X_b on the
+ * tensor cores, rounded to bf16 on chip, then Y_b = sum_r Z_b[r] W_r with fp32
+ * accumulation; Z never reaches HBM. */
+typedef struct {
+  int B;               /* samples */
+  int S;               /* seeds per sample: 64, 128, 192 or 256 */
+  int T;               /* output tokens per sample: 32 or 64 */
+  int D;               /* embedding dim: 128, 256 or 384 */
+  int k;               /* Kronecker rank: k * T a multiple of 128 */
+  int wait_timeout_us; /* bound on any single in-kernel wait; 0 = 2 s */
+} gdpa_sumkron_params_t;
+
+/* Workspace bytes (the device status block); 0 on invalid parameters. */
+GDPA_API size_t gdpa_sumkron_workspace_size(const gdpa_sumkron_params_t* p);
+
+/* y [B][T][D] from x [B][S][D], a [k][T][S] (A_1..A_k) and w [k][D][D]
+ * (W_1..W_k), all bf16 row-major device arrays, 16-byte aligned, the
+ * caller's.  The workspace's status is cleared on the stream first; read it
+ * with gdpa_get_device_status.  Asynchronous on stream. */
+GDPA_API gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, const void* x,
+                                            const void* a, const void* w, void* y,
+                                            void* workspace, size_t workspace_bytes,
+                                            gdpa_stream_t stream);
+
 /* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward
  * (backward = 1) needs for these parameters.  0 on invalid parameters. */
 GDPA_API size_t gdpa_workspace_size(const gdpa_params_t* p, int backward);

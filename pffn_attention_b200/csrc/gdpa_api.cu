@@ -164,6 +164,33 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H, int D, int 
   return r == CUDA_SUCCESS;
 }
 
+// Row-major bf16 tensor of up to three dims (innermost first), 128-byte
+// swizzled boxes whose inner extent is 64 elements.
+bool make_map_3d(CUtensorMap* m, const void* base, const cuuint64_t (&dims)[3],
+                 const cuuint64_t (&strides)[2], const cuuint32_t (&box)[3]) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                   const_cast<cuuint64_t*>(dims), const_cast<cuuint64_t*>(strides),
+                   const_cast<cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+gdpa_status_t check_sumkron(const gdpa_sumkron_params_t* p) {
+  if (!p) return GDPA_ERR_INVALID_ARG;
+  if (p->B < 0 || p->S <= 0 || p->T <= 0 || p->D <= 0 || p->k <= 0 || p->wait_timeout_us < 0)
+    return GDPA_ERR_INVALID_ARG;
+  if (p->T != 32 && p->T != 64) return GDPA_ERR_UNSUPPORTED;
+  if (p->D != 128 && p->D != 256 && p->D != 384) return GDPA_ERR_UNSUPPORTED;
+  if (p->S % 64 || p->S > 256 || ((int64_t)p->k * p->T) % 128) return GDPA_ERR_UNSUPPORTED;
+  if ((int64_t)p->k * p->D >= (int64_t(1) << 31) || (int64_t)p->B * p->S >= (int64_t(1) << 31))
+    return GDPA_ERR_UNSUPPORTED;
+  return GDPA_OK;
+}
+
 // Everything gdpa_forward checks about one problem before any launch.
 gdpa_status_t check_forward_args(const gdpa_params_t* p, const void* q, const void* k,
                                  const void* v, const int32_t* q_offsets,
@@ -696,6 +723,44 @@ gdpa_status_t gdpa_rotary_apply(int64_t total, int H, int D, const void* x, cons
   r.job[0] = RotaryJob{x, y, static_cast<const uint32_t*>(table), total};
   cudaError_t e = launch_rotary_apply(r, sms, (cudaStream_t)stream);
   return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}
+
+size_t gdpa_sumkron_workspace_size(const gdpa_sumkron_params_t* p) {
+  return check_sumkron(p) == GDPA_OK ? sizeof(DeviceStatus) : 0;
+}
+
+gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, const void* x, const void* a,
+                                   const void* w, void* y, void* workspace,
+                                   size_t workspace_bytes, gdpa_stream_t stream) {
+  gdpa_status_t st = check_sumkron(p);
+  if (st != GDPA_OK) return st;
+  if (p->B > 0 && (!x || !y)) return GDPA_ERR_INVALID_ARG;
+  if (!a || !w || !aligned16(x) || !aligned16(a) || !aligned16(w) || !aligned16(y) ||
+      !aligned16(workspace))
+    return GDPA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < sizeof(DeviceStatus)) return GDPA_ERR_WORKSPACE;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), s) != cudaSuccess) return GDPA_ERR_CUDA;
+  if (p->B == 0) return GDPA_OK;
+  const cuuint64_t S = p->S, D = p->D, kT = (cuuint64_t)p->k * p->T,
+                   kD = (cuuint64_t)p->k * p->D;
+  CUtensorMap ta, tx, tw;
+  if (!make_map_3d(&ta, a, {S, kT, 1}, {S * 2, S * kT * 2}, {64u, 128u, 1u}) ||
+      !make_map_3d(&tx, x, {D, S, (cuuint64_t)p->B}, {D * 2, S * D * 2}, {64u, 64u, 1u}) ||
+      !make_map_3d(&tw, w, {D, kD, 1}, {D * 2, kD * D * 2}, {64u, (cuuint32_t)kSumKronWRows, 1u}))
+    return GDPA_ERR_CUDA;
+  SumKronLaunch L{};
+  L.status = static_cast<DeviceStatus*>(workspace);
+  L.y = static_cast<__nv_bfloat16*>(y);
+  L.B = p->B;
+  L.S = p->S;
+  L.T = p->T;
+  L.D = p->D;
+  L.k = p->k;
+  L.timeout_ns = (uint64_t)(p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000) * 1000ull;
+  return launch_sumkron(L, ta, tx, tw, sms, s) == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 
 gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {

@@ -148,6 +148,18 @@ struct RotaryApplyArgs {
 };
 cudaError_t launch_rotary_apply(const RotaryApplyArgs& a, int sms, cudaStream_t stream);
 
+// SumKronLinear forward (maps: A [kT][S] boxes 64 x 128, X [B][S][D] boxes
+// 64 x 64 x 1, W [kD][D] boxes 64 x kSumKronWRows, bf16).
+constexpr int kSumKronWRows = 16;
+struct SumKronLaunch {
+  DeviceStatus* status;
+  __nv_bfloat16* y;
+  int B, S, T, D, k;
+  uint64_t timeout_ns;
+};
+cudaError_t launch_sumkron(const SumKronLaunch& L, const CUtensorMap& ta, const CUtensorMap& tx,
+                           const CUtensorMap& tw, int sms, cudaStream_t s);
+
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,

@@ -27,7 +27,7 @@ EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_s
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
             "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
             "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table",
-            "gdpa_rotary_apply")
+            "gdpa_rotary_apply", "gdpa_sumkron_workspace_size", "gdpa_sumkron_forward")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -40,6 +40,11 @@ class gdpa_params_t(ctypes.Structure):
                 ("wait_timeout_us", ctypes.c_int),
                 ("head_phi", ctypes.POINTER(ctypes.c_int32)),
                 ("rope_q", ctypes.c_void_p), ("rope_kv", ctypes.c_void_p)]
+
+
+class gdpa_sumkron_params_t(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("S", ctypes.c_int), ("T", ctypes.c_int), ("D", ctypes.c_int),
+                ("k", ctypes.c_int), ("wait_timeout_us", ctypes.c_int)]
 
 
 class gdpa_rotary_params_t(ctypes.Structure):
@@ -106,6 +111,11 @@ def load(path: str = LIB_PATH):
     lib.gdpa_rotary_apply.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp, vp,
                                       ctypes.c_int, st]
     lib.gdpa_rotary_apply.restype = ctypes.c_int
+    SP = ctypes.POINTER(gdpa_sumkron_params_t)
+    lib.gdpa_sumkron_workspace_size.argtypes = [SP]
+    lib.gdpa_sumkron_workspace_size.restype = sz
+    lib.gdpa_sumkron_forward.argtypes = [SP, vp, vp, vp, vp, vp, sz, st]
+    lib.gdpa_sumkron_forward.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -133,6 +143,15 @@ def gdpa_rotary_table(r: gdpa_rotary_params_t, B, total, offsets, time, table, s
 def gdpa_rotary_apply(total, H, D, x, table, y, inverse, stream) -> int:
     return int(load().gdpa_rotary_apply(int(total), int(H), int(D), x, table, y, int(inverse),
                                         stream))
+
+
+def gdpa_sumkron_workspace_size(p: gdpa_sumkron_params_t) -> int:
+    return int(load().gdpa_sumkron_workspace_size(ctypes.byref(p)))
+
+
+def gdpa_sumkron_forward(p, x, a, w, y, workspace, workspace_bytes, stream) -> int:
+    return int(load().gdpa_sumkron_forward(ctypes.byref(p), x, a, w, y, workspace,
+                                           workspace_bytes, stream))
 
 
 def gdpa_forward_grouped_workspace_size(problems) -> int:
@@ -259,6 +278,25 @@ def rotary_table(offsets, time, D, time_scale, *, theta=None, phi=None, out=None
     rc = gdpa_rotary_table(r, B, total, _ptr(offsets), _ptr(time), _ptr(out), _stream(stream))
     _check(rc, "gdpa_rotary_table")
     return out
+
+
+def sumkron_forward(x, a, w, *, out=None, workspace=None, stream=None):
+    """SumKronLinear: y [B,T,D] = sum_r a[r] @ x[b] @ w[r] for x [B,S,D],
+    a [k,T,S], w [k,D,D] (bf16 CUDA tensors).  Returns (y, workspace)."""
+    import torch
+    B, S, D = x.shape
+    k, T, _ = a.shape
+    p = gdpa_sumkron_params_t(int(B), int(S), int(T), int(D), int(k), 0)
+    if out is None:
+        out = torch.empty((B, T, D), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        n = gdpa_sumkron_workspace_size(p)
+        if n == 0:
+            raise GdpaError(2, "gdpa_sumkron_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(gdpa_sumkron_forward(p, _ptr(x), _ptr(a), _ptr(w), _ptr(out), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "gdpa_sumkron_forward")
+    return out, workspace
 
 
 def rotary_apply(x, table, *, inverse=False, out=None, stream=None):

@@ -180,7 +180,8 @@ def test_struct_layouts_match_the_header(tmp_path):
     import subprocess
     structs = {"gdpa_params_t": gdpa.gdpa_params_t,
                "gdpa_forward_problem_t": gdpa.gdpa_forward_problem_t,
-               "gdpa_rotary_params_t": gdpa.gdpa_rotary_params_t}
+               "gdpa_rotary_params_t": gdpa.gdpa_rotary_params_t,
+               "gdpa_sumkron_params_t": gdpa.gdpa_sumkron_params_t}
     lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "gdpa.h"', 'int main(void) {']
     for name, cls in structs.items():
         lines.append(f'  printf("{name} %zu\\n", sizeof({name}));')
@@ -198,3 +199,20 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert int(got[name]) == ctypes.sizeof(cls), name
         for field, _ in cls._fields_:
             assert int(got[f"{name}.{field}"]) == getattr(cls, field).offset, (name, field)
+
+
+def test_sumkron_validation(lib):
+    """Shapes the fused kernel does not cover are refused before any launch."""
+    def sp(**kw):
+        base = dict(B=4, S=256, T=32, D=384, k=8, wait_timeout_us=0)
+        base.update(kw)
+        return gdpa.gdpa_sumkron_params_t(**base)
+    assert gdpa.gdpa_sumkron_workspace_size(sp()) == 256
+    for kw, expect in [(dict(T=16), 2), (dict(D=192), 2), (dict(S=100), 2), (dict(S=320), 2),
+                       (dict(k=3), 2),
+                       (dict(B=-1), 1), (dict(k=0), 1), (dict(S=0), 1)]:
+        assert gdpa.gdpa_sumkron_workspace_size(sp(**kw)) == 0
+        assert gdpa.gdpa_sumkron_forward(sp(**kw), FAKE, FAKE, FAKE, FAKE, FAKE, 256, None) == \
+            expect, kw
+    assert gdpa.gdpa_sumkron_forward(sp(), FAKE + 8, FAKE, FAKE, FAKE, FAKE, 256, None) == 1
+    assert gdpa.gdpa_sumkron_forward(sp(), FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == 3

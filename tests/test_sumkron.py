@@ -1,0 +1,65 @@
+"""SumKronLinear on the GPU vs the fp64 oracle (``oracle.sumkron``)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import sumkron
+from parity import compare
+from workloads import SUMKRON_CONFIG, make_sumkron
+
+pytestmark = pytest.mark.gpu
+
+
+def run(gdpa, x, a, w):
+    y, ws = gdpa.sumkron_forward(x.cuda(), a.cuda(), w.cuda())
+    assert gdpa.device_status(ws) == 0
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("D", [128, 256, 384])
+@pytest.mark.parametrize("T,k", [(32, 4), (32, 8), (64, 2), (64, 4)])
+def test_shapes(cuda_lib, D, T, k):
+    # B = 7: a partial last group; S = 128: two 64-seed chunks
+    x, a, w = make_sumkron(7, 128, T, D, k, seed=D + T + k)
+    compare("Y", run(cuda_lib, x, a, w), sumkron.forward(x, a, w))
+
+
+@pytest.mark.parametrize("S", [64, 192, 256])
+@pytest.mark.parametrize("B", [1, 4, 150, 333])
+def test_seeds_and_batch(cuda_lib, S, B):
+    """Batches below, at and above one group per SM (148); seeds from one
+    chunk to four."""
+    x, a, w = make_sumkron(B, S, 32, 128, 4, seed=S + B)
+    compare("Y", run(cuda_lib, x, a, w), sumkron.forward(x, a, w))
+
+
+def test_empty_batch(cuda_lib):
+    x, a, w = make_sumkron(0, 64, 32, 128, 4)
+    y = run(cuda_lib, x, a, w)
+    assert y.shape == (0, 32, 128)
+
+
+def test_full_size_sampled(cuda_lib):
+    """The page's typical configuration at full batch: samples spread over
+    the batch (first, last, every CTA's first and later groups) against the
+    oracle one by one."""
+    c = SUMKRON_CONFIG
+    x, a, w = make_sumkron(c["B"], c["S"], c["T"], c["D"], c["k"], seed=1)
+    y = run(cuda_lib, x, a, w).cpu()
+    idx = np.unique(np.concatenate([[0, 1, 2, 3, c["B"] - 1], np.arange(5, c["B"], 97)]))
+    ref = sumkron.forward(x[idx], a, w)
+    compare("Y", y[idx], ref)
+
+
+def test_rows_are_independent(cuda_lib):
+    """Each sample's output depends on its own X only: changing one sample
+    leaves the others bit-identical."""
+    x, a, w = make_sumkron(9, 64, 32, 256, 4, seed=3)
+    y1 = run(cuda_lib, x, a, w)
+    x2 = x.clone()
+    x2[4] = -x2[4]
+    y2 = run(cuda_lib, x2, a, w)
+    keep = [i for i in range(9) if i != 4]
+    assert torch.equal(y1[keep], y2[keep])
+    assert torch.equal(y2[4], -y1[4])  # linear in X, and negation is exact

@@ -223,3 +223,19 @@ def event_times(lens, seed: int) -> np.ndarray:
             out[pos:pos + L] = starts[b] + np.cumsum(g)
         pos += L
     return out
+
+
+# SumKronLinear (second stage of Hierarchical Seed Pooling): the page's typical
+# configuration is S = 256 seeds, T = 32 tokens, D = 384, rank k = 8; the batch
+# is the seed-pooling workload's (2048 samples).  X ~ N(0, 1); A ~ N(0, 1/S)
+# and W ~ N(0, 1/(k D)), so Y = sum_r A_r X W_r has unit variance.  All bf16.
+SUMKRON_CONFIG = dict(B=2048, S=256, T=32, D=384, k=8)
+
+
+def make_sumkron(B, S, T, D, k, seed=0, device="cpu"):
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = _normal_bf16((B, S, D), 1.0, gen, device)
+    a = _normal_bf16((k, T, S), 1.0 / math.sqrt(S), gen, device)
+    w = _normal_bf16((k, D, D), 1.0 / math.sqrt(k * D), gen, device)
+    return x, a, w
