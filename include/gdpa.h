@@ -107,8 +107,9 @@ typedef struct {
    * bytes) and run the attention kernels on the copies; the backward turns dQ
    * and dK back in place at the end.  debug_flags bit 2 makes the forward turn
    * each Q tile and K block in shared memory inside the attention kernel
-   * instead (no copies; measured slower).  Not accepted by the grouped
-   * forward (GDPA_ERR_UNSUPPORTED). */
+   * instead (no copies; measured slower).  The grouped forward accepts the
+   * tables per problem (streamed turn only; bit 2 there is
+   * GDPA_ERR_UNSUPPORTED). */
   const void* rope_q;
   const void* rope_kv;
 } gdpa_params_t;

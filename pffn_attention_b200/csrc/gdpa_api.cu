@@ -238,6 +238,8 @@ struct LaunchGroup {
 // kernel writes.
 struct GroupedLayout {
   size_t off_jobs = 0, tables_end = 0, total = 0;
+  // per caller problem with rotary tables: its turned Q and K copies (0 = none)
+  std::vector<size_t> rope_q, rope_k;
 };
 
 // Validates every problem, forms the launch groups and lays out the workspace.
@@ -252,7 +254,8 @@ gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
     gdpa_status_t st = check_forward_args(p, f.q, f.k, f.v, f.q_offsets, f.kv_offsets, f.bias,
                                           f.o, f.lse);
     if (st != GDPA_OK) return st;
-    if (p->rope_q) return GDPA_ERR_UNSUPPORTED;  // rotation: single-problem calls only
+    if (p->rope_q && (p->debug_flags & kDebugFusedRotary))
+      return GDPA_ERR_UNSUPPORTED;  // grouped calls turn Q and K in a streaming pass
     const int block_n = forward_block_n(p->D, p->phi, eff_max_kv(p), p->debug_flags);
     for (int phi = 0; phi <= 3; ++phi) {
       const uint64_t heads = phi_heads(p, phi);
@@ -295,6 +298,17 @@ gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
     g.off_info = total;
     g.off_eprob = align256(g.off_info + (size_t)g.entries * sizeof(int4));
     total = align256(g.off_eprob + (size_t)g.entries * sizeof(int32_t));
+  }
+  // rotary: turned copies of each such problem's Q and K
+  lay.rope_q.assign(n, 0);
+  lay.rope_k.assign(n, 0);
+  for (int i = 0; i < n; ++i) {
+    const gdpa_params_t* p = &probs[i].params;
+    if (!p->rope_q) continue;
+    lay.rope_q[i] = total;
+    total = align256(total + (size_t)p->total_q * p->H * p->D * 2);
+    lay.rope_k[i] = total;
+    total = align256(total + (size_t)p->total_kv * p->H * p->D * 2);
   }
   lay.total = total;
   return GDPA_OK;
@@ -574,6 +588,22 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   cudaStream_t s = (cudaStream_t)stream;
 
+  // rotary problems: Q and K turned into workspace copies first (one streaming
+  // launch each); their tensor maps below read the copies
+  std::vector<const void*> qsrc(n_problems), ksrc(n_problems);
+  for (int i = 0; i < n_problems; ++i) {
+    const gdpa_params_t* p = &problems[i].params;
+    qsrc[i] = problems[i].q;
+    ksrc[i] = problems[i].k;
+    if (!p->rope_q) continue;
+    void* rq = ws + lay.rope_q[i];
+    void* rk = ws + lay.rope_k[i];
+    if (turn_qk(p, problems[i].q, problems[i].k, rq, rk, 0, sms, s) != cudaSuccess)
+      return GDPA_ERR_CUDA;
+    qsrc[i] = rq;
+    ksrc[i] = rk;
+  }
+
   // the cleared status and every table staged on the host, copied in one transfer
   std::vector<uint8_t> host(lay.tables_end, 0);
   auto at = [&](size_t off) { return host.data() + off; };
@@ -607,12 +637,12 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
       // encoded into an aligned local object, then copied into the staging bytes
       CUtensorMap m;
       if (p->total_q > 0) {
-        if (!make_map(&m, f.q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+        if (!make_map(&m, qsrc[vp.src], p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
         std::memcpy(&maps[3 * j], &m, sizeof(m));
         if (q_map[gi] < 0) q_map[gi] = (int)j;
       }
       if (p->total_kv > 0) {
-        if (!make_map(&m, f.k, p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
+        if (!make_map(&m, ksrc[vp.src], p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
         std::memcpy(&maps[3 * j + 1], &m, sizeof(m));
         if (!make_map(&m, f.v, p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
         std::memcpy(&maps[3 * j + 2], &m, sizeof(m));

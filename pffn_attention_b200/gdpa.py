@@ -339,7 +339,7 @@ def forward_grouped(problems, *, workspace=None, stream=None):
     """Several GDPA problems in one call.  problems: a list of dicts with the
     tensors q, k, v, q_offsets, kv_offsets (and optional bias, out, lse) and the
     keyword arguments of forward() (phi, scale, window, bias_kind,
-    max_seqlen_q, max_seqlen_kv, head_phi).  Returns ([(o, lse), ...], workspace)."""
+    max_seqlen_q, max_seqlen_kv, head_phi, rope).  Returns ([(o, lse), ...], workspace)."""
     import torch
     arr = (gdpa_forward_problem_t * len(problems))()
     outs, keep = [], []
@@ -350,7 +350,8 @@ def forward_grouped(problems, *, workspace=None, stream=None):
                         phi=d.get("phi", "silu"), scale=d.get("scale", 1.0),
                         window=d.get("window", (-1, -1)), bias_kind=d.get("bias_kind", "none"),
                         max_seqlen_q=d.get("max_seqlen_q", 0),
-                        max_seqlen_kv=d.get("max_seqlen_kv", 0), head_phi=d.get("head_phi"))
+                        max_seqlen_kv=d.get("max_seqlen_kv", 0), head_phi=d.get("head_phi"),
+                        rope=d.get("rope"))
         o = d.get("out") if d.get("out") is not None else torch.empty_like(q)
         lse = d.get("lse")
         if lse is None and _any_softmax(p):

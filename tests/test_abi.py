@@ -134,8 +134,9 @@ def test_grouped_forward_validation(lib):
 
 def test_rotary_validation(lib):
     """Rotary tables: D, time scale, jagged sizes and alignment are checked on
-    the host; the tables must come as a pair; the grouped forward refuses them
-    (not built); the streamed turn adds the turned copies to the workspace."""
+    the host; the tables must come as a pair; the streamed turn adds the
+    turned copies to the workspace (single and grouped calls); the grouped
+    call refuses the in-kernel turn."""
     def rp(D=64, scale=60.0):
         return gdpa.gdpa_rotary_params_t(D, scale, None, None)
     assert gdpa.gdpa_rotary_table_bytes(64, 10) == 10 * 32 * 4
@@ -172,7 +173,16 @@ def test_rotary_validation(lib):
     a[0].params = p
     for name in ("q", "k", "v", "q_offsets", "kv_offsets", "o"):
         setattr(a[0], name, FAKE)
-    assert gdpa.gdpa_forward_grouped_workspace_size(a) == 0
+    assert gdpa.gdpa_forward_grouped_workspace_size(a) == 0  # bit 2 (in-kernel turn) set
+    p.debug_flags = 0
+    a[0].params = p
+    plain = (gdpa.gdpa_forward_problem_t * 1)()
+    plain[0].params = _params()
+    for name in ("q", "k", "v", "q_offsets", "kv_offsets", "o"):
+        setattr(plain[0], name, FAKE)
+    # the grouped call keeps turned copies of the problem's Q and K
+    assert gdpa.gdpa_forward_grouped_workspace_size(a) == \
+        gdpa.gdpa_forward_grouped_workspace_size(plain) + 2560 + 2048
 
 
 def test_struct_layouts_match_the_header(tmp_path):

@@ -115,3 +115,45 @@ def test_grouped_many_small_problems(cuda_lib):
         compare("O", o, ro)
         if w.phi == PHI_SOFTMAX:
             compare_lse(lse, rlse)
+
+
+def test_grouped_with_rotary_problems(cuda_lib):
+    """Problems with the rotary temporal embedding in a grouped call: each one
+    equals its own single call (turned Q and K, bit for bit) and the oracle."""
+    from oracle import rotary
+    from workloads import EVENT_TIME_SCALE, event_times
+    specs = [
+        (make_workload(4, seed=410, q_lens=[300, 1, 129], kv_lens=[300, 1, 129], H=3,
+                       window=(127, 0)), 1),
+        (make_workload(4, seed=411, q_lens=[64, 500], kv_lens=[64, 500], H=2, D=64,
+                       window=(31, 0), scale=1.0 / 8), 2),
+        (make_workload(3, seed=412, q_lens=[32, 32], kv_lens=[200, 17], H=2), None),  # none
+    ]
+    dev_probs, angs = [], []
+    for w, seed in specs:
+        d = _to_dev(w, None)
+        if seed is not None:
+            times = event_times(w.q_lens, seed)
+            table = cuda_lib.rotary_table(d["q_offsets"], torch.tensor(times, device="cuda"),
+                                          w.D, EVENT_TIME_SCALE)
+            d["rope"] = (table, table)
+            angs.append(rotary.angles(w.q_offsets, times, w.D, EVENT_TIME_SCALE))
+        else:
+            angs.append(None)
+        dev_probs.append(d)
+    outs, ws = cuda_lib.forward_grouped(dev_probs)
+    assert cuda_lib.device_status(ws) == 0
+    torch.cuda.synchronize()
+    for (w, _), d, a, (o, lse) in zip(specs, dev_probs, angs, outs):
+        kw = {k: d[k] for k in ("phi", "scale", "window", "bias", "bias_kind", "max_seqlen_q",
+                                "max_seqlen_kv")}
+        o1, lse1, ws1 = cuda_lib.forward(d["q"], d["k"], d["v"], d["q_offsets"],
+                                         d["kv_offsets"], rope=d.get("rope"), **kw)
+        assert cuda_lib.device_status(ws1) == 0
+        assert torch.equal(o, o1) and torch.equal(lse, lse1)
+        if a is None:
+            ro, _ = oracle.forward_workload(w)
+        else:
+            ro, _ = rotary.forward(w.q, w.k, w.v, w.q_offsets, w.kv_offsets, a, a, phi=w.phi,
+                                   scale=w.scale, window=(w.window_left, w.window_right))
+        compare("O", o, ro)
