@@ -84,6 +84,8 @@ def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
 KERNEL_SOURCES = {
     "gdpa_backward": ["gdpa_bwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
     "gdpa_forward": ["gdpa_fwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_sumkron_forward": ["gdpa_sumkron.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_rotary_apply": ["gdpa_rotary.cu", "gdpa_internal.h", "sm100.cuh"],
 }
 
 
@@ -611,9 +613,14 @@ def run_rotary(args):
                                       **kw))
     t_ms = timed(lambda: gdpa.rotary_table(qo, times, w.D, EVENT_TIME_SCALE, out=table,
                                            stream=stream))
+    qr, kr = torch.empty_like(w.q), torch.empty_like(w.k)
+    a_ms = timed(lambda: (gdpa.rotary_apply(w.q, table, out=qr, stream=stream),
+                          gdpa.rotary_apply(w.k, table, out=kr, stream=stream)))
     assert gdpa.device_status(ws, stream) == 0
     flops = useful_flops(w, False)[0]
     byts = algorithmic_bytes(w, False)[0] + table.numel() * 4  # + one read of the table
+    turn_bytes = 2.0 * 2 * (w.q.numel() + w.k.numel()) + 2.0 * table.numel() * 4
+    peaks, src = load_peaks()
     return {"metric": "GDPA forward with rotary temporal embedding, sliding-window "
                       "self-attention (useful TFLOP/s)",
             "value": round(flops / (r_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
@@ -622,7 +629,14 @@ def run_rotary(args):
             "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D,
                        "window": [w.window_left, w.window_right], "l2": "inputs > L2"},
             "plain_forward_ms": round(p_ms, 4), "rotary_overhead": round(r_ms / p_ms, 3),
-            "table_ms": round(t_ms, 4), "achieved_gbs": round(byts / (r_ms * 1e-3) / 1e9, 1)}
+            "table_ms": round(t_ms, 4), "achieved_gbs": round(byts / (r_ms * 1e-3) / 1e9, 1),
+            # the turn pass (Q and K read and written, the table read once per tensor)
+            "roofline": {"bound": "hbm", "kernel": "gdpa_rotary_apply", "ms": round(a_ms, 4),
+                         "achieved": round(turn_bytes / (a_ms * 1e-3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(turn_bytes / (a_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "traffic": measured_traffic("gdpa_rotary_apply", w.B),
+                         "algorithmic": turn_bytes, "peak_source": src}}
 
 
 def run_sumkron(args):
@@ -662,7 +676,9 @@ def run_sumkron(args):
             "config": {"workload": "sumkron_hsp", **c, "l2": "inputs > L2"},
             "roofline": {"bound": "tensor", "achieved": round(tf, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                         "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "traffic": measured_traffic("gdpa_sumkron_forward", B),
+                         "traffic_unit": "bytes per launch", "algorithmic": byts,
                          "peak_source": src},
             "achieved_gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
 
