@@ -84,8 +84,8 @@ def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
 KERNEL_SOURCES = {
     "gdpa_backward": ["gdpa_bwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
     "gdpa_forward": ["gdpa_fwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
-    "gdpa_sumkron_forward": ["gdpa_sumkron.cu", "gdpa_internal.h", "sm100.cuh"],
-    "gdpa_rotary_apply": ["gdpa_rotary.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_sumkron_forward": ["gdpa_sumkron.cu", "gdpa_ops.h", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_rotary_apply": ["gdpa_rotary.cu", "gdpa_ops.h", "gdpa_internal.h", "sm100.cuh"],
 }
 
 

@@ -172,6 +172,9 @@ typedef struct {
   int D;               /* embedding dim: 128, 256 or 384 */
   int k;               /* Kronecker rank: k * T a multiple of 128 */
   int wait_timeout_us; /* bound on any single in-kernel wait; 0 = 2 s */
+  int debug_flags;     /* 0 in normal use.  Bit 0 drops one X load in CTA 0 so that
+                          the bounded-wait path can be tested (the call's status
+                          becomes GDPA_ERR_TIMEOUT); other bits are ignored */
 } gdpa_sumkron_params_t;
 
 /* Workspace bytes (the device status block); 0 on invalid parameters. */

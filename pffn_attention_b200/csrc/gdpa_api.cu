@@ -789,6 +789,7 @@ gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, const void* x
   L.T = p->T;
   L.D = p->D;
   L.k = p->k;
+  L.debug_flags = p->debug_flags;
   L.timeout_ns = (uint64_t)(p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000) * 1000ull;
   return launch_sumkron(L, ta, tx, tw, sms, s) == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }

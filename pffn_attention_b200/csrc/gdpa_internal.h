@@ -117,49 +117,6 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
                             int32_t* order, int4* info, int max_q, int max_kv,
                             DeviceStatus* status, cudaStream_t stream);
-// debug_flags bit 2: the forward turns Q and K inside the attention kernel
-// (warps 2-3, in shared memory) instead of in a streaming pass first.
-constexpr int kDebugFusedRotary = 4;
-inline bool rotary_streamed(const void* rope_q, int debug_flags) {
-  return rope_q != nullptr && !(debug_flags & kDebugFusedRotary);
-}
-
-// Rotary temporal embedding table: angles t theta_i + tau_t phi_i per token.
-struct RotaryArgs {
-  // theta_i / pi as hi + lo, and phi_i / pi: angles in half-turns
-  float theta_hi[64], theta_lo[64], phi_pi[64];
-  double time_scale;
-  int D, B;
-  int64_t total;
-};
-cudaError_t launch_rotary_table(const RotaryArgs& r, const int32_t* offsets,
-                                const int64_t* time, uint32_t* table, cudaStream_t stream);
-// y = x turned by the table's angles (or back, when inverse), bf16 [total][H][D].
-struct RotaryJob {
-  const void* x;
-  void* y;
-  const uint32_t* table;
-  int64_t total;
-};
-struct RotaryApplyArgs {
-  RotaryJob job[2];  // an unused job has total 0
-  int H, D;
-  int inverse;
-};
-cudaError_t launch_rotary_apply(const RotaryApplyArgs& a, int sms, cudaStream_t stream);
-
-// SumKronLinear forward (maps: A [kT][S] boxes 64 x 128, X [B][S][D] boxes
-// 64 x 64 x 1, W [kD][D] boxes 64 x kSumKronWRows, bf16).
-constexpr int kSumKronWRows = 16;
-struct SumKronLaunch {
-  DeviceStatus* status;
-  __nv_bfloat16* y;
-  int B, S, T, D, k;
-  uint64_t timeout_ns;
-};
-cudaError_t launch_sumkron(const SumKronLaunch& L, const CUtensorMap& ta, const CUtensorMap& tx,
-                           const CUtensorMap& tw, int sms, cudaStream_t s);
-
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
@@ -243,3 +200,5 @@ struct UnitStreamT {
 using UnitStream = UnitStreamT<false>;
 
 }  // namespace gdpa
+
+#include "gdpa_ops.h"

@@ -86,6 +86,7 @@ struct SkArgs {
   __nv_bfloat16* y;
   int B, S, k;
   int n_groups;
+  int debug_flags;
   uint64_t timeout_ns;
 };
 
@@ -127,6 +128,8 @@ __device__ void sk_producer_xa(const SkArgs& a, const SkSmem<C>& sm, const CUten
           for (int kc = 0; kc < NKC; ++kc, ++xc) {
             const int st = xc % C::NX;
             if (!SK_WAIT(C::B_XEMPTY + st, ((xc / C::NX) & 1) ^ 1, 0x000 + st)) return;
+            // test hook: CTA 0's second X chunk is never loaded
+            if ((a.debug_flags & 1) && blockIdx.x == 0 && xc == 1) continue;
             mbar_arrive_expect_tx(sm.bar(C::B_XFULL + st), C::X_BYTES);
             // samples past B read as zeros (their Y rows are not stored)
             tma_load_3d(sm.x(st), tx, sm.bar(C::B_XFULL + st), dc * 64, kc * 64,
@@ -404,6 +407,7 @@ cudaError_t launch_sumkron(const SumKronLaunch& L, const CUtensorMap& ta, const 
   a.B = L.B;
   a.S = L.S;
   a.k = L.k;
+  a.debug_flags = L.debug_flags;
   a.n_groups = (L.B + (128 / L.T) - 1) / (128 / L.T);
   a.timeout_ns = L.timeout_ns;
   if (a.n_groups == 0) return cudaSuccess;

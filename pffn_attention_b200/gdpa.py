@@ -44,7 +44,8 @@ class gdpa_params_t(ctypes.Structure):
 
 class gdpa_sumkron_params_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("S", ctypes.c_int), ("T", ctypes.c_int), ("D", ctypes.c_int),
-                ("k", ctypes.c_int), ("wait_timeout_us", ctypes.c_int)]
+                ("k", ctypes.c_int), ("wait_timeout_us", ctypes.c_int),
+                ("debug_flags", ctypes.c_int)]
 
 
 class gdpa_rotary_params_t(ctypes.Structure):
@@ -280,13 +281,15 @@ def rotary_table(offsets, time, D, time_scale, *, theta=None, phi=None, out=None
     return out
 
 
-def sumkron_forward(x, a, w, *, out=None, workspace=None, stream=None):
+def sumkron_forward(x, a, w, *, out=None, workspace=None, stream=None, wait_timeout_us=0,
+                    debug_flags=0):
     """SumKronLinear: y [B,T,D] = sum_r a[r] @ x[b] @ w[r] for x [B,S,D],
     a [k,T,S], w [k,D,D] (bf16 CUDA tensors).  Returns (y, workspace)."""
     import torch
     B, S, D = x.shape
     k, T, _ = a.shape
-    p = gdpa_sumkron_params_t(int(B), int(S), int(T), int(D), int(k), 0)
+    p = gdpa_sumkron_params_t(int(B), int(S), int(T), int(D), int(k), int(wait_timeout_us),
+                              int(debug_flags))
     if out is None:
         out = torch.empty((B, T, D), dtype=x.dtype, device=x.device)
     if workspace is None:

@@ -214,7 +214,7 @@ def test_struct_layouts_match_the_header(tmp_path):
 def test_sumkron_validation(lib):
     """Shapes the fused kernel does not cover are refused before any launch."""
     def sp(**kw):
-        base = dict(B=4, S=256, T=32, D=384, k=8, wait_timeout_us=0)
+        base = dict(B=4, S=256, T=32, D=384, k=8, wait_timeout_us=0, debug_flags=0)
         base.update(kw)
         return gdpa.gdpa_sumkron_params_t(**base)
     assert gdpa.gdpa_sumkron_workspace_size(sp()) == 256

@@ -50,3 +50,17 @@ def test_launch_errors_are_reported_at_the_call(cuda_lib):
                                ko.data_ptr(), None, o.data_ptr(), None, small.data_ptr(), 16,
                                torch.cuda.current_stream().cuda_stream)
     assert rc == 3  # GDPA_ERR_WORKSPACE
+
+
+def test_sumkron_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    """The SumKronLinear kernel's waits are bounded too: one dropped X load in
+    CTA 0 ends in GDPA_ERR_TIMEOUT, and the next call on the context is exact."""
+    from oracle import sumkron
+    from workloads import make_sumkron
+    x, a, w = make_sumkron(9, 128, 32, 128, 4, seed=7)
+    xd, ad, wd = x.cuda(), a.cuda(), w.cuda()
+    _, ws = cuda_lib.sumkron_forward(xd, ad, wd, wait_timeout_us=20000, debug_flags=1)
+    assert cuda_lib.device_status(ws) == 5  # GDPA_ERR_TIMEOUT
+    y, ws2 = cuda_lib.sumkron_forward(xd, ad, wd)
+    assert cuda_lib.device_status(ws2) == 0
+    compare("Y", y, sumkron.forward(x, a, w))
