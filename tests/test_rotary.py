@@ -266,3 +266,74 @@ def test_empty_samples(cuda_lib):
     kl = [5, 0, 0, 140]
     w = make_workload(4, seed=13, q_lens=ql, kv_lens=kl, window=(-1, -1))
     check(cuda_lib, w, seed=13, same_sequence=False)
+
+
+# -------------------------------------------------- full size, per-head activations
+@pytest.mark.slow
+def test_full_size_sliding_window_sampled(cuda_lib):
+    """The sliding-window workload at full size (B=512) with the rotary
+    embedding, forward and backward; samples spread over the batch (the
+    shortest, the longest, the last, random ones) against the oracle one by
+    one."""
+    from workloads import subset
+    w = make_workload(4, device="cuda", with_dout=True)
+    times = event_times(w.q_lens, 4)
+    tab = gpu_table(cuda_lib, w.q_offsets, times, w.D)
+    qo = _dev(w.q_offsets, torch.int32)
+    p = params(cuda_lib, w, tab, tab)
+    o, lse, _ = cuda_lib.forward(w.q, w.k, w.v, qo, qo, params=p)
+    dq, dk, dv, wsb = cuda_lib.backward(w.q, w.k, w.v, o, w.dout, lse, qo, qo, params=p)
+    assert cuda_lib.device_status(wsb) == 0
+    torch.cuda.synchronize()
+    order = np.argsort(w.q_lens)
+    picks = sorted({int(order[0]), int(order[-1]), w.B - 1, 0,
+                    *np.random.default_rng(44).choice(w.B, 4, replace=False).tolist()})
+    sub = subset(w, picks)
+    for name in ("q", "k", "v", "dout"):
+        setattr(sub, name, getattr(sub, name).cpu())
+    stimes = np.concatenate([times[w.q_offsets[b]:w.q_offsets[b + 1]] for b in picks])
+    ang = rotary.angles(sub.q_offsets, stimes, w.D, EVENT_TIME_SCALE)
+    kw = dict(phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right))
+    ro, rlse = rotary.forward(sub.q, sub.k, sub.v, sub.q_offsets, sub.kv_offsets, ang, ang, **kw)
+    rdq, rdk, rdv, _ = rotary.backward(sub.q, sub.k, sub.v, sub.dout, sub.q_offsets,
+                                       sub.kv_offsets, ang, ang, **kw)
+    rows = torch.tensor(np.concatenate([np.arange(w.q_offsets[b], w.q_offsets[b + 1])
+                                        for b in picks]), device="cuda")
+    compare("O", o[rows], ro)
+    compare("dQ", dq[rows], rdq)
+    compare("dK", dk[rows], rdk)
+    compare("dV", dv[rows], rdv)
+
+
+def test_head_phi_with_rotary(cuda_lib):
+    """A per-head activation vector with the rotary embedding: each head
+    matches the oracle with its own activation, forward and backward."""
+    import copy
+    from workloads import PHI_IDENTITY
+    ql = [200, 17, 129]
+    heads = [PHI_SOFTMAX, PHI_SILU, PHI_GELU, PHI_IDENTITY]
+    names = {PHI_SOFTMAX: "softmax", PHI_SILU: "silu", PHI_GELU: "gelu", PHI_IDENTITY: "identity"}
+    w = make_workload(2, seed=18, q_lens=ql, kv_lens=ql, H=4, D=64, scale=1.0,
+                      kv_std=1.0 / np.sqrt(64), window=(63, 0), with_dout=True, dout_std=0.125)
+    tq, tk, aq, ak = tables(cuda_lib, w, 18, True)
+    qo = _dev(w.q_offsets, torch.int32)
+    p = cuda_lib.make_params(w.B, w.H, w.D, int(w.q_offsets[-1]), int(w.kv_offsets[-1]),
+                             phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+                             max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv,
+                             head_phi=[names[h] for h in heads], rope=(tq, tk))
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    o, lse, _ = cuda_lib.forward(q, k, v, qo, qo, params=p)
+    dq, dk, dv, wsb = cuda_lib.backward(q, k, v, o, w.dout.cuda(), lse, qo, qo, params=p)
+    assert cuda_lib.device_status(wsb) == 0
+    torch.cuda.synchronize()
+    for h, phi in enumerate(heads):
+        wp = copy.copy(w)
+        wp.phi = phi
+        kw = dict(phi=phi, scale=w.scale, window=(w.window_left, w.window_right))
+        ro, _ = rotary.forward(w.q, w.k, w.v, w.q_offsets, w.kv_offsets, aq, ak, **kw)
+        rdq, rdk, rdv, _ = rotary.backward(w.q, w.k, w.v, w.dout, w.q_offsets, w.kv_offsets, aq,
+                                           ak, **kw)
+        compare(f"O[h{h}]", o[:, h], ro[:, h])
+        compare(f"dQ[h{h}]", dq[:, h], rdq[:, h])
+        compare(f"dK[h{h}]", dk[:, h], rdk[:, h])
+        compare(f"dV[h{h}]", dv[:, h], rdv[:, h])

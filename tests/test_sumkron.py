@@ -63,3 +63,13 @@ def test_rows_are_independent(cuda_lib):
     keep = [i for i in range(9) if i != 4]
     assert torch.equal(y1[keep], y2[keep])
     assert torch.equal(y2[4], -y1[4])  # linear in X, and negation is exact
+
+
+@pytest.mark.parametrize("D", [128, 384])
+def test_t64_larger_batch(cuda_lib, D):
+    """T = 64 (two samples per 128-row tile) over a batch of 301 samples (151
+    groups: one CTA takes two), k = 4, S = 256."""
+    x, a, w = make_sumkron(301, 256, 64, D, 4, seed=D + 64)
+    y = run(cuda_lib, x, a, w).cpu()
+    idx = np.arange(0, 301, 7)
+    compare("Y", y[idx], sumkron.forward(x[idx], a, w))
