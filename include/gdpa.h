@@ -142,9 +142,14 @@ GDPA_API size_t gdpa_rotary_table_bytes(int D, int64_t total);
  * the gaps to mean anything).  The position part t * theta_i is reduced
  * modulo 2 pi without rounding error (positions below 2^24; the default
  * frequencies are taken in fp64), then the cosine and sine are taken in fp32
- * and rounded to fp16.  One
- * table serves every head, the forward and the backward, and every layer that
- * sees the same sequence.  Asynchronous on stream. */
+ * and rounded to fp16.  One table serves every head, the forward and the
+ * backward, and every layer that sees the same sequence.  Asynchronous on
+ * stream.  Errors (before any launch): GDPA_ERR_UNSUPPORTED for another D;
+ * GDPA_ERR_INVALID_ARG for a time scale that is not a positive finite number,
+ * a non-finite frequency, B outside [0, 16384], total outside [0, 2^31), or a
+ * null or unaligned pointer when B and total are positive; GDPA_ERR_CUDA when
+ * the launch fails.  Offsets are trusted (clamped to [0, total] on the
+ * device). */
 GDPA_API gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, int64_t total,
                                          const int32_t* offsets, const int64_t* time,
                                          void* table, gdpa_stream_t stream);
@@ -152,7 +157,10 @@ GDPA_API gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, i
 /* y = x turned by the table's angles (inverse = 0) or turned back (inverse
  * != 0: the transpose, which maps dL/dx' to dL/dx), for x, y bf16
  * [total][H][D] (device, 16-byte aligned; y may be x) and a table from
- * gdpa_rotary_table for the same tokens.  Asynchronous on stream. */
+ * gdpa_rotary_table for the same tokens.  Asynchronous on stream.  Errors:
+ * GDPA_ERR_UNSUPPORTED for another D; GDPA_ERR_INVALID_ARG for H <= 0, total
+ * outside [0, 2^31) or a null or unaligned pointer (total > 0);
+ * GDPA_ERR_CUDA when the launch fails. */
 GDPA_API gdpa_status_t gdpa_rotary_apply(int64_t total, int H, int D, const void* x,
                                          const void* table, void* y, int inverse,
                                          gdpa_stream_t stream);
@@ -183,7 +191,12 @@ GDPA_API size_t gdpa_sumkron_workspace_size(const gdpa_sumkron_params_t* p);
 /* y [B][T][D] from x [B][S][D], a [k][T][S] (A_1..A_k) and w [k][D][D]
  * (W_1..W_k), all bf16 row-major device arrays, 16-byte aligned, the
  * caller's.  The workspace's status is cleared on the stream first; read it
- * with gdpa_get_device_status.  Asynchronous on stream. */
+ * with gdpa_get_device_status (GDPA_ERR_TIMEOUT if a bounded wait ran out).
+ * Asynchronous on stream.  Errors (before any launch): GDPA_ERR_UNSUPPORTED
+ * for shapes outside the limits above; GDPA_ERR_INVALID_ARG for negative or
+ * zero sizes, or a null or unaligned pointer; GDPA_ERR_WORKSPACE for a
+ * workspace below gdpa_sumkron_workspace_size; GDPA_ERR_CUDA when a CUDA call
+ * fails. */
 GDPA_API gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, const void* x,
                                             const void* a, const void* w, void* y,
                                             void* workspace, size_t workspace_bytes,
