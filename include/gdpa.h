@@ -293,7 +293,10 @@ GDPA_API gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* proble
  * overlap on the GPU (on different streams, or from different host threads)
  * race and must be serialised by the caller.  Each call overwrites what it
  * needs, so nothing from an earlier call leaks in.  Device-side status of
- * these calls is not readable through gdpa_get_device_status. */
+ * these calls is not readable through gdpa_get_device_status.  With rotary
+ * tables (rope_q / rope_kv) the attention kernel turns Q and K itself (as
+ * debug_flags bit 2 selects for gdpa_forward): no turned copies, the same
+ * results bit for bit. */
 GDPA_API gdpa_status_t gdpa_forward_no_alloc(const gdpa_params_t* p, const void* q,
                                              const void* k, const void* v,
                                              const int32_t* q_offsets,

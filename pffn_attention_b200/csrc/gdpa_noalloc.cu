@@ -61,6 +61,11 @@ extern "C" GDPA_API gdpa_status_t gdpa_forward_no_alloc(
     gdpa_stream_t stream) {
   if (!p) return GDPA_ERR_INVALID_ARG;
   if (p->B > kNoAllocMaxBatch) return GDPA_ERR_WORKSPACE;  // beyond the fixed scratch
+  // rotary tables: Q and K are turned inside the attention kernel, which needs
+  // no turned copies (and gives the same bits as the streamed turn)
+  gdpa_params_t pp = *p;
+  if (pp.rope_q) pp.debug_flags |= gdpa::kDebugFusedRotary;
+  p = &pp;
   const size_t need = gdpa_workspace_size(p, 0);
   if (need == 0) return GDPA_ERR_INVALID_ARG;
   if (need > kNoAllocBytes) return GDPA_ERR_WORKSPACE;

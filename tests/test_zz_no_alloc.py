@@ -51,3 +51,30 @@ def test_no_alloc_forward_matches_forward_on_consecutive_calls(cuda_lib):
 def test_no_alloc_rejects_batches_beyond_its_scratch(cuda_lib):
     p = cuda_lib.make_params(16385, 1, 64, 16385, 16385)
     assert cuda_lib.gdpa_forward_no_alloc(p, 16, 16, 16, 16, 16, None, 16, None, None) == 3
+
+
+def test_no_alloc_with_rotary_matches_forward(cuda_lib):
+    """With rotary tables the no-alloc call turns Q and K inside the attention
+    kernel (no copies to hold) and gives gdpa_forward's streamed result bit for
+    bit."""
+    from workloads import EVENT_TIME_SCALE, event_times
+    ql = [300, 5, 129]
+    w = make_workload(4, seed=21, q_lens=ql, kv_lens=ql)
+    dev = torch.device("cuda")
+    qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    table = cuda_lib.rotary_table(qo, torch.tensor(event_times(ql, 21), device=dev), w.D,
+                                  EVENT_TIME_SCALE)
+    kw = dict(phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+              max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv)
+    ref_o, ref_lse, ws = cuda_lib.forward(q, k, v, qo, qo, rope=(table, table), **kw)
+    assert cuda_lib.device_status(ws) == 0
+    p = cuda_lib.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, rope=(table, table), **kw)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((w.H, w.total_q), float("nan"), device=dev)
+    rc = cuda_lib.gdpa_forward_no_alloc(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        qo.data_ptr(), qo.data_ptr(), None, o.data_ptr(),
+                                        lse.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, cuda_lib.gdpa_status_string(rc)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse)
