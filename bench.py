@@ -585,7 +585,7 @@ def run_rotary(args):
     from workloads import EVENT_TIME_SCALE, event_times
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = make_workload(4, device=dev, with_dout=False)
+    w = make_workload(4, device=dev, with_dout=True)
     stream = torch.cuda.Stream(device=dev)
     qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
     times = torch.tensor(event_times(w.q_lens, 4), dtype=torch.int64, device=dev)
@@ -616,6 +616,26 @@ def run_rotary(args):
     qr, kr = torch.empty_like(w.q), torch.empty_like(w.k)
     a_ms = timed(lambda: (gdpa.rotary_apply(w.q, table, out=qr, stream=stream),
                           gdpa.rotary_apply(w.k, table, out=kr, stream=stream)))
+    # training step (forward + backward), with and without the rotary turn
+    dq, dk, dv = torch.empty_like(w.q), torch.empty_like(w.k), torch.empty_like(w.v)
+    _, _, _, wsb = gdpa.backward(w.q, w.k, w.v, o, w.dout, lse, qo, qo, rope=(table, table),
+                                 dq=dq, dk=dk, dv=dv, **kw)
+    _, _, _, wsb2 = gdpa.backward(w.q, w.k, w.v, o2, w.dout, lse2, qo, qo, dq=dq, dk=dk, dv=dv,
+                                  **kw)
+
+    def step(rope):
+        if rope:
+            gdpa.forward(w.q, w.k, w.v, qo, qo, rope=(table, table), out=o, lse=lse, workspace=ws,
+                         **kw)
+            gdpa.backward(w.q, w.k, w.v, o, w.dout, lse, qo, qo, rope=(table, table), dq=dq,
+                          dk=dk, dv=dv, workspace=wsb, **kw)
+        else:
+            gdpa.forward(w.q, w.k, w.v, qo, qo, out=o2, lse=lse2, workspace=ws2, **kw)
+            gdpa.backward(w.q, w.k, w.v, o2, w.dout, lse2, qo, qo, dq=dq, dk=dk, dv=dv,
+                          workspace=wsb2, **kw)
+    sr_ms = timed(lambda: step(True))
+    sp_ms = timed(lambda: step(False))
+    assert gdpa.device_status(wsb, stream) == 0
     assert gdpa.device_status(ws, stream) == 0
     flops = useful_flops(w, False)[0]
     byts = algorithmic_bytes(w, False)[0] + table.numel() * 4  # + one read of the table
@@ -630,6 +650,8 @@ def run_rotary(args):
                        "window": [w.window_left, w.window_right], "l2": "inputs > L2"},
             "plain_forward_ms": round(p_ms, 4), "rotary_overhead": round(r_ms / p_ms, 3),
             "table_ms": round(t_ms, 4), "achieved_gbs": round(byts / (r_ms * 1e-3) / 1e9, 1),
+            "train_step_ms": round(sr_ms, 4), "plain_train_step_ms": round(sp_ms, 4),
+            "train_rotary_overhead": round(sr_ms / sp_ms, 3),
             # the turn pass (Q and K read and written, the table read once per tensor)
             "roofline": {"bound": "hbm", "kernel": "gdpa_rotary_apply", "ms": round(a_ms, 4),
                          "achieved": round(turn_bytes / (a_ms * 1e-3) / 1e9, 1),
