@@ -157,7 +157,11 @@ GDPA_API gdpa_status_t gdpa_rotary_table(const gdpa_rotary_params_t* r, int B, i
 /* y = x turned by the table's angles (inverse = 0) or turned back (inverse
  * != 0: the transpose, which maps dL/dx' to dL/dx), for x, y bf16
  * [total][H][D] (device, 16-byte aligned; y may be x) and a table from
- * gdpa_rotary_table for the same tokens.  Asynchronous on stream.  Errors:
+ * gdpa_rotary_table for the same tokens.  A training step can turn Q and K
+ * once with this call, pass the turned copies (and no tables) to both
+ * gdpa_forward and gdpa_backward, and turn dQ and dK back with inverse = 1:
+ * two streaming passes instead of the three that rope_q / rope_kv imply.
+ * Asynchronous on stream.  Errors:
  * GDPA_ERR_UNSUPPORTED for another D; GDPA_ERR_INVALID_ARG for H <= 0, total
  * outside [0, 2^31) or a null or unaligned pointer (total > 0);
  * GDPA_ERR_CUDA when the launch fails. */
