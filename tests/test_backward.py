@@ -173,3 +173,14 @@ def test_bias_gradient(cuda_lib, phi, bias_kind, window):
         k0 = int(w.kv_offsets[4])
         assert torch.all(dbias[:, k0 + 64:k0 + 500] == 0)
         assert torch.all(dbias[:, int(w.kv_offsets[3]):int(w.kv_offsets[4])] == 0)
+
+
+def test_max_batch_backward(cuda_lib):
+    """16384 samples (the batch limit), softmax with a gate: dQ, dK, dV and dG
+    against the oracle."""
+    rng = np.random.default_rng(16385)
+    ql = rng.integers(0, 9, 16384)
+    kl = rng.integers(0, 17, 16384)
+    w = make_workload(5, seed=17, q_lens=ql, kv_lens=kl, H=2, D=32, with_dout=True,
+                      dout_std=0.125)
+    check_backward(cuda_lib, w)

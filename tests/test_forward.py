@@ -160,3 +160,17 @@ def test_kv_ring_resident_and_streamed(cuda_lib, phi, kv_lens):
         w = make_workload(2, seed=7 + sum(kv_lens), q_lens=ql, kv_lens=kv_lens, H=3, D=128,
                           phi=phi, scale=1.0, kv_std=1.0 / np.sqrt(128))
     check_against_oracle(cuda_lib, w)
+
+
+# -------------------------------------------------- the batch limit
+def test_max_batch(cuda_lib):
+    """16384 samples, the library's batch limit (the schedule's single-CTA
+    sort), with jagged tiny lengths including empty samples: every output row
+    against the oracle.  SiLU with the PFFN value distributions (K, V ~
+    N(0, 1/D), scale 1), as every element-wise test uses."""
+    rng = np.random.default_rng(16384)
+    ql = rng.integers(0, 9, 16384)
+    kl = rng.integers(0, 17, 16384)
+    w = make_workload(2, seed=16, q_lens=ql, kv_lens=kl, H=2, D=32, phi=PHI_SILU, scale=1.0,
+                      kv_std=1.0 / np.sqrt(32))
+    check_against_oracle(cuda_lib, w)

@@ -157,3 +157,23 @@ def test_grouped_with_rotary_problems(cuda_lib):
             ro, _ = rotary.forward(w.q, w.k, w.v, w.q_offsets, w.kv_offsets, a, a, phi=w.phi,
                                    scale=w.scale, window=(w.window_left, w.window_right))
         compare("O", o, ro)
+
+
+def test_grouped_at_the_entry_limit(cuda_lib):
+    """One launch group holding 16384 entries (its limit): two problems of the
+    same class, 12000 + 4384 tiny samples."""
+    rng = np.random.default_rng(420)
+    probs = []
+    for i, B in enumerate((12000, 4384)):
+        ql = rng.integers(0, 9, B).tolist()
+        kl = rng.integers(1, 17, B).tolist()
+        w = make_workload(2, seed=420 + i, q_lens=ql, kv_lens=kl, H=2, D=32, phi=PHI_SILU,
+                          scale=1.0, kv_std=1.0 / np.sqrt(32))
+        probs.append((w, None))
+    dev_probs = [_to_dev(w, None) for w, _ in probs]
+    outs, ws = cuda_lib.forward_grouped(dev_probs)
+    assert cuda_lib.device_status(ws) == 0
+    torch.cuda.synchronize()
+    for (w, _), (o, _) in zip(probs, outs):
+        ro, _ = oracle.forward_workload(w)
+        compare("O", o, ro)
