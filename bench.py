@@ -297,6 +297,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                if args.workload == DEFAULT_WORKLOAD and not args.phi else None)
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+                "spec_peak": SPEC_HBM_GBS, "spec_frac": round(achieved_gbs / SPEC_HBM_GBS, 4),
                 "traffic": None if traffic is None else round(traffic / 1e9, 3),
                 "traffic_unit": "GB per launch", "algorithmic": round(dom_bytes / 1e9, 3),
                 "kernel": dom_name, "peak_source": peak_src,
@@ -306,6 +307,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, p, qo, ko, training, dev, world)
+    per_workload = None
+    if world == 1 and args.workload == DEFAULT_WORKLOAD and args.batch is None \
+            and not args.no_per_workload:
+        per_workload = run_per_workload(args, dev, peaks, peak_src)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -328,11 +333,60 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "fwd_tflops": round(f_fwd / (fwd_ms * 1e-3) / 1e12, 1),
         "bwd_tflops": round(f_bwd / (bwd_ms * 1e-3) / 1e12, 1) if training else None,
         "roofline": roofline,
+        "per_workload": per_workload,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
     }
     return line, w
+
+
+def run_per_workload(args, dev, peaks, peak_src):
+    """The three forward-only workloads at full size (PFFN SiLU, seed pooling,
+    sliding window): each timed as its own gdpa_forward call, median of 20
+    CUDA-event-timed calls after 5 warm-ups, inputs (0.6 to 6 GB) larger than
+    L2.  Useful TFLOP/s, and algorithmic bytes over time as a fraction of the
+    measured HBM copy bandwidth and of the 8 TB/s spec."""
+    import torch
+
+    from pffn_attention_b200 import gdpa
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for cfg in (2, 3, 4):
+        w = make_workload(cfg, device=dev, seed=cfg, with_dout=False)
+        qo = torch.tensor(w.q_offsets, dtype=torch.int32, device=dev)
+        ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
+        kw = dict(phi=w.phi, scale=w.scale, window=(w.window_left, w.window_right),
+                  bias=w.bias, bias_kind=w.bias_kind, max_seqlen_q=w.max_q,
+                  max_seqlen_kv=w.max_kv, stream=stream)
+        torch.cuda.synchronize(dev)
+        o, lse, ws = gdpa.forward(w.q, w.k, w.v, qo, ko, **kw)
+        for _ in range(5):
+            gdpa.forward(w.q, w.k, w.v, qo, ko, out=o, lse=lse, workspace=ws, **kw)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(20)]
+        for e0, e1 in evs:
+            e0.record(stream)
+            gdpa.forward(w.q, w.k, w.v, qo, ko, out=o, lse=lse, workspace=ws, **kw)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if gdpa.device_status(ws, stream) != 0:
+            raise RuntimeError(f"device status after {w.name}")
+        ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+        fl, _ = useful_flops(w, False)
+        by, _ = algorithmic_bytes(w, False)
+        gbs = by / (ms * 1e-3) / 1e9
+        tf = fl / (ms * 1e-3) / 1e12
+        out[w.name] = {"B": w.B, "H": w.H, "D": w.D, "fwd_ms": round(ms, 4),
+                       "useful_tflops": round(tf, 1),
+                       "tensor_frac": round(tf / peaks["bf16_tflops"], 4),
+                       "algorithmic_gb": round(by / 1e9, 3), "achieved_gbs": round(gbs, 1),
+                       "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+                       "hbm_frac_spec": round(gbs / SPEC_HBM_GBS, 4), "bound": "hbm",
+                       "peak_source": peak_src, "timing": "median of 20 calls, 5 warm-ups"}
+        del w, o, lse, ws, qo, ko
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, w, p, qo, ko, training, dev, world):
@@ -732,6 +786,8 @@ def main(argv=None):
                     help="replace the workload's activation (diagnostics)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the forward-only workloads' per-workload timings")
     ap.add_argument("--grouped", action="store_true",
                     help="time the event-type problems as one grouped call vs separate calls")
     ap.add_argument("--rotary", action="store_true",

@@ -40,8 +40,9 @@
  * Errors: argument errors are reported at the call (GDPA_ERR_*), before
  * anything is launched.  Launch failures return GDPA_ERR_CUDA.  Errors found
  * by the device (a bounded wait that ran out, an offset beyond the declared
- * maximum length) are recorded in the workspace and read back with
- * gdpa_get_device_status.  Offsets contents are trusted beyond those checks.
+ * maximum length, offsets that decrease or reach past total_q / total_kv) are
+ * recorded in the workspace and read back with gdpa_get_device_status; the
+ * offending sample is skipped, so its output rows are not written.
  */
 #ifndef GDPA_H_
 #define GDPA_H_
@@ -68,7 +69,10 @@ typedef enum {
   GDPA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdpa_workspace_size */
   GDPA_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed */
   GDPA_ERR_TIMEOUT = 5,      /* device: a bounded wait inside a kernel ran out */
-  GDPA_ERR_DEVICE_CHECK = 6  /* device: a sample is longer than max_seqlen_q / _kv */
+  GDPA_ERR_DEVICE_CHECK = 6  /* device: a sample is longer than max_seqlen_q / _kv, or
+                                its offsets decrease or reach past total_q / total_kv;
+                                such a sample is skipped and its output rows are left
+                                unwritten */
 } gdpa_status_t;
 
 enum { GDPA_PHI_SILU = 0, GDPA_PHI_SOFTMAX = 1, GDPA_PHI_IDENTITY = 2, GDPA_PHI_GELU = 3 };
@@ -297,7 +301,12 @@ GDPA_API gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* proble
  * overlap on the GPU (on different streams, or from different host threads)
  * race and must be serialised by the caller.  Each call overwrites what it
  * needs, so nothing from an earlier call leaks in.  Device-side status of
- * these calls is not readable through gdpa_get_device_status.  With rotary
+ * these calls is not readable through gdpa_get_device_status: a bounded wait
+ * that runs out, or a sample that fails the device checks (see
+ * GDPA_ERR_DEVICE_CHECK), leaves the affected O and LSE rows unwritten while
+ * the call still returns GDPA_OK.  A caller that must detect this can fill O
+ * with a sentinel (NaN) before the call, or check the offsets on the host
+ * against max_seqlen_q / _kv and the totals.  With rotary
  * tables (rope_q / rope_kv) the attention kernel turns Q and K itself (as
  * debug_flags bit 2 selects for gdpa_forward): no turned copies, the same
  * results bit for bit. */

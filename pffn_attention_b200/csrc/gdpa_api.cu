@@ -114,6 +114,7 @@ WorkspaceLayout make_layout(const gdpa_params_t* p, int backward, int sms) {
   off += align256((size_t)(p->B + 1) * 4);
   L.info = off;
   off += align256((size_t)std::max(p->B, 1) * 16);
+  off = schedule_ws_bytes(p->B);  // the same end, by the rule that also sizes the no-alloc array
   if (backward) {
     L.delta = off;
     if (any_softmax(p)) off += align256((size_t)p->H * (size_t)p->total_q * 4);
@@ -328,7 +329,7 @@ const char* gdpa_status_string(gdpa_status_t s) {
     case GDPA_ERR_WORKSPACE: return "workspace missing or too small";
     case GDPA_ERR_CUDA: return "CUDA error";
     case GDPA_ERR_TIMEOUT: return "device wait timed out";
-    case GDPA_ERR_DEVICE_CHECK: return "sample longer than the declared maximum length";
+    case GDPA_ERR_DEVICE_CHECK: return "sample beyond the declared maximum length or the tensors";
   }
   return "unknown status";
 }
@@ -361,8 +362,8 @@ gdpa_status_t gdpa_tile_schedule(const gdpa_params_t* p, int block_m, int block_
   int sms = 0;
   if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, block_m, block_n, p->window_left,
-                                  p->window_right, tile_start, order, nullptr, 0, 0, nullptr,
-                                  (cudaStream_t)stream);
+                                  p->window_right, tile_start, order, nullptr, 0, 0, p->total_q,
+                                  p->total_kv, nullptr, (cudaStream_t)stream);
   return e == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
 
@@ -387,7 +388,7 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
 
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, block_n,
                                   p->window_left, p->window_right, tile_start, order, info,
-                                  eff_max_q(p), eff_max_kv(p), status, s);
+                                  eff_max_q(p), eff_max_kv(p), p->total_q, p->total_kv, status, s);
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
   if (p->B == 0 || p->total_q == 0) return GDPA_OK;
 
@@ -481,7 +482,7 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
 
   cudaError_t e = launch_schedule(q_offsets, kv_offsets, p->B, kBlockM, 128, p->window_left,
                                   p->window_right, tile_start, order, info, eff_max_q(p),
-                                  eff_max_kv(p), status, s);
+                                  eff_max_kv(p), p->total_q, p->total_kv, status, s);
   if (e != cudaSuccess) return GDPA_ERR_CUDA;
   if (dbias && p->total_kv > 0) {
     // the kernel adds each key's two column-half sums into it
@@ -655,6 +656,8 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
       sp[j].wr = p->window_right;
       sp[j].max_q = eff_max_q(p);
       sp[j].max_kv = eff_max_kv(p);
+      sp[j].total_q = p->total_q;
+      sp[j].total_kv = p->total_kv;
       ebase += p->B;
       timeouts[gi] = std::max(timeouts[gi], timeout_ns(p));
     }

@@ -149,6 +149,7 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
   uint32_t kvi = 0, qi = 0;
+  bool dropped = false;
   UnitStream units(a.info, a.H, a.n_units, a.head_mask);
   BUnit t;
   while (units.next(t)) {
@@ -187,6 +188,11 @@ __device__ void bwd_producer(const BwdArgs& a, const BSmem<C>& sm, const CUtenso
           if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((qi / C::NQ) & 1) ^ 1, abort, a.status,
                          a.timeout_ns, 0x1000 + C::B_QEMPTY + qs))
             return false;
+          if ((a.debug_flags & 1) && !dropped && blockIdx.x == 0) {
+            dropped = true;  // test hook: this Q/dO tile is never loaded
+            ++qi;
+            return true;
+          }
           mbar_arrive_expect_tx(sm.bar(C::B_QFULL + qs), 2 * C::QT_BYTES);
           for (int p = 0; p < C::NPANEL; ++p) {
             tma_load_3d(sm.q(qs) + p * C::BM * C::PANEL_BYTES, tq, sm.bar(C::B_QFULL + qs),

@@ -26,6 +26,15 @@ struct WorkspaceLayout {
   int grid;
 };
 
+constexpr size_t ws_align256(size_t x) { return (x + 255) & ~size_t(255); }
+// Bytes of the part every call's workspace starts with: the status block, the
+// sample order, the tile prefix and the per-sample descriptors for B samples.
+// This is the whole of a forward's workspace without rotary copies.
+constexpr size_t schedule_ws_bytes(int B) {
+  return 256 + ws_align256((size_t)(B > 1 ? B : 1) * 4) + ws_align256((size_t)(B + 1) * 4) +
+         ws_align256((size_t)(B > 1 ? B : 1) * 16);
+}
+
 // One forward problem's own data: every field a kernel role reads per unit.
 // A single-problem call carries it inline (FwdArgs::p0); a grouped call keeps
 // one per problem in device memory (FwdArgs::probs).
@@ -98,6 +107,7 @@ struct BwdArgs {
 struct GroupSchedProblem {
   const int32_t* q_offsets;
   const int32_t* kv_offsets;
+  int64_t total_q, total_kv;
   int B, ebase;
   int wl, wr;
   int max_q, max_kv;
@@ -115,8 +125,8 @@ struct GroupSchedJob {
 // Launchers (defined next to their kernels).
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
-                            int32_t* order, int4* info, int max_q, int max_kv,
-                            DeviceStatus* status, cudaStream_t stream);
+                            int32_t* order, int4* info, int max_q, int max_kv, int64_t total_q,
+                            int64_t total_kv, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,

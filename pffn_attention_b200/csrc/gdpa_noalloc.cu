@@ -24,15 +24,12 @@
 
 namespace {
 
-// status (256 B) + order[16384] (64 KiB) + tile_start[16385] + info[16384]
-// (16 B each), each rounded up to 256 B: enough for the largest batch the
-// library accepts.
-constexpr int kNoAllocMaxBatch = 16384;
-constexpr size_t kRound = 256;
-constexpr size_t kNoAllocBytes =
-    256 + ((kNoAllocMaxBatch * 4 + kRound - 1) / kRound) * kRound +
-    (((kNoAllocMaxBatch + 1) * 4 + kRound - 1) / kRound) * kRound +
-    ((kNoAllocMaxBatch * 16 + kRound - 1) / kRound) * kRound;
+// status (256 B) + order[B] + tile_start[B+1] + info[B] (16 B each), each
+// rounded up to 256 B, for the largest batch the library accepts:
+// 393,728 bytes.
+constexpr int kNoAllocMaxBatch = gdpa::kMaxSortBatch;
+constexpr size_t kNoAllocBytes = gdpa::schedule_ws_bytes(kNoAllocMaxBatch);
+static_assert(kNoAllocBytes == 393728, "documented size of the fixed scratch array");
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 

@@ -38,11 +38,37 @@ __device__ __forceinline__ unsigned long long sample_cost(int Lq, int Lk, int BM
   return cost;
 }
 
+// Sample b's rows.  With check set, a sample whose lengths exceed the
+// declared maxima, whose offsets decrease, or whose rows reach past the
+// tensors (offsets beyond total_q / total_kv) gets zero lengths and true is
+// returned: the kernels then skip it instead of reading or writing outside
+// the caller's buffers.  Without check, only a negative length is clamped.
+__device__ __forceinline__ bool sample_lengths(const int32_t* __restrict__ q_offsets,
+                                               const int32_t* __restrict__ kv_offsets, int b,
+                                               bool check, int max_q, int max_kv,
+                                               int64_t total_q, int64_t total_kv, int& q0,
+                                               int& Lq, int& k0, int& Lk) {
+  q0 = q_offsets[b];
+  k0 = kv_offsets[b];
+  Lq = q_offsets[b + 1] - q0;
+  Lk = kv_offsets[b + 1] - k0;
+  bool bad = Lq < 0 || Lk < 0;
+  if (check)
+    bad = bad || Lq > max_q || Lk > max_kv || q0 < 0 || k0 < 0 ||
+          (int64_t)q0 + Lq > total_q || (int64_t)k0 + Lk > total_kv;
+  if (bad) {
+    Lq = 0;
+    Lk = 0;
+  }
+  return bad;
+}
+
 __global__ void __launch_bounds__(kSchedThreads)
     gdpa_schedule_kernel(const int32_t* __restrict__ q_offsets,
                          const int32_t* __restrict__ kv_offsets, int B, int BM, int BN, int wl,
                          int wr, int32_t* __restrict__ tile_start, int32_t* __restrict__ order,
-                         int4* __restrict__ info, int max_q, int max_kv, DeviceStatus* status) {
+                         int4* __restrict__ info, int max_q, int max_kv, int64_t total_q,
+                         int64_t total_kv, DeviceStatus* status) {
   extern __shared__ unsigned long long keys[];
   __shared__ long long warp_tot[kSchedThreads / 32];
   const int tid = threadIdx.x;
@@ -57,8 +83,9 @@ __global__ void __launch_bounds__(kSchedThreads)
   for (int i = tid; i < n; i += kSchedThreads) {
     unsigned long long key = ~0ull;
     if (i < B) {
-      const int Lq = q_offsets[i + 1] - q_offsets[i];
-      const int Lk = kv_offsets[i + 1] - kv_offsets[i];
+      int q0, Lq, k0, Lk;
+      sample_lengths(q_offsets, kv_offsets, i, info != nullptr, max_q, max_kv, total_q, total_kv,
+                     q0, Lq, k0, Lk);
       unsigned long long c = sample_cost(Lq, Lk, BM, BN, wl, wr);
       if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
       key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
@@ -89,14 +116,14 @@ __global__ void __launch_bounds__(kSchedThreads)
   for (int p = beg; p < end; ++p) {
     const int b = (int)(keys[p] & 0xFFFFFFFFull);
     order[p] = b;
-    const int q0 = q_offsets[b], Lq = q_offsets[b + 1] - q0;
-    const int k0 = kv_offsets[b], Lk = kv_offsets[b + 1] - k0;
+    int q0, Lq, k0, Lk;
+    const bool bad = sample_lengths(q_offsets, kv_offsets, b, info != nullptr, max_q, max_kv,
+                                    total_q, total_kv, q0, Lq, k0, Lk);
     local += (Lq + BM - 1) / BM;
     if (info) {
-      // a sample longer than the declared bound is reported and skipped
-      const bool bad = Lq > max_q || Lk > max_kv;
+      // a sample outside the declared bounds is reported and skipped
       if (bad && status) record_error(status, 6, b);
-      info[p] = make_int4(q0, bad ? 0 : Lq, k0, bad ? 0 : Lk);
+      info[p] = make_int4(q0, Lq, k0, Lk);
     }
   }
   // block-wide exclusive scan of `local`
@@ -121,8 +148,9 @@ __global__ void __launch_bounds__(kSchedThreads)
   long long run = warp_tot[warp] + incl - local;
   for (int p = beg; p < end; ++p) {
     tile_start[p] = (int32_t)run;
-    const int b = order[p];
-    const int Lq = q_offsets[b + 1] - q_offsets[b];
+    int q0, Lq, k0, Lk;
+    sample_lengths(q_offsets, kv_offsets, order[p], info != nullptr, max_q, max_kv, total_q,
+                   total_kv, q0, Lq, k0, Lk);
     run += (Lq + BM - 1) / BM;
   }
   if (end == B && beg < end) tile_start[B] = (int32_t)run;
@@ -162,8 +190,9 @@ __global__ void __launch_bounds__(kSchedThreads)
     if (i < n_entries) {
       const GroupSchedProblem& P = sp[problem_of(i)];
       const int b = i - P.ebase;
-      const int Lq = P.q_offsets[b + 1] - P.q_offsets[b];
-      const int Lk = P.kv_offsets[b + 1] - P.kv_offsets[b];
+      int q0, Lq, k0, Lk;
+      sample_lengths(P.q_offsets, P.kv_offsets, b, true, P.max_q, P.max_kv, P.total_q,
+                     P.total_kv, q0, Lq, k0, Lk);
       unsigned long long c = sample_cost(Lq, Lk, BM, BN, P.wl, P.wr);
       if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
       key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
@@ -192,12 +221,12 @@ __global__ void __launch_bounds__(kSchedThreads)
     const int p = problem_of(e);
     const GroupSchedProblem& P = sp[p];
     const int b = e - P.ebase;
-    const int q0 = P.q_offsets[b], Lq = P.q_offsets[b + 1] - q0;
-    const int k0 = P.kv_offsets[b], Lk = P.kv_offsets[b + 1] - k0;
-    // a sample longer than its problem's declared bound is reported and skipped
-    const bool bad = Lq > P.max_q || Lk > P.max_kv;
+    int q0, Lq, k0, Lk;
+    // a sample outside its problem's declared bounds is reported and skipped
+    const bool bad = sample_lengths(P.q_offsets, P.kv_offsets, b, true, P.max_q, P.max_kv,
+                                    P.total_q, P.total_kv, q0, Lq, k0, Lk);
     if (bad && status) record_error(status, 6, e);
-    info[pos] = make_int4(q0, bad ? 0 : Lq, k0, bad ? 0 : Lk);
+    info[pos] = make_int4(q0, Lq, k0, Lk);
     eprob[pos] = p;
   }
 }
@@ -220,8 +249,8 @@ cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max
 
 cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets, int B,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
-                            int32_t* order, int4* info, int max_q, int max_kv,
-                            DeviceStatus* status, cudaStream_t stream) {
+                            int32_t* order, int4* info, int max_q, int max_kv, int64_t total_q,
+                            int64_t total_kv, DeviceStatus* status, cudaStream_t stream) {
   int n = 1;
   while (n < B) n <<= 1;
   const size_t smem = (size_t)n * sizeof(unsigned long long);
@@ -231,7 +260,8 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
   if (e != cudaSuccess) return e;
   gdpa_schedule_kernel<<<1, kSchedThreads, smem, stream>>>(q_offsets, kv_offsets, B, block_m,
                                                            block_n, wl, wr, tile_start, order,
-                                                           info, max_q, max_kv, status);
+                                                           info, max_q, max_kv, total_q, total_kv,
+                                                           status);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,10 @@
 """Device-side failure detection, without faulting the GPU.
 
 Every wait inside the kernels is bounded.  A debug flag drops one Q-tile load
-in CTA 0, so the MMA issuer's wait for it runs out after 20 ms; the kernel
-must record GDPA_ERR_TIMEOUT, leave cleanly, and leave the context usable.
+(forward) or one Q/dO-tile load (backward) in CTA 0, so the MMA issuer's wait
+for it runs out after 20 ms; the kernel must record GDPA_ERR_TIMEOUT, leave
+cleanly, and leave the context usable.  Malformed offsets are caught by the
+schedule and reported instead of being read or written past the tensors.
 """
 import pytest
 import torch
@@ -64,3 +66,56 @@ def test_sumkron_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     y, ws2 = cuda_lib.sumkron_forward(xd, ad, wd)
     assert cuda_lib.device_status(ws2) == 0
     compare("Y", y, sumkron.forward(x, a, w))
+
+
+@pytest.mark.parametrize("cfg", [2, 5])
+def test_backward_bounded_wait_reports_timeout_and_context_survives(cuda_lib, cfg):
+    w = make_workload(cfg, B=6, with_dout=True)
+    q, k, v, qo, ko = _args(w)
+    bias = w.bias.cuda() if w.bias is not None else None
+    dout = w.dout.cuda()
+    kw = dict(phi=w.phi, scale=w.scale, bias=bias, bias_kind=w.bias_kind,
+              max_seqlen_q=w.max_q, max_seqlen_kv=w.max_kv)
+    o, lse, ws = cuda_lib.forward(q, k, v, qo, ko, **kw)
+    assert cuda_lib.device_status(ws) == 0
+    p = cuda_lib.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale,
+                             bias_kind=w.bias_kind, max_seqlen_q=w.max_q,
+                             max_seqlen_kv=w.max_kv, debug_flags=1, wait_timeout_us=20000)
+    _, _, _, wsb = cuda_lib.backward(q, k, v, o, dout, lse, qo, ko, bias=bias, params=p)
+    assert cuda_lib.device_status(wsb) == 5  # GDPA_ERR_TIMEOUT
+    # the same context, a normal call afterwards
+    dq, dk, dv, wsb2 = cuda_lib.backward(q, k, v, o, dout, lse, qo, ko, **kw)
+    assert cuda_lib.device_status(wsb2) == 0
+    rdq, rdk, rdv, _ = oracle.backward_workload(w)
+    compare("dQ", dq, rdq)
+    compare("dK", dk, rdk)
+    compare("dV", dv, rdv)
+
+
+@pytest.mark.parametrize("which", ["decreasing", "past_total", "negative_start"])
+def test_malformed_offsets_are_reported_and_skipped(cuda_lib, which):
+    """Offsets that decrease, or that reach past total_q, must neither be read
+    nor written past the tensors: the schedule reports GDPA_ERR_DEVICE_CHECK and
+    skips the sample, and the other samples' rows are still exact."""
+    w = make_workload(2, B=4)
+    q, k, v, qo, ko = _args(w)
+    good = list(w.q_offsets)
+    bad = list(good)
+    if which == "decreasing":
+        bad[2] = bad[1] - 5          # sample 1 gets a negative length
+    elif which == "past_total":
+        bad[3] = int(w.total_q) + 7  # sample 2 ends past the tensor, sample 3 starts there
+    else:
+        bad[1] = -3                  # sample 0 has a negative length, sample 1 starts outside
+    qo_bad = torch.tensor(bad, dtype=torch.int32, device="cuda")
+    sentinel = float("nan")
+    o = torch.full_like(q, sentinel)
+    _, _, ws = cuda_lib.forward(q, k, v, qo_bad, ko, phi=w.phi, scale=w.scale,
+                                max_seqlen_q=0, max_seqlen_kv=0, out=o)
+    assert cuda_lib.device_status(ws) == 6  # GDPA_ERR_DEVICE_CHECK
+    ro, _ = oracle.forward_workload(w)
+    # samples whose offsets are intact still match the oracle
+    for b in range(w.B):
+        lo, hi = bad[b], bad[b + 1]
+        if lo == good[b] and hi == good[b + 1] and hi >= lo:
+            compare(f"O sample {b}", o[lo:hi], ro[lo:hi])
