@@ -123,6 +123,17 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register budget");
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Move a warpgroup from the launch's per-thread count FROM to N registers:
+// an increase for N > FROM, a release for N < FROM (a decrease may never name
+// a count above the current one, nor an increase one below it).
+template <int N, int FROM>
+__device__ __forceinline__ void setmaxnreg_to() {
+  if constexpr (N > FROM) {
+    setmaxnreg_inc<N>();
+  } else if constexpr (N < FROM) {
+    setmaxnreg_dec<N>();
+  }
+}
 
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
@@ -260,6 +271,22 @@ __device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 
+// tmem_ld32p for fp32 accumulators: the columns land as floats.
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]),
+        "=f"(r[7]), "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]),
+        "=f"(r[13]), "=f"(r[14]), "=f"(r[15]), "=f"(r[16]), "=f"(r[17]), "=f"(r[18]),
+        "=f"(r[19]), "=f"(r[20]), "=f"(r[21]), "=f"(r[22]), "=f"(r[23]), "=f"(r[24]),
+        "=f"(r[25]), "=f"(r[26]), "=f"(r[27]), "=f"(r[28]), "=f"(r[29]), "=f"(r[30]),
+        "=f"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 // 16 consecutive 32-bit columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -358,6 +385,35 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Two floats as an fp16 pair (round to nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// The fp16 pair back as an fp32 pair (exact).
+__device__ __forceinline__ uint64_t unpack_f16x2(uint32_t h) {
+  uint64_t r;
+  asm("{\n\t.reg .f16 a, b;\n\t.reg .f32 x, y;\n\t"
+      "mov.b32 {a, b}, %1;\n\tcvt.f32.f16 x, a;\n\tcvt.f32.f16 y, b;\n\t"
+      "mov.b64 %0, {x, y};\n\t}"
+      : "=l"(r) : "r"(h));
+  return r;
+}
+// v[0..3] += p, kept in program order relative to the other volatile asm of
+// the thread (a TMEM load after it cannot be scheduled before it, which would
+// keep both the addends and the new values in registers at once).
+__device__ __forceinline__ void add4_ordered(float* v, float4 p) {
+  asm volatile("add.f32 %0, %0, %4;\n\tadd.f32 %1, %1, %5;\n\t"
+               "add.f32 %2, %2, %6;\n\tadd.f32 %3, %3, %7;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3])
+               : "f"(p.x), "f"(p.y), "f"(p.z), "f"(p.w));
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -379,6 +435,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Two floats as a bf16 pair, lo in the low half, rounded to nearest with ties
+// away from zero, using integer operations only (an add of half a bf16 ulp to
+// each bit pattern, then a byte permute), so it does not compete with ex2 for
+// the conversion unit.  Finite inputs only (the callers' values are finite).
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 // Global fp32x4 load / store with an L2 eviction-priority policy.
