@@ -9,26 +9,30 @@
 //
 // One persistent CTA per SM walks (sample, head) units in longest-first order
 // and, within a unit, its 128-row query tiles.  Tiles alternate between two
-// slots, each with its own phi warpgroup, Q buffer and TMEM (S of one 128-key
-// block and the O accumulator: 2 x 256 columns), so one slot's MMAs run while
-// the other slot's phi warpgroup works.  P (bf16) goes back into TMEM over the
-// S columns it came from and is the A operand of the PV MMA.  K/V blocks come
-// through one ring shared by both slots; a unit without a band whose blocks
-// fit in the ring loads them once for all its tiles.  A tile only loads the
-// key blocks it can see (all of them, or the band of the sliding window,
-// Kunlun paper review §2.5).  128-key blocks keep the MMA count low: a
-// tcgen05.mma of 128 x N x 16 costs about the same for N = 64 and N = 128.
+// slots, each with its own phi warpgroup, epilogue warpgroup and TMEM (S of
+// one 128-key block and the O accumulator: 2 x 256 columns), so one slot's
+// MMAs run while the other slot's phi warpgroup works, and a tile's O is
+// written out while the slot's next tile is under way.  P (bf16) goes back
+// into TMEM over the S columns it came from and is the A operand of the PV
+// MMA.  Q tiles come through a ring of stages; K/V blocks through one ring
+// shared by both slots; a unit without a band whose blocks fit in the ring
+// loads them once for all its tiles.  A tile only loads the key blocks it can
+// see (all of them, or the band of the sliding window, Kunlun paper review
+// §2.5).  128-key blocks keep the MMA count low: a tcgen05.mma of 128 x N x 16
+// costs about the same for N = 64 and N = 128.
 //
-// Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles, K/V blocks (tile order)
-//   warp 1      MMA issuer (one thread), event driven over both slots:
-//               S = Q K^T into the slot's free S buffer, O += P V
-//   warp 2      TMEM allocator; bias warp of slot 0
-//   warp 3      bias warp of slot 1: beta of each key block (log sigma(G))
-//   warps 4-7   phi / epilogue warpgroup of slot 0, warps 8-11 of slot 1: one
-//               thread per query row; reads S from TMEM, applies the mask and
-//               phi, writes P to TMEM, rescales O when the running max moves,
-//               and writes O (bf16) and LSE at the end of the tile.
+// Warp roles (640 threads):
+//   warp 0       TMA producer: Q tiles, K/V blocks (tile order)
+//   warp 1       MMA issuer (one thread), event driven over both slots:
+//                S = Q K^T into the slot's S columns, O += P V
+//   warp 2       TMEM allocator; bias warp of slot 0
+//   warp 3       bias warp of slot 1: beta of each key block (log sigma(G))
+//   warps 4-7    phi warpgroup of slot 0, warps 8-11 of slot 1: one thread
+//                per query row; reads S from TMEM, applies the mask and phi,
+//                writes P to TMEM, rescales O when the running max moves,
+//                writes LSE at the end of the tile
+//   warps 12-15  epilogue warpgroup of slot 0, warps 16-19 of slot 1: O of
+//                each tile from TMEM, times 1/l, to bf16 in global memory
 // Every wait is bounded; on expiry the kernel records GDPA_ERR_TIMEOUT in the
 // workspace status, all roles leave their loops, TMEM is freed and the kernel
 // returns.
@@ -43,13 +47,21 @@
 namespace gdpa {
 namespace {
 
-constexpr int kThreads = 384;
-// keys per block: 128, or 64 when no sample has more than 64 keys (a 128-key
-// block would then be half masked, in the MMAs and in phi)
-constexpr int kRegsLaunch = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int kRegsControl = 104;  // warpgroup 0: producer, MMA issuer, allocator, bias
-constexpr int kRegsPhi = 200;      // the two phi warpgroups
-static_assert(128 * kRegsControl + 256 * kRegsPhi <= kThreads * kRegsLaunch,
+constexpr int kThreads = 640;
+constexpr int kRegsLaunch = 96;    // 65536 / 640 rounded down to a multiple of 8
+#ifndef GDPA_FWD_RC
+#define GDPA_FWD_RC 96
+#endif
+#ifndef GDPA_FWD_RP
+#define GDPA_FWD_RP 112
+#endif
+#ifndef GDPA_FWD_RE
+#define GDPA_FWD_RE 80
+#endif
+constexpr int kRegsControl = GDPA_FWD_RC;  // warpgroup 0: producer, MMA issuer, allocator, bias
+constexpr int kRegsPhi = GDPA_FWD_RP;      // warpgroups 1-2: phi of slot 0 / 1
+constexpr int kRegsEpi = GDPA_FWD_RE;      // warpgroups 3-4: O epilogue of slot 0 / 1
+static_assert(128 * kRegsControl + 256 * kRegsPhi + 256 * kRegsEpi <= kThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -71,20 +83,33 @@ struct FwdCfg {
   static constexpr uint32_t LAYOUT = D >= 64 ? LAYOUT_SW128 : LAYOUT_SW64;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;  // one K (or V) block
-  // K/V ring: up to 128 KB of stages (D = 128: 2 of 128 keys or 4 of 64), at most 8
-  static constexpr int NKV = (64 * 1024) / KV_BYTES > 8 ? 8 : (64 * 1024) / KV_BYTES;
-  static constexpr int STAGE_WARP = 32 * 128;  // O staging: 32 rows x 128 B per phi warp
-  static constexpr int OFF_Q = 0;                                // [2 slots]
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;              // [NKV]
+  // Q tiles come through a ring of NQ stages, so the producer loads a few tiles
+  // ahead of the MMAs (one load's latency no longer sits in every tile's
+  // chain): 4 stages for D <= 64, 2 (one per slot) for D = 128, where shared
+  // memory is full.
+  static constexpr int NQ = D >= 128 ? 2 : 4;
+  // K/V ring: 128 KB of stages for D = 128 (2 of 128 keys or 4 of 64), 64 KB
+  // for smaller D, at most 8
+  static constexpr int KV_RING = (D >= 128 ? 64 : 32) * 1024;
+  static constexpr int NKV = KV_RING / KV_BYTES > 8 ? 8 : KV_RING / KV_BYTES;
+  static constexpr int STAGE_WARP = 32 * 64;   // O staging: 32 rows x 64 B per epilogue warp
+  static constexpr int OFF_Q = 0;                                // [NQ]
+  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;             // [NKV]
   static constexpr int OFF_V = OFF_K + NKV * KV_BYTES;           // [NKV]
-  static constexpr int OFF_STAGE = OFF_V + NKV * KV_BYTES;       // [8 phi warps]
-  static constexpr int OFF_BIAS = OFF_STAGE + 8 * STAGE_WARP;    // float [2 slots][2][BN]
-  static constexpr int OFF_KVCNT = OFF_BIAS + 2 * 2 * BN * 4;    // int [3][8]
-  static constexpr int OFF_BAR = OFF_KVCNT + 3 * 8 * 4;
-  // barrier indices (per slot s: [s]; bias buffers of slot s: [2s + b])
+  static constexpr int OFF_STAGE = OFF_V + NKV * KV_BYTES;       // [8 epilogue warps]
+  static constexpr int OFF_INV = OFF_STAGE + 8 * STAGE_WARP;     // float [2 slots][2][BM]
+  static constexpr int OFF_BIAS = OFF_INV + 2 * 2 * BM * 4;      // float [2 slots][2][BN]
+  static constexpr int OFF_KVCNT = OFF_BIAS + 2 * 2 * BN * 4;    // int [4][8]
+  // tile records, producer -> other roles: a ring of NT (even, so a ring
+  // entry always holds tiles of the same slot)
+  static constexpr int NT = 16;
+  static constexpr int OFF_TREC = OFF_KVCNT + 4 * 8 * 4;         // FTile [NT]
+  static constexpr int OFF_BAR = OFF_TREC + NT * 64;
+  // barrier indices (Q ring stage i: [i]; per slot s: [s]; bias buffers of
+  // slot s: [2s + b])
   static constexpr int B_QFULL = 0;
-  static constexpr int B_QEMPTY = B_QFULL + 2;
-  static constexpr int B_KVFULL = B_QEMPTY + 2;
+  static constexpr int B_QEMPTY = B_QFULL + NQ;
+  static constexpr int B_KVFULL = B_QEMPTY + NQ;
   static constexpr int B_KVEMPTY = B_KVFULL + NKV;
   static constexpr int B_SFULL = B_KVEMPTY + NKV;
   static constexpr int B_PFULL = B_SFULL + 2;
@@ -96,7 +121,13 @@ struct FwdCfg {
   // rotary: Q of slot s, K of ring stage i turned and ready for the MMA
   static constexpr int B_QROT = B_BEMPTY + 4;
   static constexpr int B_KROT = B_QROT + 2;
-  static constexpr int NBARS = B_KROT + NKV;
+  // softmax row scales 1/l of a tile, phi -> epilogue (slot s, buffer b: [2s + b])
+  static constexpr int B_LFULL = B_KROT + NKV;
+  static constexpr int B_LEMPTY = B_LFULL + 4;
+  // tile record ring entry i written / read by all its readers
+  static constexpr int B_TFULL = B_LEMPTY + 4;
+  static constexpr int B_TEMPTY = B_TFULL + NT;
+  static constexpr int NBARS = B_TEMPTY + NT;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem addr, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES;  // base is 1024-aligned (checked at entry)
@@ -107,6 +138,7 @@ struct FwdCfg {
   static constexpr int TMEM_COLS = 512;
   static_assert(BN + D <= TMEM_SLOT, "TMEM slot");
   static_assert(NKV >= 2 && NKV <= 8, "K/V ring");
+  static_assert(NQ >= 2 && NQ <= 8, "Q ring");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "align");
 };
@@ -135,17 +167,21 @@ __device__ __forceinline__ void kv_range(int m0, int Lk, int wl, int wr, int& kb
   }
 }
 
-// One query tile of the CTA's walk.
-struct FTile {
-  int h, q0, Lq, k0, Lk;
-  int m0, kb0, kb1;     // first local row; visible key blocks [kb0, kb1)
-  int ntile;            // query tiles of the unit
-  uint32_t kv0;         // K/V ring index of block kb0 (the tile's blocks are consecutive)
-  bool resident;        // the unit's blocks are loaded once, at its first tile
-  bool unit_first;      // first tile of its unit
-  int slot;             // 0 or 1: tiles alternate between the two slots
-  int prob;             // its problem (grouped launch; 0 otherwise)
+// One query tile of the CTA's walk (64 bytes: the record the producer
+// publishes to the other roles in shared memory).
+struct __align__(16) FTile {
+  int h, q0, Lq, k0;
+  int Lk, m0, kb0, kb1;  // first local row; visible key blocks [kb0, kb1)
+  int ntile;             // query tiles of the unit
+  int prob;              // its problem (grouped launch; 0 otherwise)
+  int slot;              // 0 or 1: tiles alternate between the two slots
+  int resident;          // the unit's blocks are loaded once, at its first tile
+  int unit_first;        // first tile of its unit
+  int end;               // no tile: the walk is over
+  uint32_t kv0;          // K/V ring index of block kb0 (the tile's blocks are consecutive)
+  uint32_t qi;           // Q ring index: tiles with visible keys before this one
 };
+static_assert(sizeof(FTile) == 64, "tile record");
 
 // The CTA's tiles in the order every role uses.  Units come from UnitStream
 // (longest first, boustrophedon over the grid); K/V ring indices advance by
@@ -157,11 +193,11 @@ struct TileWalk {
   UnitStreamT<C::GROUPED> units;
   Unit t;
   int wl, wr, ntile, mt, nkb;
-  uint32_t g, kvi, unit_kv0;
+  uint32_t g, kvi, unit_kv0, nq;
   bool resident, in_unit;
   __device__ explicit TileWalk(const FwdArgs& a)
       : args(&a), units(a.info, a.H, a.n_units, a.head_mask, a.eprob, a.probs), t{},
-        wl(a.p0.wl), wr(a.p0.wr), ntile(0), mt(0), nkb(0), g(0), kvi(0), unit_kv0(0),
+        wl(a.p0.wl), wr(a.p0.wr), ntile(0), mt(0), nkb(0), g(0), kvi(0), unit_kv0(0), nq(0),
         resident(false), in_unit(false) {}
   __device__ bool next(FTile& x) {
     for (;;) {
@@ -191,8 +227,9 @@ struct TileWalk {
       x.m0 = mt * kBlockM;
       kv_range<C::BN>(x.m0, t.Lk, wl, wr, x.kb0, x.kb1);
       x.ntile = ntile;
-      x.resident = resident;
-      x.unit_first = mt == 0;
+      x.resident = resident ? 1 : 0;
+      x.unit_first = mt == 0 ? 1 : 0;
+      x.end = 0;
       if (resident) {
         x.kv0 = unit_kv0 + x.kb0;
       } else {
@@ -201,16 +238,12 @@ struct TileWalk {
       }
       x.slot = (int)(g & 1);
       x.prob = t.prob;
+      x.qi = nq;
+      if (x.kb1 > x.kb0) ++nq;  // only tiles with keys load a Q tile
       ++g;
       ++mt;
       return true;
     }
-  }
-  // next tile of slot s
-  __device__ bool next_slot(FTile& x, int s) {
-    while (next(x))
-      if (x.slot == s) return true;
-    return false;
   }
 };
 
@@ -218,13 +251,17 @@ template <class C>
 struct Smem {
   uint32_t base;  // shared address of the 1024-aligned base
   uint8_t* ptr;
-  __device__ uint32_t q(int s) const { return base + C::OFF_Q + s * C::Q_BYTES; }
+  __device__ uint32_t q(int st) const { return base + C::OFF_Q + st * C::Q_BYTES; }
   __device__ uint32_t k(int st) const { return base + C::OFF_K + st * C::KV_BYTES; }
   __device__ uint32_t v(int st) const { return base + C::OFF_V + st * C::KV_BYTES; }
-  // O staging of phi warp pw (0..7), row j (0..31), 16-byte chunk c of a
-  // 128-byte row segment, chunks XOR-swizzled by row (mask m)
-  __device__ uint32_t stage(int pw, int j, int c, int m) const {
-    return base + C::OFF_STAGE + pw * C::STAGE_WARP + j * 128 + ((c ^ (j & m)) << 4);
+  // O staging of epilogue warp ew (0..7), row j (0..31), 16-byte chunk c of a
+  // 64-byte row segment, chunks XOR-swizzled by row
+  __device__ uint32_t stage(int ew, int j, int c) const {
+    return base + C::OFF_STAGE + ew * C::STAGE_WARP + j * 64 + ((c ^ ((j >> 1) & 3)) << 4);
+  }
+  // softmax row scales 1/l of slot s, buffer b
+  __device__ float* inv(int s, int b) const {
+    return reinterpret_cast<float*>(ptr + C::OFF_INV) + (s * 2 + b) * C::BM;
   }
   __device__ float* bias(int s, int b) const {
     return reinterpret_cast<float*>(ptr + C::OFF_BIAS) + (s * 2 + b) * C::BN;
@@ -238,10 +275,62 @@ struct Smem {
   __device__ volatile int* kv_tag() const {
     return reinterpret_cast<volatile int*>(ptr + C::OFF_KVCNT) + 2 * 8;
   }
+  // per Q ring stage: the Q ring index the producer is loading into it
+  __device__ volatile int* q_tag() const {
+    return reinterpret_cast<volatile int*>(ptr + C::OFF_KVCNT) + 3 * 8;
+  }
+  __device__ uint32_t trec(int i) const { return base + C::OFF_TREC + i * 64; }
   __device__ uint32_t bar(int i) const { return base + C::OFF_BAR + i * 8; }
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(ptr + C::OFF_MISC); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(ptr + C::OFF_MISC + 4);
+  }
+};
+
+// Readers of tile record i (ring entry i % NT, of slot i % 2): the MMA issuer,
+// the slot's phi and epilogue warps and its side warps (the bias warp of the
+// slot, or both rotary warps).
+template <class C>
+__device__ __forceinline__ int trec_readers(const FwdArgs& a) {
+  const int side = C::ROPE ? 2 : ((C::GROUPED || a.p0.bias_kind != 0) ? 1 : 0);
+  return 1 + 4 + 4 + side;
+}
+
+// Reader of the producer's tile records: records first, first + step, ... (a
+// reader of one slot steps by 2).  Each record is copied out and released at
+// once: by the calling thread, or, for a warp reading together (WARP), by
+// lane 0 after the whole warp has copied it.
+template <class C, bool WARP>
+struct TileRing {
+  uint32_t i;
+  int step;
+  __device__ TileRing(int first, int step_) : i((uint32_t)first), step(step_) {}
+  __device__ __forceinline__ void take(const Smem<C>& sm, FTile& x) {
+    const int e = (int)(i % C::NT);
+    uint4* d = reinterpret_cast<uint4*>(&x);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) d[k] = ld_shared_v4(sm.trec(e) + 16 * k);
+    if (WARP) __syncwarp();
+    if (!WARP || (threadIdx.x & 31) == 0) mbar_arrive(sm.bar(C::B_TEMPTY + e));
+    i += (uint32_t)step;
+  }
+  // Blocking (bounded) read of the next record; false at the end of the walk
+  // or when the wait gave up.
+  __device__ bool next(const FwdArgs& a, const Smem<C>& sm, FTile& x) {
+    const int e = (int)(i % C::NT);
+    bool ok = mbar_wait(sm.bar(C::B_TFULL + e), (i / C::NT) & 1, sm.abort_flag(), a.status,
+                        a.timeout_ns, 0x700 + e);
+    if (WARP) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    take(sm, x);
+    return !x.end;
+  }
+  // Non-blocking: the next record, if the producer has written it.
+  __device__ bool poll(const Smem<C>& sm, FTile& x) {
+    const int e = (int)(i % C::NT);
+    if (!mbar_test_wait(sm.bar(C::B_TFULL + e), (i / C::NT) & 1)) return false;
+    take(sm, x);
+    return true;
   }
 };
 
@@ -256,7 +345,6 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   volatile int* abort = sm.abort_flag();
   const uint64_t pol_stream = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_last();
-  uint32_t nq[2] = {0u, 0u};
   bool dropped = false;
   TileWalk<C> walk(a);
   FTile x{};
@@ -282,22 +370,41 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
     }
     return true;
   };
+  // publish tile record g to the other roles (the ring entry is free once
+  // every reader of its previous record has copied it)
+  uint32_t g = 0;
+  auto publish = [&](const FTile& t) -> bool {
+    const int e = (int)(g % C::NT);
+    if (!mbar_wait(sm.bar(C::B_TEMPTY + e), ((g / C::NT) & 1) ^ 1, abort, a.status,
+                   a.timeout_ns, 0x000 + C::B_TEMPTY + e))
+      return false;
+    const uint4* src = reinterpret_cast<const uint4*>(&t);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 v = src[k];
+      st_shared_v4(sm.trec(e) + 16 * k, v.x, v.y, v.z, v.w);
+    }
+    mbar_arrive(sm.bar(C::B_TFULL + e));  // release: the record is visible to the waiters
+    ++g;
+    return true;
+  };
   while (walk.next(x)) {
-    if (x.kb1 <= x.kb0) continue;  // no visible keys: the phi warpgroup writes zeros
-    const int s = x.slot;
-    if (!mbar_wait(sm.bar(C::B_QEMPTY + s), (nq[s] & 1) ^ 1, abort, a.status, a.timeout_ns,
-                   0x000 + C::B_QEMPTY + s))
+    if (!publish(x)) return;
+    if (x.kb1 <= x.kb0) continue;  // no visible keys: the epilogue warpgroup writes zeros
+    const int qs = (int)(x.qi % C::NQ);
+    if (!mbar_wait(sm.bar(C::B_QEMPTY + qs), ((x.qi / C::NQ) & 1) ^ 1, abort, a.status,
+                   a.timeout_ns, 0x000 + C::B_QEMPTY + qs))
       return;
+    sm.q_tag()[qs] = (int)x.qi;  // published by the arrive below (release)
     if ((a.debug_flags & 1) && !dropped && blockIdx.x == 0) {
       dropped = true;  // test hook: this Q tile is never loaded
     } else {
-      mbar_arrive_expect_tx(sm.bar(C::B_QFULL + s), C::Q_BYTES);
+      mbar_arrive_expect_tx(sm.bar(C::B_QFULL + qs), C::Q_BYTES);
       const CUtensorMap* mq = map_of(x.prob, 0);
       for (int pnl = 0; pnl < C::NPANEL; ++pnl)
-        tma_load_3d(sm.q(s) + pnl * kBlockM * C::PANEL_BYTES, mq, sm.bar(C::B_QFULL + s),
+        tma_load_3d(sm.q(qs) + pnl * kBlockM * C::PANEL_BYTES, mq, sm.bar(C::B_QFULL + qs),
                     pnl * C::PANEL_ELEMS, x.h, x.q0 + x.m0, pol_stream);
     }
-    ++nq[s];
     if (x.resident && !x.unit_first) continue;  // the unit's blocks are in the ring
     if (x.unit_first) {
       // warm L2 with the next unit's first blocks (its loads wait for ring stages)
@@ -316,6 +423,10 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
     for (int kb = x.kb0; kb < x.kb1; ++kb)
       if (!load_kv(x.kv0 + (uint32_t)(kb - x.kb0), kb)) return;
   }
+  // one end record per slot
+  FTile last{};
+  last.end = 1;
+  if (publish(last)) publish(last);
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -349,51 +460,65 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   }
 
   struct Slot {
+    uint32_t qi;          // Q ring index of the tile
     uint32_t kv0;         // ring index of the tile's first block
     int nkv, ntile;       // blocks of the tile; tiles of its unit
-    bool resident, have;
+    int resident;
+    bool have, done;      // a tile in hand; the slot's walk is over
     int ns, npv;          // S and PV issued for the tile
     uint32_t pc, tq;      // PV and non-empty tile counts of the slot
   };
   Slot sl[2];
-  TileWalk<C> walk0(a), walk1(a);
-  auto advance = [&](Slot& z, TileWalk<C>& w, int s) {
+  // each slot's tiles from the producer's records (every other record); tiles
+  // without visible keys are skipped.  Polled, never waited on: the producer
+  // may itself wait for a Q stage that only the other slot's S MMA frees.
+  TileRing<C, false> ring0(0, 2), ring1(1, 2);
+  auto fetch = [&](Slot& z, TileRing<C, false>& rg) -> bool {
     FTile x;
-    z.have = false;
-    while (w.next_slot(x, s)) {
-      if (x.kb1 > x.kb0) {
+    while (!z.have && !z.done && rg.poll(sm, x)) {
+      if (x.end) {
+        z.done = true;
+      } else if (x.kb1 > x.kb0) {
         z.have = true;
+        z.qi = x.qi;
         z.kv0 = x.kv0;
         z.nkv = x.kb1 - x.kb0;
         z.ntile = x.ntile;
         z.resident = x.resident;
-        break;
+        z.ns = z.npv = 0;
+        return true;
       }
     }
-    z.ns = z.npv = 0;
+    return false;
   };
-  sl[0].pc = sl[0].tq = 0;
-  sl[1].pc = sl[1].tq = 0;
-  advance(sl[0], walk0, 0);
-  advance(sl[1], walk1, 1);
+  for (int s = 0; s < 2; ++s) {
+    sl[s].pc = sl[s].tq = 0;
+    sl[s].have = sl[s].done = false;
+  }
 
   uint64_t idle_since = 0;
   uint32_t idle_polls = 0;
-  while (sl[0].have || sl[1].have) {
+  while (!(sl[0].done && sl[1].done)) {
     bool progress = false;
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       Slot& z = sl[s];
-      if (!z.have) continue;
+      if (!z.have && !fetch(z, s == 0 ? ring0 : ring1)) continue;
       const uint32_t tslot = tmem + s * C::TMEM_SLOT;
       // ---- S = Q K^T of block ns
       if (z.ns < z.nkv && z.ns == z.npv) {
         const uint32_t ring = z.kv0 + (uint32_t)z.ns;
         const int st = (int)(ring % C::NKV);
-        // Q and K are ready once loaded, or once turned when rotary
-        constexpr int QREADY = C::ROPE ? C::B_QROT : C::B_QFULL;
+        // Q and K are ready once loaded, or once turned when rotary (the
+        // turning warps arrive per slot, in the slot's tile order).  Like a K/V
+        // stage, a Q stage's full barrier identifies this tile's phase only
+        // once the producer has started loading it.
         constexpr int KREADY = C::ROPE ? C::B_KROT : C::B_KVFULL;
-        bool ok = z.ns > 0 || mbar_test_wait(sm.bar(QREADY + s), z.tq & 1);
+        const int qst = (int)(z.qi % C::NQ);
+        bool ok = z.ns > 0 ||
+                  (C::ROPE ? mbar_test_wait(sm.bar(C::B_QROT + s), z.tq & 1)
+                           : (sm.q_tag()[qst] == (int)z.qi &&
+                              mbar_test_wait(sm.bar(C::B_QFULL + qst), (z.qi / C::NQ) & 1)));
         // The other slot may be far ahead or behind in the ring: the stage's
         // full barrier identifies this ring index's phase only once the
         // producer has started loading it (the previous content's phase done).
@@ -402,7 +527,7 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
         ok = ok && (z.pc == 0 || mbar_test_wait(sm.bar(C::B_PVDONE + s), (z.pc - 1) & 1));
         if (ok) {
           tc_fence_after();
-          const uint64_t qd = qdesc0 + (uint64_t)((s * C::Q_BYTES) >> 4);
+          const uint64_t qd = qdesc0 + (uint64_t)((qst * C::Q_BYTES) >> 4);
           const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < C::D / 16; ++kk) {
@@ -415,7 +540,7 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
                         kk > 0 ? 1u : 0u);
           }
           mma_commit(sm.bar(C::B_SFULL + s));
-          if (z.ns == z.nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + s));
+          if (z.ns == z.nkv - 1) mma_commit(sm.bar(C::B_QEMPTY + qst));
           ++z.ns;
           progress = true;
         }
@@ -448,7 +573,7 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
           if (z.npv == z.nkv) {
             mma_commit(sm.bar(C::B_OFULL + s));
             ++z.tq;
-            advance(z, s == 0 ? walk0 : walk1, s);
+            z.have = false;
           }
           progress = true;
         }
@@ -480,9 +605,9 @@ __device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, int s, bool softm
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
   uint32_t bc = 0;
-  TileWalk<C> walk(a);
+  TileRing<C, true> ring(s, 2);
   FTile x{};
-  while (walk.next_slot(x, s)) {
+  while (ring.next(a, sm, x)) {
     const FwdProblem P = fwd_problem<C>(a, x.prob);
     if (P.bias_kind == 0) continue;  // the phi warpgroup adds no bias for this tile
     for (int j = x.kb0; j < x.kb1; ++j) {
@@ -572,23 +697,24 @@ __device__ void role_rotary(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
   const int w = (threadIdx.x >> 5) - 2;  // 0 or 1
   const int lane = threadIdx.x & 31;
   const bool has_bias = a.p0.bias_kind != 0;
-  uint32_t nq[2] = {0u, 0u}, bc[2] = {0u, 0u};
-  TileWalk<C> walk(a);
+  uint32_t bc[2] = {0u, 0u};
+  TileRing<C, true> ring(0, 1);
   FTile x{};
 #define ROT_WAIT(bar_, par_, where_)                                                   \
   do {                                                                               \
     bool ok_ = mbar_wait(sm.bar(bar_), (par_), abort, a.status, a.timeout_ns, where_); \
     if (!__all_sync(0xffffffffu, ok_)) return;                                       \
   } while (0)
-  while (walk.next(x)) {
-    if (x.kb1 <= x.kb0) continue;  // nothing loaded: the phi warpgroup writes zeros
+  while (ring.next(a, sm, x)) {
+    if (x.kb1 <= x.kb0) continue;  // nothing loaded: the epilogue warpgroup writes zeros
     const int s = x.slot;
-    ROT_WAIT(C::B_QFULL + s, nq[s] & 1, 0x500 + C::B_QFULL + s);
-    rotate_tile<C>(sm.q(s), kBlockM, w * (kBlockM / 2), (w + 1) * (kBlockM / 2), x.Lq - x.m0,
+    // tiles are turned in load order, so this wait identifies the tile's phase
+    const int qs = (int)(x.qi % C::NQ);
+    ROT_WAIT(C::B_QFULL + qs, (x.qi / C::NQ) & 1, 0x500 + C::B_QFULL + qs);
+    rotate_tile<C>(sm.q(qs), kBlockM, w * (kBlockM / 2), (w + 1) * (kBlockM / 2), x.Lq - x.m0,
                    a.rope_q, (int64_t)x.q0 + x.m0, lane);
     fence_proxy_async_smem();  // the MMA reads the turned tile through the async proxy
     mbar_arrive(sm.bar(C::B_QROT + s));
-    ++nq[s];
     const bool loads = !(x.resident && !x.unit_first);
     for (int kb = x.kb0; kb < x.kb1; ++kb) {
       if (loads) {
@@ -623,16 +749,20 @@ __device__ void role_rotary(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
 }
 
 // ------------------------------------------------------------------ phi warpgroups
+// One warpgroup per slot; thread r owns row r of the slot's tiles.  Per key
+// block: x = scale s + beta from the S columns, P = phi(x) written back over
+// them as bf16 pairs (softmax: the block's row maximum first, O rescaled when
+// it grows).  At the end of a softmax tile the row's 1/l goes to the slot's
+// epilogue warpgroup through shared memory, and the LSE row is written here.
 template <class C, bool SOFTMAX>
 __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
   volatile int* abort = sm.abort_flag();
   const int warp = threadIdx.x >> 5;
   const int wq = warp & 3;                  // TMEM lane quarter of this warp
-  const int pw = warp - 4;                  // phi warp index: its O staging slice
   const int lane = threadIdx.x & 31;
   const int r = wq * 32 + lane;             // row of the tile owned by this thread
   const uint32_t tslot = tmem + ((uint32_t)(wq * 32) << 16) + s * C::TMEM_SLOT;
-  uint32_t nsb = 0, tq = 0, bc = 0;  // S blocks, non-empty tiles, bias blocks of the slot
+  uint32_t nsb = 0, bc = 0, lt = 0;  // S blocks, bias blocks, softmax tiles of the slot
 
 #define PHI_WAIT(bar_, par_, where_)                                                   \
   do {                                                                               \
@@ -640,32 +770,19 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
     if (!__all_sync(0xffffffffu, ok_)) return;                                       \
   } while (0)
 
-  TileWalk<C> walk(a);
+  TileRing<C, true> ring(s, 2);
   FTile x{};
-  while (walk.next_slot(x, s)) {
-    // this tile's problem: its outputs, scale, activation, bias and band
+  while (ring.next(a, sm, x)) {
+    const int nkv = x.kb1 - x.kb0;
+    if (nkv <= 0) continue;  // no visible keys: the epilogue warpgroup writes the tile
+    // this tile's problem: scale, activation, bias and band
     const FwdProblem P = fwd_problem<C>(a, x.prob);
-    __nv_bfloat16* const out = P.o;
-    float* const lse_out = P.lse;
-    const int Hp = P.H;
-    const int64_t tqp = P.total_q;
     const int wl = P.wl, wr = P.wr;
     const bool has_bias = P.bias_kind != 0;
     const bool identity = P.phi == 2;
     const bool gelu = P.phi == 3;
     const float sc = SOFTMAX ? P.scale * kLog2e : P.scale;
     const int row = x.m0 + r;
-    const bool row_ok = row < x.Lq;
-    const int nkv = x.kb1 - x.kb0;
-    if (nkv <= 0) {
-      if (row_ok) {
-        __nv_bfloat16* orow = out + ((int64_t)(x.q0 + row) * Hp + x.h) * C::D;
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
-        if (SOFTMAX && lse_out) lse_out[(int64_t)x.h * tqp + x.q0 + row] = -INFINITY;
-      }
-      continue;
-    }
     // visible keys of this row: [lo, hi]
     const int lo = wl >= 0 ? row - wl : INT_MIN;
     const int hi = min(x.Lk - 1, wr >= 0 ? row + wr : INT_MAX);
@@ -799,13 +916,13 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
         PHI_WAIT(C::B_PVDONE + s, (nsb - 1) & 1, 0x400 + C::B_PVDONE + s);
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < C::D / 16; ++c) {
+        for (int c = 0; c < C::D; c += 16) {
           uint32_t raw[16];
-          tmem_ld16(tslot + C::TMEM_O + c * 16, raw);
+          tmem_ld16(tslot + C::TMEM_O + c, raw);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * factor);
-          tmem_st16(tslot + C::TMEM_O + c * 16, raw);
+          tmem_st16(tslot + C::TMEM_O + c, raw);
         }
       }
       tmem_wait_st();
@@ -813,57 +930,105 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
       mbar_arrive(sm.bar(C::B_PFULL + s));
       ++nsb;
     }
-    // epilogue: O row from TMEM -> bf16 -> this warp's staging rows in shared
-    // memory -> 128-byte row segments to global memory, 64 columns per pass
-    PHI_WAIT(C::B_OFULL + s, tq & 1, 0x400 + C::B_OFULL + s);
-    tc_fence_after();
+    if (SOFTMAX) {
+      // 1/l of the row to the epilogue; the LSE row from here
+      const int b = lt & 1;
+      PHI_WAIT(C::B_LEMPTY + 2 * s + b, ((lt >> 1) & 1) ^ 1, 0x400 + C::B_LEMPTY + 2 * s + b);
+      sm.inv(s, b)[r] = l_run > 0.f ? 1.f / l_run : 0.f;
+      mbar_arrive(sm.bar(C::B_LFULL + 2 * s + b));
+      ++lt;
+      if (row < x.Lq && P.lse)
+        P.lse[(int64_t)x.h * P.total_q + x.q0 + row] =
+            l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+    }
+  }
+#undef PHI_WAIT
+}
+
+// ------------------------------------------------------------------ epilogue warpgroups
+// One warpgroup per slot: O of each tile from TMEM (released to the next
+// tile's PV as soon as it is read), times 1/l for softmax, to bf16, through
+// the warp's staging rows in shared memory to 64-byte row segments in global
+// memory, 32 columns per pass.  Tiles without visible keys get O = 0 (and LSE
+// = -inf) here.  Each warp handles its 32 rows on its own.
+template <class C, bool SOFTMAX>
+__device__ void role_epilogue(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
+  volatile int* abort = sm.abort_flag();
+  const int warp = threadIdx.x >> 5;
+  const int wq = warp & 3;                  // TMEM lane quarter of this warp
+  const int ew = warp - 12;                 // epilogue warp index: its staging slice
+  const int lane = threadIdx.x & 31;
+  const int r = wq * 32 + lane;
+  const uint32_t tO = tmem + ((uint32_t)(wq * 32) << 16) + s * C::TMEM_SLOT + C::TMEM_O;
+  uint32_t tq = 0, lt = 0;  // tiles with keys; softmax tiles (1/l buffers)
+
+#define EPI_WAIT(bar_, par_, where_)                                                   \
+  do {                                                                               \
+    bool ok_ = mbar_wait(sm.bar(bar_), (par_), abort, a.status, a.timeout_ns, where_); \
+    if (!__all_sync(0xffffffffu, ok_)) return;                                       \
+  } while (0)
+
+  TileRing<C, true> ring(s, 2);
+  FTile x{};
+  while (ring.next(a, sm, x)) {
+    const FwdProblem P = fwd_problem<C>(a, x.prob);
+    __nv_bfloat16* const out = P.o;
+    const int Hp = P.H;
+    const int row = x.m0 + r;
+    if (x.kb1 <= x.kb0) {
+      if (row < x.Lq) {
+        __nv_bfloat16* orow = out + ((int64_t)(x.q0 + row) * Hp + x.h) * C::D;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < C::D; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+        if (SOFTMAX && P.lse) P.lse[(int64_t)x.h * P.total_q + x.q0 + row] = -INFINITY;
+      }
+      continue;
+    }
     float inv = 1.f;
-    if (SOFTMAX) inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    constexpr int PW = C::D < 64 ? C::D : 64;  // columns per pass
-    constexpr int NPASS = C::D / PW;
-    constexpr int CPR = PW * 2 / 16;           // 16-byte chunks per row segment
-    constexpr int SWM = CPR - 1;
+    if (SOFTMAX) {
+      const int b = lt & 1;
+      EPI_WAIT(C::B_LFULL + 2 * s + b, (lt >> 1) & 1, 0x600 + C::B_LFULL + 2 * s + b);
+      inv = sm.inv(s, b)[r];
+      mbar_arrive(sm.bar(C::B_LEMPTY + 2 * s + b));
+      ++lt;
+    }
+    EPI_WAIT(C::B_OFULL + s, tq & 1, 0x600 + C::B_OFULL + s);
+    tc_fence_after();
+    constexpr int NPASS = C::D / 32;
 #pragma unroll 1
     for (int ps = 0; ps < NPASS; ++ps) {
 #pragma unroll
-      for (int c = 0; c < PW / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tslot + C::TMEM_O + ps * PW + c * 32, raw);
+      for (int hf = 0; hf < 2; ++hf) {  // 16 columns per TMEM load
+        uint32_t raw[16];
+        tmem_ld16(tO + ps * 32 + hf * 16, raw);
         tmem_wait_ld();
+        if (ps == NPASS - 1 && hf == 1) {  // O fully read: the slot's next tile may overwrite it
+          tc_fence_before();
+          mbar_arrive(sm.bar(C::B_OEMPTY + s));
+        }
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          const int cc = (c * 32 + e) / 8;  // 16-byte chunk of the row segment
-          st_shared_v4(sm.stage(pw, lane, cc, SWM),
+        for (int e = 0; e < 16; e += 8)
+          st_shared_v4(sm.stage(ew, lane, hf * 2 + (e >> 3)),
                        pack_bf16x2(__uint_as_float(raw[e + 0]) * inv, __uint_as_float(raw[e + 1]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 2]) * inv, __uint_as_float(raw[e + 3]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv));
-        }
-      }
-      if (ps == NPASS - 1) {  // O fully read: the slot's next tile may overwrite it
-        tc_fence_before();
-        mbar_arrive(sm.bar(C::B_OEMPTY + s));
       }
       __syncwarp();
-#pragma unroll 1
-      for (int it = 0; it < CPR; ++it) {
-        const int lin = it * 32 + lane;
-        const int j = lin / CPR, cc = lin % CPR;  // row of this warp, chunk
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int j = it * 8 + (lane >> 2), cc = lane & 3;  // row of this warp, chunk
         const int grow = x.m0 + wq * 32 + j;
-        const uint4 v = ld_shared_v4(sm.stage(pw, j, cc, SWM));
+        const uint4 v = ld_shared_v4(sm.stage(ew, j, cc));
         if (grow < x.Lq)
-          *reinterpret_cast<uint4*>(out + ((int64_t)(x.q0 + grow) * Hp + x.h) * C::D +
-                                    ps * PW + cc * 8) = v;
+          *reinterpret_cast<uint4*>(out + ((int64_t)(x.q0 + grow) * Hp + x.h) * C::D + ps * 32 +
+                                    cc * 8) = v;
       }
       __syncwarp();
     }
     ++tq;
-    if (SOFTMAX && row_ok && lse_out) {
-      lse_out[(int64_t)x.h * tqp + x.q0 + row] =
-          l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-    }
   }
-#undef PHI_WAIT
+#undef EPI_WAIT
 }
 
 template <int D, int BN, bool SOFTMAX, bool GROUPED, bool ROPE>
@@ -881,9 +1046,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(sm.bar(C::B_QFULL + i), 1);
+      mbar_init(sm.bar(C::B_QEMPTY + i), 1);
+      sm.q_tag()[i] = -1;
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(sm.bar(C::B_QFULL + s), 1);
-      mbar_init(sm.bar(C::B_QEMPTY + s), 1);
       mbar_init(sm.bar(C::B_SFULL + s), 1);
       mbar_init(sm.bar(C::B_PFULL + s), 128);
       mbar_init(sm.bar(C::B_PVDONE + s), 1);
@@ -897,6 +1065,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) {
       mbar_init(sm.bar(C::B_BFULL + i), C::ROPE ? 64 : 32);  // rotary: both warps write beta
       mbar_init(sm.bar(C::B_BEMPTY + i), 128);
+      mbar_init(sm.bar(C::B_LFULL + i), 128);
+      mbar_init(sm.bar(C::B_LEMPTY + i), 128);
+    }
+    for (int i = 0; i < C::NT; ++i) {
+      mbar_init(sm.bar(C::B_TFULL + i), 1);
+      mbar_init(sm.bar(C::B_TEMPTY + i), trec_readers<C>(a));
     }
     if (C::ROPE) {
       for (int s = 0; s < 2; ++s) mbar_init(sm.bar(C::B_QROT + s), 64);
@@ -920,10 +1094,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  // Registers: warpgroup 0 needs few, the phi warpgroups (a 128-column S row
-  // each) take the rest; each budget is set inside its own branch.
+  // Registers: the phi warpgroups take the most, the epilogue warpgroups the
+  // fewest; each budget is set inside its own branch.
   if (warp < 4) {
-    setmaxnreg_dec<kRegsControl>();
+    setmaxnreg_to<kRegsControl, kRegsLaunch>();
     if (warp == 0) {
       if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
     } else if (warp == 1) {
@@ -934,9 +1108,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // a grouped launch may mix problems with and without a bias
       if (C::GROUPED || a.p0.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
     }
-  } else {
-    setmaxnreg_inc<kRegsPhi>();
+  } else if (warp < 12) {
+    setmaxnreg_to<kRegsPhi, kRegsLaunch>();
     role_phi<C, SOFTMAX>(a, sm, tmem, (warp - 4) >> 2);
+  } else {
+    setmaxnreg_to<kRegsEpi, kRegsLaunch>();
+    role_epilogue<C, SOFTMAX>(a, sm, tmem, (warp - 12) >> 2);
   }
   __syncwarp();
   tc_fence_before();
@@ -961,13 +1138,16 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
                        const CUtensorMap& tv, int sms, cudaStream_t stream) {
   using C = FwdCfg<D, BN, GROUPED, ROPE>;
   auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED, ROPE>;
-  // the phi warpgroups raise their register budget with setmaxnreg, which waits
-  // until the block's launch registers cover it: never launch a build whose
-  // per-thread count would leave that wait unsatisfiable
+  // when the roles' register budgets differ, the raising side's setmaxnreg
+  // waits until the block's launch registers cover it: never launch a build
+  // whose per-thread count would leave that wait unsatisfiable
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  if (fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsPhi) return cudaErrorInvalidValue;
+  constexpr bool kSplit =
+      kRegsControl != kRegsLaunch || kRegsPhi != kRegsLaunch || kRegsEpi != kRegsLaunch;
+  if (kSplit && fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsPhi + 256 * kRegsEpi)
+    return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
