@@ -22,11 +22,13 @@
 // costs about the same for N = 64 and N = 128.
 //
 // Warp roles (640 threads):
-//   warp 0       TMA producer: Q tiles, K/V blocks (tile order)
-//   warp 1       MMA issuer (one thread), event driven over both slots:
+//   warp 0       TMA producer: Q tiles, K/V blocks (tile order); publishes
+//                each tile's record to the other roles
+//   warps 1, 3   MMA issuers (one thread each) of slot 0 and slot 1:
 //                S = Q K^T into the slot's S columns, O += P V
-//   warp 2       TMEM allocator; bias warp of slot 0
-//   warp 3       bias warp of slot 1: beta of each key block (log sigma(G))
+//   warp 2       TMEM allocator; bias warp: beta of each key block (log
+//                sigma(G)) for both slots
+//   (rotary: warp 1 issues for both slots, warps 2-3 turn Q and K)
 //   warps 4-7    phi warpgroup of slot 0, warps 8-11 of slot 1: one thread
 //                per query row; reads S from TMEM, applies the mask and phi,
 //                writes P to TMEM, rescales O when the running max moves,
@@ -74,6 +76,9 @@ struct FwdCfg {
   static constexpr int BN = BN_;
   static constexpr bool GROUPED = GROUPED_;  // units of several problems
   static constexpr bool ROPE = ROPE_;        // Q and K turned by the rotation tables
+  // one MMA issuer per slot (warps 1 and 3), or one for both when warps 2-3
+  // turn Q and K (rotary)
+  static constexpr bool DUAL = !ROPE_;
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
   // (64 B, 64-byte swizzle) when D = 32.
@@ -110,8 +115,9 @@ struct FwdCfg {
   static constexpr int B_QFULL = 0;
   static constexpr int B_QEMPTY = B_QFULL + NQ;
   static constexpr int B_KVFULL = B_QEMPTY + NQ;
+  // K/V stage i released by MMA issuer j: [2i + j] (one issuer: j = 0 only)
   static constexpr int B_KVEMPTY = B_KVFULL + NKV;
-  static constexpr int B_SFULL = B_KVEMPTY + NKV;
+  static constexpr int B_SFULL = B_KVEMPTY + 2 * NKV;
   static constexpr int B_PFULL = B_SFULL + 2;
   static constexpr int B_PVDONE = B_PFULL + 2;
   static constexpr int B_OFULL = B_PVDONE + 2;
@@ -287,13 +293,14 @@ struct Smem {
   }
 };
 
-// Readers of tile record i (ring entry i % NT, of slot i % 2): the MMA issuer,
-// the slot's phi and epilogue warps and its side warps (the bias warp of the
-// slot, or both rotary warps).
+// Readers of tile record i (ring entry i % NT, of slot i % 2): the MMA
+// issuer(s) (each reads every record), the slot's phi and epilogue warps, and
+// the side warps (the bias warp, or both rotary warps; each reads every
+// record).
 template <class C>
 __device__ __forceinline__ int trec_readers(const FwdArgs& a) {
   const int side = C::ROPE ? 2 : ((C::GROUPED || a.p0.bias_kind != 0) ? 1 : 0);
-  return 1 + 4 + 4 + side;
+  return (C::DUAL ? 2 : 1) + 4 + 4 + side;
 }
 
 // Reader of the producer's tile records: records first, first + step, ... (a
@@ -355,9 +362,10 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   };
   auto load_kv = [&](uint32_t ring, int kb) -> bool {
     const int st = (int)(ring % C::NKV);
-    if (!mbar_wait(sm.bar(C::B_KVEMPTY + st), ((ring / C::NKV) & 1) ^ 1, abort, a.status,
-                   a.timeout_ns, 0x000 + C::B_KVEMPTY + st))
-      return false;
+    for (int j = 0; j < (C::DUAL ? 2 : 1); ++j)
+      if (!mbar_wait(sm.bar(C::B_KVEMPTY + 2 * st + j), ((ring / C::NKV) & 1) ^ 1, abort,
+                     a.status, a.timeout_ns, 0x000 + C::B_KVEMPTY + 2 * st + j))
+        return false;
     sm.kv_tag()[st] = (int)ring;  // published by the arrive below (release)
     mbar_arrive_expect_tx(sm.bar(C::B_KVFULL + st), 2 * C::KV_BYTES);
     const CUtensorMap* mk = map_of(x.prob, 1);
@@ -429,9 +437,10 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   if (publish(last)) publish(last);
 }
 
-// ------------------------------------------------------------------ MMA issuer
-// Per slot: S of block i goes once the slot's previous PV has completed (P
-// lives in the S columns); PV of block i goes once the phi warpgroup has
+// ------------------------------------------------------------------ MMA issuers
+// One issuer for both slots (the rotary kernels, whose warps 2-3 turn Q and
+// K).  Per slot: S of block i goes once the slot's previous PV has completed
+// (P lives in the S columns); PV of block i goes once the phi warpgroup has
 // written P (and, for the tile's first block, the epilogue has read the
 // previous O).  The issuer polls both slots without blocking and issues
 // whatever is ready, so one slot's MMAs run while the other slot's phi works.
@@ -567,7 +576,7 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
             kv_ring[st] = (int)ring + 1;
             kv_left[st] = z.resident ? z.ntile : 1;
           }
-          if (--kv_left[st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + st));
+          if (--kv_left[st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + 2 * st));
           ++z.npv;
           ++z.pc;
           if (z.npv == z.nkv) {
@@ -598,19 +607,140 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   }
 }
 
-// ------------------------------------------------------------------ bias warps
-// beta of each key block a tile of slot s sees, into the slot's 2-buffer ring.
+// One slot's MMA issuer (warp 1 for slot 0, warp 3 for slot 1): S of block i,
+// then PV of block i once the phi warpgroup has written P, then S of block
+// i + 1 once that PV has completed (P lives in the S columns).  It waits on
+// its own slot's barriers only, so neither slot's MMAs wait for the other
+// slot's events.
+//
+// Each issuer reads every tile record, to release K/V stages: a stage use
+// (one ring index) is released by both issuers, each with a commit on its own
+// barrier after its last PV that reads it, or, when none of its tiles reads
+// it, as soon as the producer has taken the stage for it (a commit, which
+// still follows the issuer's earlier MMAs).  A resident unit's stages are
+// read by all its tiles, which alternate slots from the slot of its first
+// tile.
 template <class C>
-__device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, int s, bool softmax) {
+__device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
+  volatile int* abort = sm.abort_flag();
+  constexpr uint32_t idesc_s = make_idesc_bf16(kBlockM, C::BN, 0, 0);
+  constexpr uint32_t idesc_o = make_idesc_bf16(kBlockM, C::D, 0, 1);
+  constexpr uint32_t SBO = 8 * C::PANEL_BYTES;
+  const uint64_t qdesc0 = make_smem_desc(sm.q(0), 16, SBO, C::LAYOUT);
+  const uint64_t kdesc0 = make_smem_desc(sm.k(0), 16, SBO, C::LAYOUT);
+  const uint64_t vdesc0 = make_smem_desc(sm.v(0), C::BN * C::PANEL_BYTES, SBO, C::LAYOUT);
+  int* kv_left = sm.kv_count(s);  // this issuer's PVs still to read each stage
+  for (int i = 0; i < C::NKV; ++i) kv_left[i] = 0;
+  const uint32_t tslot = tmem + s * C::TMEM_SLOT;
+  uint32_t pc = 0, tq = 0;  // PVs and tiles of the slot
+
+#define MMA_WAIT(bar_, par_, where_)                                                    \
+  do {                                                                                \
+    if (!mbar_wait(sm.bar(bar_), (par_), abort, a.status, a.timeout_ns, where_)) return; \
+  } while (0)
+  // a stage's full barrier identifies this use's phase only once the producer
+  // has started loading it (its tag names the use)
+  auto wait_tag = [&](volatile int* tag, int want, int where) -> bool {
+    if (*tag == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (*tag != want) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        *abort = 1;
+        record_error(a.status, 5, where);
+        return false;
+      }
+      __nanosleep(32);
+    }
+    return true;
+  };
+
+  TileRing<C, false> ring(0, 1);
+  FTile x{};
+  while (ring.next(a, sm, x)) {
+    const int nb = x.kb1 - x.kb0;
+    if (nb <= 0) continue;
+    const bool mine = x.slot == s;
+    if (!x.resident || x.unit_first) {
+      // K/V stage uses that start at this tile: how many of this issuer's PVs
+      // read each (a streamed tile's uses, possibly more than the ring's
+      // stages, are each read by the tile's own PV, released right after it)
+      const int n_mine = x.resident ? (x.ntile + (x.slot == s ? 1 : 0)) / 2 : (mine ? 1 : 0);
+      for (int j = 0; j < nb && (x.resident || !mine); ++j) {
+        const int st = (int)((x.kv0 + (uint32_t)j) % C::NKV);
+        if (n_mine == 0) {
+          // not before the producer has taken the stage for this use: a
+          // release ahead of its wait would complete the phase it waits on
+          // for the next use
+          if (!wait_tag(sm.kv_tag() + st, (int)(x.kv0 + (uint32_t)j), 0x190 + st)) return;
+          mma_commit(sm.bar(C::B_KVEMPTY + 2 * st + s));
+        } else {
+          kv_left[st] = n_mine;
+        }
+      }
+    }
+    if (!mine) continue;
+    const int qst = (int)(x.qi % C::NQ);
+    for (int idx = 0; idx < nb; ++idx) {
+      const uint32_t ring_i = x.kv0 + (uint32_t)idx;
+      const int st = (int)(ring_i % C::NKV);
+      // ---- S = Q K^T
+      if (idx == 0) {
+        if (!wait_tag(sm.q_tag() + qst, (int)x.qi, 0x180 + qst)) return;
+        MMA_WAIT(C::B_QFULL + qst, (x.qi / C::NQ) & 1, 0x100 + C::B_QFULL + qst);
+      }
+      if (!wait_tag(sm.kv_tag() + st, (int)ring_i, 0x190 + st)) return;
+      MMA_WAIT(C::B_KVFULL + st, (ring_i / C::NKV) & 1, 0x100 + C::B_KVFULL + st);
+      if (pc > 0) MMA_WAIT(C::B_PVDONE + s, (pc - 1) & 1, 0x100 + C::B_PVDONE + s);
+      tc_fence_after();
+      const uint64_t qd = qdesc0 + (uint64_t)((qst * C::Q_BYTES) >> 4);
+      const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < C::D / 16; ++kk) {
+        const int pnl = kk * 16 / C::PANEL_ELEMS;
+        const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
+        mma_bf16_ss(tslot, desc_add(qd, (pnl * kBlockM * C::PANEL_BYTES + within) >> 4),
+                    desc_add(kd, (pnl * C::BN * C::PANEL_BYTES + within) >> 4), idesc_s,
+                    kk > 0 ? 1u : 0u);
+      }
+      mma_commit(sm.bar(C::B_SFULL + s));
+      if (idx == nb - 1) mma_commit(sm.bar(C::B_QEMPTY + qst));
+      // ---- O += P V
+      MMA_WAIT(C::B_PFULL + s, pc & 1, 0x100 + C::B_PFULL + s);
+      if (idx == 0) MMA_WAIT(C::B_OEMPTY + s, (tq & 1) ^ 1, 0x100 + C::B_OEMPTY + s);
+      tc_fence_after();
+      const uint64_t vd = vdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < C::BN / 16; ++kk)
+        mma_bf16_ts(tslot + C::TMEM_O, tslot + kk * 8,
+                    desc_add(vd, (kk * 16 * C::PANEL_BYTES) >> 4), idesc_o,
+                    (idx > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(sm.bar(C::B_PVDONE + s));
+      if (!x.resident || --kv_left[st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + 2 * st + s));
+      ++pc;
+    }
+    mma_commit(sm.bar(C::B_OFULL + s));
+    ++tq;
+  }
+#undef MMA_WAIT
+}
+
+// ------------------------------------------------------------------ bias warp
+// beta of each key block a tile sees, into its slot's 2-buffer ring, in tile
+// order over both slots.
+template <class C>
+__device__ void role_bias(const FwdArgs& a, const Smem<C>& sm, bool softmax) {
   volatile int* abort = sm.abort_flag();
   const int lane = threadIdx.x & 31;
-  uint32_t bc = 0;
-  TileRing<C, true> ring(s, 2);
+  uint32_t bcs[2] = {0u, 0u};
+  TileRing<C, true> ring(0, 1);
   FTile x{};
   while (ring.next(a, sm, x)) {
     const FwdProblem P = fwd_problem<C>(a, x.prob);
     if (P.bias_kind == 0) continue;  // the phi warpgroup adds no bias for this tile
+    const int s = x.slot;
     for (int j = x.kb0; j < x.kb1; ++j) {
+      uint32_t& bc = bcs[s];
       const int bb = bc & 1;
       bool ok = mbar_wait(sm.bar(C::B_BEMPTY + 2 * s + bb), ((bc >> 1) & 1) ^ 1, abort, a.status,
                           a.timeout_ns, 0x300 + C::B_BEMPTY + 2 * s + bb);
@@ -1060,7 +1190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < C::NKV; ++i) {
       mbar_init(sm.bar(C::B_KVFULL + i), 1);
-      mbar_init(sm.bar(C::B_KVEMPTY + i), 1);
+      mbar_init(sm.bar(C::B_KVEMPTY + 2 * i), 1);
+      mbar_init(sm.bar(C::B_KVEMPTY + 2 * i + 1), 1);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(sm.bar(C::B_BFULL + i), C::ROPE ? 64 : 32);  // rotary: both warps write beta
@@ -1100,13 +1231,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_to<kRegsControl, kRegsLaunch>();
     if (warp == 0) {
       if (lane == 0) role_producer<C>(a, sm, &tq, &tk, &tv);
-    } else if (warp == 1) {
-      if (lane == 0) role_mma<C>(a, sm, tmem);
     } else if constexpr (C::ROPE) {
-      role_rotary<C>(a, sm, SOFTMAX);
+      if (warp == 1) {
+        if (lane == 0) role_mma<C>(a, sm, tmem);
+      } else {
+        role_rotary<C>(a, sm, SOFTMAX);
+      }
+    } else if (warp == 1 || warp == 3) {
+      if (lane == 0) role_mma_slot<C>(a, sm, tmem, warp >> 1);
     } else {
       // a grouped launch may mix problems with and without a bias
-      if (C::GROUPED || a.p0.bias_kind != 0) role_bias<C>(a, sm, warp - 2, SOFTMAX);
+      if (C::GROUPED || a.p0.bias_kind != 0) role_bias<C>(a, sm, SOFTMAX);
     }
   } else if (warp < 12) {
     setmaxnreg_to<kRegsPhi, kRegsLaunch>();
