@@ -955,42 +955,59 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
             if (c0 + e < clo || c0 + e > chi) v[e] = __float_as_uint(fill);
         }
       };
-      bool need_rescale = false;
+      // Softmax in one pass: a chunk's P is taken against the running row
+      // maximum m_run while the chunk's maximum stays within kRescaleThreshold
+      // of it (so P <= 2^threshold).  A chunk that goes beyond moves m_run up
+      // to its maximum and scales by 2^(m_old - m_new) what was taken against
+      // the old value: the block's P chunks already in TMEM, the block's
+      // partial sums and l, and O (at the end of the block).
+      bool need_rescale = false;  // this row's O needs `factor` (not the tile's first block)
       float factor = 1.f;
-      if (SOFTMAX) {
-        // pass 1: the block's row maximum (4 independent partial maxima)
-        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int c0 = 0; c0 < C::BN; c0 += 32) {
-          uint32_t v[32];
-          scores(c0, v);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            pm[(e >> 1) & 3] = fmax3(pm[(e >> 1) & 3], __uint_as_float(v[e]),
-                                     __uint_as_float(v[e + 1]));
-        }
-        const float bm = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
-        if (idx == 0) {
-          m_run = bm;
-        } else if (bm > m_run + kRescaleThreshold) {
-          factor = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - bm);
-          need_rescale = true;
-          l_run *= factor;
-          m_run = bm;
-        }
-      }
-      // pass 2: P = phi(x), 32 columns at a time, written back as bf16 pairs over
-      // the S columns: chunk c0 lands in columns [c0/2, c0/2 + 16), which only
-      // hold S columns of chunks already read
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
       const uint64_t half2 = f2_pack(0.5f, 0.5f);
       uint64_t ps2[2] = {0ull, 0ull};  // packed partial sums (softmax)
+      // P = phi(x), 32 columns at a time, written back as bf16 pairs over the
+      // S columns: chunk c0 lands in columns [c0/2, c0/2 + 16), which only
+      // hold S columns of chunks already read
 #pragma unroll 1
       for (int c0 = 0; c0 < C::BN; c0 += 32) {
         uint32_t v[32];
         scores(c0, v);
         if (SOFTMAX) {
+          float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pm[(e >> 1) & 3] = fmax3(pm[(e >> 1) & 3], __uint_as_float(v[e]),
+                                     __uint_as_float(v[e + 1]));
+          const float cm = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
+          const bool grow = cm > m_run + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, grow)) {
+            float f = 1.f;
+            if (grow) {
+              f = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - cm);
+              m_run = cm;
+              l_run *= f;
+              factor *= f;
+              need_rescale = idx > 0;
+              const uint64_t f2 = f2_pack(f, f);
+              ps2[0] = f2_mul(ps2[0], f2);
+              ps2[1] = f2_mul(ps2[1], f2);
+            }
+            // the block's P pairs already written: columns [0, c0 / 2)
+            tmem_wait_st();
+#pragma unroll 1
+            for (int c = 0; c < c0 / 2; c += 16) {
+              uint32_t pr[16];
+              tmem_ld16(tslot + c, pr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                pr[e] = pack_bf16x2(__uint_as_float(pr[e] << 16) * f,
+                                    __uint_as_float(pr[e] & 0xffff0000u) * f);
+              tmem_st16(tslot + c, pr);
+            }
+          }
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t d2 =
@@ -1040,7 +1057,7 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
         f2_unpack(ps2[1], s2, s3);
         l_run += (s0 + s1) + (s2 + s3);
       }
-      if (SOFTMAX && __any_sync(0xffffffffu, need_rescale)) {
+      if (SOFTMAX && idx > 0 && __any_sync(0xffffffffu, need_rescale)) {
         // O must hold every earlier PV of the tile before it is rescaled: the
         // commit of the previous block's PV covers all of them
         PHI_WAIT(C::B_PVDONE + s, (nsb - 1) & 1, 0x400 + C::B_PVDONE + s);

@@ -100,6 +100,22 @@ def test_single_sample_single_key(cuda_lib):
     assert torch.equal(o.cpu(), w.v)  # softmax over one key returns V_0 exactly
 
 
+@pytest.mark.parametrize("slope", [0.15, 2.0, -2.0])
+def test_softmax_running_max_moves(cuda_lib, slope):
+    # An additive bias rising along the keys moves each row's maximum up
+    # within and across 128-key blocks: with slope 2.0 every 32-key chunk moves
+    # it far past the rescale threshold (earlier P chunks, the partial sums, l
+    # and O are all rescaled); with 0.15 only every second chunk or so; a
+    # falling bias never moves it after the first chunk.
+    kl = [300, 513, 64, 1000]
+    w = make_workload(5, seed=44, q_lens=[130, 7, 64, 200], kv_lens=kl, bias=BIAS_ADD,
+                      with_dout=False)
+    for b in range(w.B):
+        k0, k1 = int(w.kv_offsets[b]), int(w.kv_offsets[b + 1])
+        w.bias[:, k0:k1] = slope * torch.arange(k1 - k0, dtype=torch.float32)
+    check_against_oracle(cuda_lib, w)
+
+
 def test_repeat_calls_bit_identical(cuda_lib):
     w = make_workload(2, B=8)
     o1, _ = run_gpu_forward(cuda_lib, w)
