@@ -165,6 +165,22 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H, int D, int 
   return r == CUDA_SUCCESS;
 }
 
+// O [rows][H][D] bf16 for the forward's TMA stores: boxes of 32 rows x one
+// head x 32 columns (64 bytes, 64-byte swizzle, the epilogue's staging
+// layout).
+bool make_map_o(CUtensorMap* m, void* base, int64_t rows, int H, int D) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {32u, 1u, 32u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Row-major bf16 tensor of up to three dims (innermost first), 128-byte
 // swizzled boxes whose inner extent is 64 elements.
 bool make_map_3d(CUtensorMap* m, const void* base, const cuuint64_t (&dims)[3],
@@ -291,7 +307,7 @@ gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
     const size_t nv = g.vp.size();
     g.off_probs = total;
     g.off_maps = align256(g.off_probs + nv * sizeof(FwdProblem));
-    g.off_sched = align256(g.off_maps + 3 * nv * sizeof(CUtensorMap));
+    g.off_sched = align256(g.off_maps + 4 * nv * sizeof(CUtensorMap));
     total = align256(g.off_sched + nv * sizeof(GroupSchedProblem));
   }
   lay.tables_end = total;
@@ -401,8 +417,9 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
     q = rq;
     k = rk;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_map(&tq, q, p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
+  if (!make_map_o(&to, const_cast<void*>(o), p->total_q, p->H, p->D)) return GDPA_ERR_CUDA;
   if (p->total_kv > 0) {
     if (!make_map(&tk, k, p->total_kv, p->H, p->D, block_n)) return GDPA_ERR_CUDA;
     if (!make_map(&tv, v, p->total_kv, p->H, p->D, block_n)) return GDPA_ERR_CUDA;
@@ -440,7 +457,7 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
     a.p0.phi = phi;
     a.p0.head_mask = heads;
     a.p0.lse = phi == GDPA_PHI_SOFTMAX ? lse : nullptr;
-    e = launch_forward(a, p->D, block_n, tq, tk, tv, sms, s);
+    e = launch_forward(a, p->D, block_n, tq, tk, tv, to, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;
@@ -639,14 +656,16 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
       CUtensorMap m;
       if (p->total_q > 0) {
         if (!make_map(&m, qsrc[vp.src], p->total_q, p->H, p->D, kBlockM)) return GDPA_ERR_CUDA;
-        std::memcpy(&maps[3 * j], &m, sizeof(m));
+        std::memcpy(&maps[4 * j], &m, sizeof(m));
+        if (!make_map_o(&m, f.o, p->total_q, p->H, p->D)) return GDPA_ERR_CUDA;
+        std::memcpy(&maps[4 * j + 3], &m, sizeof(m));
         if (q_map[gi] < 0) q_map[gi] = (int)j;
       }
       if (p->total_kv > 0) {
         if (!make_map(&m, ksrc[vp.src], p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
-        std::memcpy(&maps[3 * j + 1], &m, sizeof(m));
+        std::memcpy(&maps[4 * j + 1], &m, sizeof(m));
         if (!make_map(&m, f.v, p->total_kv, p->H, p->D, g.block_n)) return GDPA_ERR_CUDA;
-        std::memcpy(&maps[3 * j + 2], &m, sizeof(m));
+        std::memcpy(&maps[4 * j + 2], &m, sizeof(m));
       }
       sp[j].q_offsets = f.q_offsets;
       sp[j].kv_offsets = f.kv_offsets;
@@ -664,10 +683,10 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
     // maps of empty tensors are never read; keep every slot a valid map
     if (q_map[gi] >= 0)
       for (size_t j = 0; j < nv; ++j)
-        for (int w = 0; w < 3; ++w)
+        for (int w = 0; w < 4; ++w)
           if (problems[g.vp[j].src].params.total_q == 0 ||
-              (w > 0 && problems[g.vp[j].src].params.total_kv == 0))
-            std::memcpy(&maps[3 * j + w], &maps[3 * q_map[gi]], sizeof(CUtensorMap));
+              ((w == 1 || w == 2) && problems[g.vp[j].src].params.total_kv == 0))
+            std::memcpy(&maps[4 * j + w], &maps[4 * q_map[gi]], sizeof(CUtensorMap));
     jobs[gi].probs = reinterpret_cast<const GroupSchedProblem*>(ws + g.off_sched);
     jobs[gi].n_probs = (int)nv;
     jobs[gi].n_entries = g.entries;
@@ -698,8 +717,8 @@ gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* problems, int n
     a.probs = reinterpret_cast<const FwdProblem*>(ws + g.off_probs);
     a.maps = reinterpret_cast<const CUtensorMap*>(ws + g.off_maps);
     CUtensorMap m0;  // kernel parameters, unused when grouped
-    std::memcpy(&m0, at(g.off_maps) + 3 * q_map[gi] * sizeof(CUtensorMap), sizeof(m0));
-    e = launch_forward(a, g.D, g.block_n, m0, m0, m0, sms, s);
+    std::memcpy(&m0, at(g.off_maps) + 4 * q_map[gi] * sizeof(CUtensorMap), sizeof(m0));
+    e = launch_forward(a, g.D, g.block_n, m0, m0, m0, m0, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;

@@ -55,10 +55,10 @@ constexpr int kRegsLaunch = 96;    // 65536 / 640 rounded down to a multiple of 
 #define GDPA_FWD_RC 96
 #endif
 #ifndef GDPA_FWD_RP
-#define GDPA_FWD_RP 112
+#define GDPA_FWD_RP 104
 #endif
 #ifndef GDPA_FWD_RE
-#define GDPA_FWD_RE 80
+#define GDPA_FWD_RE 88
 #endif
 constexpr int kRegsControl = GDPA_FWD_RC;  // warpgroup 0: producer, MMA issuer, allocator, bias
 constexpr int kRegsPhi = GDPA_FWD_RP;      // warpgroups 1-2: phi of slot 0 / 1
@@ -357,7 +357,7 @@ __device__ void role_producer(const FwdArgs& a, const Smem<C>& sm, const CUtenso
   FTile x{};
   // a grouped launch keeps each problem's Q, K, V maps in device memory
   auto map_of = [&](int prob, int which) -> const CUtensorMap* {
-    if constexpr (C::GROUPED) return a.maps + 3 * prob + which;
+    if constexpr (C::GROUPED) return a.maps + 4 * prob + which;
     return which == 0 ? tq : which == 1 ? tk : tv;
   };
   auto load_kv = [&](uint32_t ring, int kb) -> bool {
@@ -1094,12 +1094,16 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
 
 // ------------------------------------------------------------------ epilogue warpgroups
 // One warpgroup per slot: O of each tile from TMEM (released to the next
-// tile's PV as soon as it is read), times 1/l for softmax, to bf16, through
-// the warp's staging rows in shared memory to 64-byte row segments in global
-// memory, 32 columns per pass.  Tiles without visible keys get O = 0 (and LSE
-// = -inf) here.  Each warp handles its 32 rows on its own.
+// tile's PV as soon as it is read), times 1/l for softmax, to bf16 in the
+// warp's staging box in shared memory (32 rows x 32 columns, 64-byte
+// swizzle), 32 columns per pass; a box whose 32 rows all lie in the sample
+// goes out as one TMA store (the async proxy: no load-store unit traffic,
+// which the other roles' shared-memory and barrier operations share), a
+// ragged one as plain stores of its valid rows.  Tiles without visible keys
+// get O = 0 (and LSE = -inf) here.  Each warp handles its 32 rows on its own.
 template <class C, bool SOFTMAX>
-__device__ void role_epilogue(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
+__device__ void role_epilogue(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s,
+                              const CUtensorMap* to) {
   volatile int* abort = sm.abort_flag();
   const int warp = threadIdx.x >> 5;
   const int wq = warp & 3;                  // TMEM lane quarter of this warp
@@ -1141,9 +1145,14 @@ __device__ void role_epilogue(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
     }
     EPI_WAIT(C::B_OFULL + s, tq & 1, 0x600 + C::B_OFULL + s);
     tc_fence_after();
+    const CUtensorMap* omap = C::GROUPED ? a.maps + 4 * x.prob + 3 : to;
+    const int r0 = x.m0 + wq * 32;          // this warp's first row in the sample
+    const bool boxed = r0 + 32 <= x.Lq;     // all 32 rows in the sample
     constexpr int NPASS = C::D / 32;
 #pragma unroll 1
     for (int ps = 0; ps < NPASS; ++ps) {
+      if (lane == 0) bulk_wait_read_all();  // the previous box has left the staging rows
+      __syncwarp();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {  // 16 columns per TMEM load
         uint32_t raw[16];
@@ -1161,27 +1170,37 @@ __device__ void role_epilogue(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
                        pack_bf16x2(__uint_as_float(raw[e + 4]) * inv, __uint_as_float(raw[e + 5]) * inv),
                        pack_bf16x2(__uint_as_float(raw[e + 6]) * inv, __uint_as_float(raw[e + 7]) * inv));
       }
-      __syncwarp();
+      if (boxed) {
+        fence_proxy_async_smem();  // the staged rows, visible to the TMA engine
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(omap, sm.stage(ew, 0, 0), ps * 32, x.h, x.q0 + r0);
+          bulk_commit_group();
+        }
+      } else {
+        __syncwarp();
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int j = it * 8 + (lane >> 2), cc = lane & 3;  // row of this warp, chunk
-        const int grow = x.m0 + wq * 32 + j;
-        const uint4 v = ld_shared_v4(sm.stage(ew, j, cc));
-        if (grow < x.Lq)
-          *reinterpret_cast<uint4*>(out + ((int64_t)(x.q0 + grow) * Hp + x.h) * C::D + ps * 32 +
-                                    cc * 8) = v;
+        for (int it = 0; it < 4; ++it) {
+          const int j = it * 8 + (lane >> 2), cc = lane & 3;  // row of this warp, chunk
+          const uint4 v = ld_shared_v4(sm.stage(ew, j, cc));
+          if (r0 + j < x.Lq)
+            *reinterpret_cast<uint4*>(out + ((int64_t)(x.q0 + r0 + j) * Hp + x.h) * C::D +
+                                      ps * 32 + cc * 8) = v;
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     ++tq;
   }
+  if (lane == 0) bulk_wait_all();  // every box written before the CTA ends
 #undef EPI_WAIT
 }
 
 template <int D, int BN, bool SOFTMAX, bool GROUPED, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     gdpa_fwd_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap tq,
-                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                    const __grid_constant__ CUtensorMap to) {
   using C = FwdCfg<D, BN, GROUPED, ROPE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem<C> sm;
@@ -1232,6 +1251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&to);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(sm.tmem_slot()), C::TMEM_COLS);
@@ -1265,7 +1285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     role_phi<C, SOFTMAX>(a, sm, tmem, (warp - 4) >> 2);
   } else {
     setmaxnreg_to<kRegsEpi, kRegsLaunch>();
-    role_epilogue<C, SOFTMAX>(a, sm, tmem, (warp - 12) >> 2);
+    role_epilogue<C, SOFTMAX>(a, sm, tmem, (warp - 12) >> 2, &to);
   }
   __syncwarp();
   tc_fence_before();
@@ -1287,7 +1307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int BN, bool SOFTMAX, bool GROUPED, bool ROPE = false>
 cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                       const CUtensorMap& tv, int sms, cudaStream_t stream) {
+                       const CUtensorMap& tv, const CUtensorMap& to, int sms,
+                       cudaStream_t stream) {
   using C = FwdCfg<D, BN, GROUPED, ROPE>;
   auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED, ROPE>;
   // when the roles' register budgets differ, the raising side's setmaxnreg
@@ -1308,7 +1329,7 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
   // the kernel allocates all 512 TMEM columns: exactly one CTA per SM
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
   const int grid = std::max(1, std::min(a.n_units, sms));
-  kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv);
+  kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv, to);
   return cudaGetLastError();
 }
 
@@ -1322,8 +1343,8 @@ int forward_block_n(int D, int phi, int max_kv, int debug_flags) {
 }
 
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, int sms,
-                           cudaStream_t stream) {
+                           const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                           int sms, cudaStream_t stream) {
   const bool sm = a.phi == 1;
   const bool grouped = a.probs != nullptr;
   const bool rope = a.rope_q != nullptr;
@@ -1331,13 +1352,13 @@ cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorM
 #define GDPA_FWD_CASE(D_, BN_)                                                         \
   if (D == D_ && block_n == BN_) {                                                     \
     if (grouped)                                                                       \
-      return sm ? launch_one<D_, BN_, true, true>(a, tq, tk, tv, sms, stream)          \
-                : launch_one<D_, BN_, false, true>(a, tq, tk, tv, sms, stream);        \
+      return sm ? launch_one<D_, BN_, true, true>(a, tq, tk, tv, to, sms, stream)          \
+                : launch_one<D_, BN_, false, true>(a, tq, tk, tv, to, sms, stream);        \
     if (rope)                                                                          \
-      return sm ? launch_one<D_, BN_, true, false, true>(a, tq, tk, tv, sms, stream)   \
-                : launch_one<D_, BN_, false, false, true>(a, tq, tk, tv, sms, stream); \
-    return sm ? launch_one<D_, BN_, true, false>(a, tq, tk, tv, sms, stream)           \
-              : launch_one<D_, BN_, false, false>(a, tq, tk, tv, sms, stream);         \
+      return sm ? launch_one<D_, BN_, true, false, true>(a, tq, tk, tv, to, sms, stream)   \
+                : launch_one<D_, BN_, false, false, true>(a, tq, tk, tv, to, sms, stream); \
+    return sm ? launch_one<D_, BN_, true, false>(a, tq, tk, tv, to, sms, stream)           \
+              : launch_one<D_, BN_, false, false>(a, tq, tk, tv, to, sms, stream);         \
   }
   GDPA_FWD_CASE(32, 64)
   GDPA_FWD_CASE(32, 128)

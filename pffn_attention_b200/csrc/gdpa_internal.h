@@ -62,11 +62,11 @@ struct FwdArgs {
   uint64_t head_mask;       // single problem: heads computed (bit h), ~0 = all
   // Grouped launch: problem of sorted entry e is eprob[e]; units are
   // (entry, head) with head stride H (the group's largest), units a problem
-  // lacks are skipped; per-problem data and Q/K/V maps in device memory.
+  // lacks are skipped; per-problem data and Q/K/V/O maps in device memory.
   // All nullptr for a single problem (p0 and the kernel's map parameters).
   const int32_t* eprob;
   const FwdProblem* probs;
-  const CUtensorMap* maps;  // [problem][Q, K, V]
+  const CUtensorMap* maps;  // [problem][Q, K, V, O]
   FwdProblem p0;
   // rotary temporal embedding (single problem): per-token (cos, sin) fp16
   // pairs, [total_q][D/2] and [total_kv][D/2]; nullptr = no rotation
@@ -130,8 +130,8 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
 cudaError_t launch_group_schedule(const GroupSchedJob* jobs, int n_jobs, int max_entries,
                                   int block_m, DeviceStatus* status, cudaStream_t stream);
 cudaError_t launch_forward(const FwdArgs& a, int D, int block_n, const CUtensorMap& tq,
-                           const CUtensorMap& tk, const CUtensorMap& tv, int sms,
-                           cudaStream_t stream);
+                           const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                           int sms, cudaStream_t stream);
 int forward_block_n(int D, int phi, int max_kv, int debug_flags);
 cudaError_t launch_bwd_preprocess(const __nv_bfloat16* o, const __nv_bfloat16* dout,
                                   float* delta, int64_t total_q, int H, int D,
