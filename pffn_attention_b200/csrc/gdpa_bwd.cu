@@ -36,9 +36,7 @@
 // it, then dQ (fp32, D columns); then dK, dV.
 // Shared memory: K, V of the key block; 2-stage rings of Q and dO tiles; dS
 // (bf16, the MN-major A operand of dQ), which also stages the dK, dV rows at
-// the end of a key block; LSE / delta rows of two tiles.  P and dS are
-// rounded to bf16 with integer operations (round to nearest, ties away), which
-// leaves the conversion unit to ex2.
+// the end of a key block; LSE / delta rows of two tiles.
 //
 // Warp roles (512 threads): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator and
 // LSE / delta loader, 3 idle; warpgroups 1-2 compute P and dS (a thread owns
@@ -589,7 +587,7 @@ __device__ void bwd_compute(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem)
                 k0 = v0 ? k0 : 0.f;
                 k1 = v1 ? k1 : 0.f;
               }
-              pk[e2] = pack_bf16x2_int(p0, p1);
+              pk[e2] = pack_bf16x2(p0, p1);
               if (!SOFTMAX) kk[e2] = pack_f16x2(k0, k1);  // phi' in [-0.2, 1.2]: fp16
             }
             // P^T chunk -> the first 32 S^T columns of this warpgroup (read in
@@ -649,7 +647,7 @@ __device__ void bwd_compute(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem)
               dsum2 = f2_add(dsum2, ds2);
               float d0, d1;
               f2_unpack(ds2, d0, d1);
-              pk[e2] = pack_bf16x2_int(d0, d1);
+              pk[e2] = pack_bf16x2(d0, d1);
             }
             tmem_st16(tmem + tl + C::T_DP + c0 + ch * 16, pk);
             // dS^T row r -> panel g (queries 64g .. 64g+63), 128-byte swizzle
