@@ -729,9 +729,10 @@ def run_rotary(args):
 
 
 def run_sumkron(args):
-    """SumKronLinear forward on the page's typical configuration (seed
-    summaries of the seed-pooling batch): useful FLOPs of the cheaper
-    association, 2 k T S D + 2 k T D^2 per sample."""
+    """SumKronLinear forward and backward on the page's typical configuration
+    (seed summaries of the seed-pooling batch).  Useful FLOPs of the cheaper
+    association: forward 2 k T S D + 2 k T D^2 per sample; backward twice
+    that (dY W^T, A^T U, U X^T, Z^T dY; the recomputed Z = A X excluded)."""
     import torch
 
     from pffn_attention_b200 import gdpa
@@ -741,35 +742,52 @@ def run_sumkron(args):
     c = SUMKRON_CONFIG
     B, S, T, D, k = c["B"], c["S"], c["T"], c["D"], c["k"]
     x, a, w = make_sumkron(B, S, T, D, k, seed=1, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+    dy = torch.randn((B, T, D), generator=gen, device=dev).to(torch.bfloat16)
     stream = torch.cuda.Stream(device=dev)
     y, ws = gdpa.sumkron_forward(x, a, w, stream=stream)
-    for _ in range(args.warmup):
-        gdpa.sumkron_forward(x, a, w, out=y, workspace=ws, stream=stream)
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        gdpa.sumkron_forward(x, a, w, out=y, workspace=ws, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    _, _, _, wsb = gdpa.sumkron_backward(x, a, w, dy, stream=stream)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_f = timed(lambda: gdpa.sumkron_forward(x, a, w, out=y, workspace=ws, stream=stream))
     assert gdpa.device_status(ws, stream) == 0
-    ms = e0.elapsed_time(e1) / args.steps
-    flops = B * (2.0 * k * T * S * D + 2.0 * k * T * D * D)
+    ms_b = timed(lambda: gdpa.sumkron_backward(x, a, w, dy, workspace=wsb, stream=stream))
+    assert gdpa.device_status(wsb, stream) == 0
+    flops_f = B * (2.0 * k * T * S * D + 2.0 * k * T * D * D)
+    flops_b = 2.0 * flops_f
     byts = 2.0 * (x.numel() + y.numel() + a.numel() + w.numel())
     peaks, src = load_peaks()
-    tf = flops / (ms * 1e-3) / 1e12
-    return {"metric": "SumKronLinear forward, HSP second stage (useful TFLOP/s)",
+    tf_f = flops_f / (ms_f * 1e-3) / 1e12
+    tf_b = flops_b / (ms_b * 1e-3) / 1e12
+    tf = (flops_f + flops_b) / ((ms_f + ms_b) * 1e-3) / 1e12
+    return {"metric": "SumKronLinear forward + backward, HSP second stage (useful TFLOP/s)",
             "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "dtype": "bf16", "data": "synthetic",
+            "warmup": args.warmup, "ms_per_step": round(ms_f + ms_b, 4),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "sumkron_hsp", **c, "l2": "inputs > L2"},
-            "roofline": {"bound": "tensor", "achieved": round(tf, 2),
+            "fwd_ms": round(ms_f, 4), "fwd_tflops": round(tf_f, 2),
+            "bwd_ms": round(ms_b, 4), "bwd_tflops": round(tf_b, 2),
+            "roofline": {"bound": "tensor", "achieved": round(tf_f, 2),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "frac": round(tf_f / peaks["bf16_tflops"], 4),
+                         "kernel": "gdpa_sumkron_forward",
                          "traffic": measured_traffic("gdpa_sumkron_forward", B),
                          "traffic_unit": "bytes per launch", "algorithmic": byts,
-                         "peak_source": src},
-            "achieved_gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
+                         "peak_source": src,
+                         "bwd_frac": round(tf_b / peaks["bf16_tflops"], 4)},
+            "achieved_gbs": round(byts / (ms_f * 1e-3) / 1e9, 1)}
 
 
 def main(argv=None):
@@ -793,7 +811,7 @@ def main(argv=None):
     ap.add_argument("--rotary", action="store_true",
                     help="time the sliding-window forward with the rotary temporal embedding")
     ap.add_argument("--sumkron", action="store_true",
-                    help="time the fused SumKronLinear forward (HSP second stage)")
+                    help="time the SumKronLinear forward and backward (HSP second stage)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -210,6 +210,32 @@ GDPA_API gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, cons
                                             void* workspace, size_t workspace_bytes,
                                             gdpa_stream_t stream);
 
+/* Workspace bytes of gdpa_sumkron_backward: the status block, two bf16
+ * intermediates of B x k T x D elements each, and fp32 partial sums of dA
+ * (min(B, 64) x k T x S) and dW (min(B, 8) x k D x D).  0 on invalid
+ * parameters. */
+GDPA_API size_t gdpa_sumkron_backward_workspace_size(const gdpa_sumkron_params_t* p);
+
+/* Gradients of y = SumKronLinear(x; a, w) (Kunlun paper review §2.4; the map
+ * of gdpa_sumkron_forward, Y_b = sum_r A_r X_b W_r) for the upstream gradient
+ * dy [B][T][D]:
+ *   dx [B][S][D] = sum_r A_r^T dY_b W_r^T
+ *   da [k][T][S] = sum_b (dY_b W_r^T) X_b^T        (one T x S block per r)
+ *   dw [k][D][D] = sum_b (A_r X_b)^T dY_b          (one D x D block per r)
+ * All bf16 row-major device arrays, 16-byte aligned, the caller's; fp32
+ * accumulation (the sums over samples are split into fp32 partials in the
+ * workspace and added in fp32).  x, a, w are the forward's inputs.  Same
+ * parameter limits as the forward, and B <= 65535; B = 0 gives zero da and
+ * dw.  The workspace's status is cleared on the stream first (read it with
+ * gdpa_get_device_status; GDPA_ERR_TIMEOUT if a bounded wait ran out).
+ * Asynchronous on stream.  Errors (before any launch): as
+ * gdpa_sumkron_forward, with GDPA_ERR_WORKSPACE below
+ * gdpa_sumkron_backward_workspace_size. */
+GDPA_API gdpa_status_t gdpa_sumkron_backward(const gdpa_sumkron_params_t* p, const void* x,
+                                             const void* a, const void* w, const void* dy,
+                                             void* dx, void* da, void* dw, void* workspace,
+                                             size_t workspace_bytes, gdpa_stream_t stream);
+
 /* Bytes of device workspace gdpa_forward (backward = 0) or gdpa_backward
  * (backward = 1) needs for these parameters.  0 on invalid parameters. */
 GDPA_API size_t gdpa_workspace_size(const gdpa_params_t* p, int backward);

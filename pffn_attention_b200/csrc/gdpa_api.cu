@@ -333,6 +333,48 @@ gdpa_status_t plan_grouped(const gdpa_forward_problem_t* probs, int n,
 
 }  // namespace
 
+// ---------------------------------------------------------------- SumKronLinear backward
+// For Y_b = sum_r A_r X_b W_r and the upstream gradient dY (Kunlun paper review
+// §2.4; the reading of the map is the forward's):
+//   Z_b   = [A_1; ...; A_k] X_b                   (k T x D, recomputed)
+//   U_b   = dY_b [W_1^T ... W_k^T], stored as [r][t][d]      (k T x D)
+//   dX_b  = sum_r A_r^T U_b[r] = [A_1; ...; A_k]^T U_b         (S x D)
+//   dA_r  = sum_b U_b[r] X_b^T                                  (T x S)
+//   dW_r  = sum_b Z_b[r]^T dY_b                                 (D x D)
+// five batched GEMMs (gdpa_gemm.cu); dA and dW sum over the samples, split
+// across CTAs into fp32 partials that a last pass adds up.
+namespace {
+
+int sk_splits_a(int B) { return std::max(1, std::min(B, 64)); }
+int sk_splits_w(int B) { return std::max(1, std::min(B, 8)); }
+
+struct SkBwdLayout {
+  size_t z, u, pa, pw, end;
+};
+SkBwdLayout sk_bwd_layout(const gdpa_sumkron_params_t* p) {
+  SkBwdLayout L{};
+  const size_t kT = (size_t)p->k * p->T;
+  size_t off = align256(sizeof(DeviceStatus));
+  L.z = off;
+  off = align256(off + (size_t)p->B * kT * p->D * 2);
+  L.u = off;
+  off = align256(off + (size_t)p->B * kT * p->D * 2);
+  L.pa = off;
+  off = align256(off + (size_t)sk_splits_a(p->B) * kT * p->S * 4);
+  L.pw = off;
+  off = align256(off + (size_t)sk_splits_w(p->B) * p->k * p->D * p->D * 4);
+  L.end = off;
+  return L;
+}
+
+// bf16 [dim2][dim1][dim0] (dim0 contiguous), boxes box0 x box1 x 1, 128-byte swizzle
+bool sk_map(CUtensorMap* m, const void* base, cuuint64_t d0, cuuint64_t d1, cuuint64_t d2,
+            cuuint32_t box0, cuuint32_t box1) {
+  return make_map_3d(m, base, {d0, d1, d2}, {d0 * 2, d0 * d1 * 2}, {box0, box1, 1u});
+}
+
+}  // namespace
+
 extern "C" {
 
 int gdpa_version(void) { return 100; }
@@ -814,6 +856,105 @@ gdpa_status_t gdpa_sumkron_forward(const gdpa_sumkron_params_t* p, const void* x
   L.debug_flags = p->debug_flags;
   L.timeout_ns = (uint64_t)(p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000) * 1000ull;
   return launch_sumkron(L, ta, tx, tw, sms, s) == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}
+
+
+size_t gdpa_sumkron_backward_workspace_size(const gdpa_sumkron_params_t* p) {
+  return check_sumkron(p) == GDPA_OK ? sk_bwd_layout(p).end : 0;
+}
+
+gdpa_status_t gdpa_sumkron_backward(const gdpa_sumkron_params_t* p, const void* x, const void* a,
+                                    const void* w, const void* dy, void* dx, void* da, void* dw,
+                                    void* workspace, size_t workspace_bytes,
+                                    gdpa_stream_t stream) {
+  gdpa_status_t st = check_sumkron(p);
+  if (st != GDPA_OK) return st;
+  if (p->B > 0 && (!x || !dy || !dx)) return GDPA_ERR_INVALID_ARG;
+  if (!a || !w || !da || !dw || !aligned16(x) || !aligned16(a) || !aligned16(w) ||
+      !aligned16(dy) || !aligned16(dx) || !aligned16(da) || !aligned16(dw) ||
+      !aligned16(workspace))
+    return GDPA_ERR_INVALID_ARG;
+  const SkBwdLayout L = sk_bwd_layout(p);
+  if (!workspace || workspace_bytes < L.end) return GDPA_ERR_WORKSPACE;
+  int sms = 0;
+  if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), s) != cudaSuccess) return GDPA_ERR_CUDA;
+  const int B = p->B, S = p->S, T = p->T, D = p->D, k = p->k, kT = k * T;
+  if (B > 65535) return GDPA_ERR_UNSUPPORTED;  // samples are a grid dimension
+  if (B == 0) {  // no sample: the parameter gradients are zero
+    if (cudaMemsetAsync(da, 0, (size_t)kT * S * 2, s) != cudaSuccess ||
+        cudaMemsetAsync(dw, 0, (size_t)k * D * D * 2, s) != cudaSuccess)
+      return GDPA_ERR_CUDA;
+    return GDPA_OK;
+  }
+  void* z = ws + L.z;
+  void* u = ws + L.u;
+  float* pa = reinterpret_cast<float*>(ws + L.pa);
+  float* pw = reinterpret_cast<float*>(ws + L.pw);
+  const cuuint32_t bT = (cuuint32_t)T;
+  CUtensorMap m_ak, m_xmn, m_dyk, m_wk, m_amn, m_umn, m_uk, m_xk, m_zmn, m_dymn;
+  if (!sk_map(&m_ak, a, S, kT, 1, 64, 128) ||                    // A [kT][S], K-major (K = s)
+      !sk_map(&m_xmn, x, D, S, B, 64, 64) ||                     // X [B][S][D], MN-major (K = s)
+      !sk_map(&m_dyk, dy, D, (cuuint64_t)B * T, 1, 64, 128) ||   // dY [B T][D], K-major (K = e)
+      !sk_map(&m_wk, w, D, (cuuint64_t)k * D, 1, 64, 128) ||     // W [k D][D], K-major (K = e)
+      !sk_map(&m_amn, a, S, kT, 1, 64, 64) ||                    // A, MN-major (M = s, K = r t)
+      !sk_map(&m_umn, u, D, kT, B, 64, 64) ||                    // U [B][kT][D], MN-major
+      !sk_map(&m_uk, u, D, kT, B, 64, 128) ||                    // U, K-major (K = d)
+      !sk_map(&m_xk, x, D, S, B, 64, 128) ||                     // X, K-major (K = d)
+      !sk_map(&m_zmn, z, D, kT, B, 64, bT) ||                    // Z [B][kT][D], MN-major (K = t)
+      !sk_map(&m_dymn, dy, D, T, B, 64, bT))                     // dY [B][T][D], MN-major (K = t)
+    return GDPA_ERR_CUDA;
+  GemmLaunch g{};
+  g.status = reinterpret_cast<DeviceStatus*>(ws);
+  g.timeout_ns = (uint64_t)(p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000) * 1000ull;
+  auto run = [&](const CUtensorMap& ta, const CUtensorMap& tb) {
+    return launch_gemm(g, ta, tb, s) == cudaSuccess;
+  };
+  // Z_b = A X_b: M = kT, N = D, K = S; per sample
+  g.M = kT; g.N = D; g.Z = B; g.n_rb = 1; g.nkc = S / 64; g.kc = 64; g.splits = 1;
+  g.a = GemmOperand{0, 0, 0};
+  g.b = GemmOperand{1, 0, 2};
+  g.f32_out = 0; g.out = z; g.mT = kT; g.nD = D;
+  g.sZ = (int64_t)kT * D; g.sMb = 0; g.sMt = D; g.sNr = 0;
+  if (!run(m_ak, m_xmn)) return GDPA_ERR_CUDA;
+  // U = dY [W_1 ... W_k]^T: M = B T rows (b, t), N = k D columns (r, d), K = D;
+  // row (b, t), column (r, d) stored at U[b][r][t][d]
+  g.M = B * T; g.N = k * D; g.Z = 1; g.n_rb = 1; g.nkc = D / 64; g.kc = 64; g.splits = 1;
+  g.a = GemmOperand{0, 0, 0};
+  g.b = GemmOperand{0, 0, 0};
+  g.f32_out = 0; g.out = u; g.mT = T; g.nD = D;
+  g.sZ = 0; g.sMb = (int64_t)kT * D; g.sMt = D; g.sNr = (int64_t)T * D;
+  if (!run(m_dyk, m_wk)) return GDPA_ERR_CUDA;
+  // dX_b = A^T U_b: M = S, N = D, K = kT; per sample
+  g.M = S; g.N = D; g.Z = B; g.n_rb = 1; g.nkc = kT / 64; g.kc = 64; g.splits = 1;
+  g.a = GemmOperand{1, 0, 0};
+  g.b = GemmOperand{1, 0, 2};
+  g.f32_out = 0; g.out = dx; g.mT = S; g.nD = D;
+  g.sZ = (int64_t)S * D; g.sMb = 0; g.sMt = D; g.sNr = 0;
+  if (!run(m_amn, m_umn)) return GDPA_ERR_CUDA;
+  // dA = sum_b U_b X_b^T: M = kT, N = S, K = D per sample, samples split
+  const int spa = sk_splits_a(B);
+  g.M = kT; g.N = S; g.Z = 1; g.n_rb = B; g.nkc = D / 64; g.kc = 64; g.splits = spa;
+  g.a = GemmOperand{0, 0, 1};
+  g.b = GemmOperand{0, 0, 1};
+  g.f32_out = 1; g.out = pa;
+  if (!run(m_uk, m_xk)) return GDPA_ERR_CUDA;
+  if (launch_sum_splits(pa, spa, (int64_t)kT * S, static_cast<__nv_bfloat16*>(da), sms, s) !=
+      cudaSuccess)
+    return GDPA_ERR_CUDA;
+  // dW_r = sum_b Z_b[r]^T dY_b: M = N = D, K = T per sample, per r, samples split
+  const int spw = sk_splits_w(B);
+  g.M = D; g.N = D; g.Z = k; g.n_rb = B; g.nkc = 1; g.kc = T; g.splits = spw;
+  g.a = GemmOperand{1, T, 1};
+  g.b = GemmOperand{1, 0, 1};
+  g.f32_out = 1; g.out = pw;
+  if (!run(m_zmn, m_dymn)) return GDPA_ERR_CUDA;
+  if (launch_sum_splits(pw, spw, (int64_t)k * D * D, static_cast<__nv_bfloat16*>(dw), sms, s) !=
+      cudaSuccess)
+    return GDPA_ERR_CUDA;
+  return GDPA_OK;
 }
 
 gdpa_status_t gdpa_get_device_status(const void* workspace, gdpa_stream_t stream) {

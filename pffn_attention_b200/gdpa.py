@@ -27,7 +27,8 @@ EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_s
             "gdpa_forward_tile_shape", "gdpa_get_device_status", "gdpa_status_string",
             "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
             "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table",
-            "gdpa_rotary_apply", "gdpa_sumkron_workspace_size", "gdpa_sumkron_forward")
+            "gdpa_rotary_apply", "gdpa_sumkron_workspace_size", "gdpa_sumkron_forward",
+            "gdpa_sumkron_backward_workspace_size", "gdpa_sumkron_backward")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -117,6 +118,10 @@ def load(path: str = LIB_PATH):
     lib.gdpa_sumkron_workspace_size.restype = sz
     lib.gdpa_sumkron_forward.argtypes = [SP, vp, vp, vp, vp, vp, sz, st]
     lib.gdpa_sumkron_forward.restype = ctypes.c_int
+    lib.gdpa_sumkron_backward_workspace_size.argtypes = [SP]
+    lib.gdpa_sumkron_backward_workspace_size.restype = sz
+    lib.gdpa_sumkron_backward.argtypes = [SP, vp, vp, vp, vp, vp, vp, vp, vp, sz, st]
+    lib.gdpa_sumkron_backward.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -153,6 +158,15 @@ def gdpa_sumkron_workspace_size(p: gdpa_sumkron_params_t) -> int:
 def gdpa_sumkron_forward(p, x, a, w, y, workspace, workspace_bytes, stream) -> int:
     return int(load().gdpa_sumkron_forward(ctypes.byref(p), x, a, w, y, workspace,
                                            workspace_bytes, stream))
+
+
+def gdpa_sumkron_backward_workspace_size(p: gdpa_sumkron_params_t) -> int:
+    return int(load().gdpa_sumkron_backward_workspace_size(ctypes.byref(p)))
+
+
+def gdpa_sumkron_backward(p, x, a, w, dy, dx, da, dw, workspace, workspace_bytes, stream) -> int:
+    return int(load().gdpa_sumkron_backward(ctypes.byref(p), x, a, w, dy, dx, da, dw, workspace,
+                                            workspace_bytes, stream))
 
 
 def gdpa_forward_grouped_workspace_size(problems) -> int:
@@ -300,6 +314,27 @@ def sumkron_forward(x, a, w, *, out=None, workspace=None, stream=None, wait_time
     _check(gdpa_sumkron_forward(p, _ptr(x), _ptr(a), _ptr(w), _ptr(out), _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "gdpa_sumkron_forward")
     return out, workspace
+
+
+def sumkron_backward(x, a, w, dy, *, workspace=None, stream=None, wait_timeout_us=0):
+    """Gradients of SumKronLinear for dy [B,T,D]: returns (dx [B,S,D], da [k,T,S],
+    dw [k,D,D], workspace) (bf16 CUDA tensors)."""
+    import torch
+    B, S, D = x.shape
+    k, T, _ = a.shape
+    p = gdpa_sumkron_params_t(int(B), int(S), int(T), int(D), int(k), int(wait_timeout_us), 0)
+    dx = torch.empty_like(x)
+    da = torch.empty_like(a)
+    dw = torch.empty_like(w)
+    if workspace is None:
+        n = gdpa_sumkron_backward_workspace_size(p)
+        if n == 0:
+            raise GdpaError(2, "gdpa_sumkron_backward_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check(gdpa_sumkron_backward(p, _ptr(x), _ptr(a), _ptr(w), _ptr(dy), _ptr(dx), _ptr(da),
+                                 _ptr(dw), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "gdpa_sumkron_backward")
+    return dx, da, dw, workspace
 
 
 def rotary_apply(x, table, *, inverse=False, out=None, stream=None):
