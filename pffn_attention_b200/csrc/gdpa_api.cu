@@ -609,16 +609,15 @@ gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k
   a.wr = p->window_right;
   a.debug_flags = p->debug_flags;
   a.timeout_ns = timeout_ns(p);
+  // dQ = R^T dQ', dK = R^T dK' (the turn is orthogonal): in the kernel's epilogue
+  a.rope_q = static_cast<const uint32_t*>(p->rope_q);
+  a.rope_kv = static_cast<const uint32_t*>(p->rope_kv);
   for (int phi = 0; phi <= 3; ++phi) {
     const uint64_t heads = phi_heads(p, phi);
     if (!heads) continue;
     a.phi = phi;
     a.head_mask = heads;
     e = launch_backward(a, p->D, tq, tk, tv, tdo, L.grid, s);
-    if (e != cudaSuccess) return GDPA_ERR_CUDA;
-  }
-  if (p->rope_q) {  // dQ = R^T dQ', dK = R^T dK' (the turn is orthogonal), in place
-    e = turn_qk(p, dq, dk, dq, dk, 1, sms, s);
     if (e != cudaSuccess) return GDPA_ERR_CUDA;
   }
   return GDPA_OK;

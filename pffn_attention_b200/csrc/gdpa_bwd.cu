@@ -38,12 +38,18 @@
 // (bf16, the MN-major A operand of dQ), which also stages the dK, dV rows at
 // the end of a key block; LSE / delta rows of two tiles.
 //
+// With the rotary temporal embedding the kernel reads turned Q and K and turns
+// dQ and dK back (the transpose of each token's turn) in its epilogue, so no
+// pass over the gradients follows it.
+//
 // Warp roles (512 threads): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator and
 // LSE / delta loader, 3 idle; warpgroups 1-2 compute P and dS (a thread owns
 // one key, each warpgroup half of the tile's 128 query columns); warpgroup 3
 // drains dQ from TMEM (summing it over key blocks in a per-CTA fp32 scratch
 // slot) and writes dK, dV at the end of each key block.
 #include <climits>
+
+#include <cuda_fp16.h>
 
 #include "gdpa_internal.h"
 
@@ -688,6 +694,28 @@ __device__ void bwd_compute(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem)
 #undef CMP_WAIT
 }
 
+// (x0, x1) turned back by the angle whose (cos, sin) is the fp16 pair cs (the
+// transpose of the forward turn of a rotary pair).
+__device__ __forceinline__ void unturn_pair(float& x0, float& x1, uint32_t cs) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cs));
+  const float y0 = fmaf(x0, f.x, x1 * f.y);
+  x1 = fmaf(x1, f.x, -x0 * f.y);
+  x0 = y0;
+}
+// 32 consecutive values (16 rotary pairs from pair p0) of a row turned back by
+// the token's table row.
+__device__ __forceinline__ void unturn32(float* v, const uint32_t* row, int p0) {
+  const uint4* t = reinterpret_cast<const uint4*>(row + p0);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 cs = __ldg(t + q);
+    unturn_pair(v[8 * q + 0], v[8 * q + 1], cs.x);
+    unturn_pair(v[8 * q + 2], v[8 * q + 3], cs.y);
+    unturn_pair(v[8 * q + 4], v[8 * q + 5], cs.z);
+    unturn_pair(v[8 * q + 6], v[8 * q + 7], cs.w);
+  }
+}
+
 // ------------------------------------------------------------------ reducer warpgroup
 // Thread = query row r of the tile for dQ, key row r of the block for dK/dV.
 // dQ of a pair is summed over the key blocks that reach its tile in this CTA's
@@ -699,7 +727,9 @@ __device__ void bwd_compute(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem)
 // half's read without waiting on a global load.  Final dQ rows go straight to
 // global memory (a thread writes its own row); dK and dV rows are staged in
 // this warp's quarter of the dS panel (free once the block's last dQ MMA has
-// completed) and written as whole rows.
+// completed) and written as whole rows.  With the rotary embedding, final dQ
+// rows and dK rows are turned back (by the transpose of their token's turn)
+// as they are written.
 template <class C>
 __device__ void bwd_reduce(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) {
   volatile int* abort = sm.abort_flag();
@@ -816,6 +846,12 @@ __device__ void bwd_reduce(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) 
                                   make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]),
                                   pol_keep);
             } else if (row_ok) {
+              if (a.rope_q) {
+#pragma unroll
+                for (int c = 0; c < HW; c += 32)
+                  unturn32(v + c, a.rope_q + (t.q0 + m0 + r) * (int64_t)(C::D / 2),
+                           (h * HW + c) / 2);
+              }
 #pragma unroll
               for (int c8 = 0; c8 < HW / 8; ++c8)
                 *reinterpret_cast<uint4*>(dq_row + h * HW + c8 * 8) = make_uint4(
@@ -841,6 +877,8 @@ __device__ void bwd_reduce(const BwdArgs& a, const BSmem<C>& sm, uint32_t tmem) 
               float kr[32];
               tmem_ld32f(tmem + tl + C::T_DK + ck * 32, kr);
               tmem_wait_ld();
+              if (a.rope_kv && wkey + lane < t.Lk)
+                unturn32(kr, a.rope_kv + (t.k0 + wkey + lane) * (int64_t)(C::D / 2), ck * 16);
               stage_chunk(ck, kr, a.scale);
             }
             flush_rows(a.dk + (int64_t)t.h * C::D, (int64_t)t.k0 + wkey, t.Lk - wkey);

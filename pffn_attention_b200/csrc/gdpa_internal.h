@@ -100,6 +100,11 @@ struct BwdArgs {
   int debug_flags;
   uint64_t timeout_ns;
   uint64_t head_mask;       // heads this launch computes (bit h), ~0 = all
+  // rotary temporal embedding: per-token (cos, sin) fp16 pairs [total][D/2];
+  // the kernel ran on turned Q and K, and turns dQ and dK back as it writes
+  // them.  nullptr = no rotation.
+  const uint32_t* rope_q;
+  const uint32_t* rope_kv;
 };
 
 // Per problem of a grouped forward launch, for its schedule: the problem's
