@@ -79,6 +79,15 @@ struct FwdCfg {
   // one MMA issuer per slot (warps 1 and 3), or one for both when warps 2-3
   // turn Q and K (rotary)
   static constexpr bool DUAL = !ROPE_;
+  // per-slot issuers with 64-key blocks send S in two halves so that phi of
+  // block i + 1 starts after half an S (see role_mma_slot); with 128-key
+  // blocks the two N = 64 halves cost more tensor time than the overlap
+  // returns (measured), so S goes whole after the previous PV
+  static constexpr bool SPLIT = DUAL && BN_ == 64;
+  // phi of odd blocks takes the key chunks in descending order and writes P
+  // over the upper half of the S columns (what a split S needs; the one-issuer
+  // kernels with 64-key blocks do the same, so both compute the same values)
+  static constexpr bool ALT = BN_ == 64;
   static constexpr int BM = kBlockM;
   // Q/K/V panels: 64 bf16 (128 B) wide with 128-byte swizzle, or 32 wide
   // (64 B, 64-byte swizzle) when D = 32.
@@ -117,8 +126,11 @@ struct FwdCfg {
   static constexpr int B_KVFULL = B_QEMPTY + NQ;
   // K/V stage i released by MMA issuer j: [2i + j] (one issuer: j = 0 only)
   static constexpr int B_KVEMPTY = B_KVFULL + NKV;
+  // S of a key block in halves (per-slot issuers): SFULL the half phi takes
+  // first, SFULLB the other (one issuer: SFULL the whole block)
   static constexpr int B_SFULL = B_KVEMPTY + 2 * NKV;
-  static constexpr int B_PFULL = B_SFULL + 2;
+  static constexpr int B_SFULLB = B_SFULL + 2;
+  static constexpr int B_PFULL = B_SFULLB + 2;
   static constexpr int B_PVDONE = B_PFULL + 2;
   static constexpr int B_OFULL = B_PVDONE + 2;
   static constexpr int B_OEMPTY = B_OFULL + 2;
@@ -565,9 +577,12 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
           const uint64_t vd = vdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk) {
-            // A = P [128 x BN] from TMEM (bf16 pairs, 8 columns per 16 keys);
+            // A = P [128 x BN] from TMEM (bf16 pairs, 8 columns per 16 keys,
+            // over the lower half of the S columns; the upper half for odd
+            // blocks of the slot with 64-key blocks);
             // B = V [BN keys x D], N (= D) contiguous: MN-major, 16 keys per step
-            mma_bf16_ts(tslot + C::TMEM_O, tslot + kk * 8,
+            mma_bf16_ts(tslot + C::TMEM_O,
+                        tslot + ((C::ALT && (z.pc & 1)) ? C::BN / 2 : 0) + kk * 8,
                         desc_add(vd, (kk * 16 * C::PANEL_BYTES) >> 4), idesc_o,
                         (z.npv > 0 || kk > 0) ? 1u : 0u);
           }
@@ -607,11 +622,16 @@ __device__ void role_mma(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem) {
   }
 }
 
-// One slot's MMA issuer (warp 1 for slot 0, warp 3 for slot 1): S of block i,
-// then PV of block i once the phi warpgroup has written P, then S of block
-// i + 1 once that PV has completed (P lives in the S columns).  It waits on
-// its own slot's barriers only, so neither slot's MMAs wait for the other
-// slot's events.
+// One slot's MMA issuer (warp 1 for slot 0, warp 3 for slot 1).  S of a key
+// block goes in two halves of BN/2 keys: phi writes block i's P over one half
+// of the S columns (the lower half for even i, the upper for odd i) and reads
+// the other half first in block i + 1.  So once block i's phi is done, the
+// issuer sends S of block i + 1 into the half without P, then block i's PV,
+// then the other half of S over block i's P (one thread's tcgen05.mma
+// execute in issue order, so that half is written after the PV has read P):
+// phi of block i + 1 starts after half an S, not after PV + S.  The issuer
+// waits on its own slot's barriers only, so neither slot's MMAs wait for the
+// other slot's events.
 //
 // Each issuer reads every tile record, to release K/V stages: a stage use
 // (one ring index) is released by both issuers, each with a commit on its own
@@ -624,6 +644,7 @@ template <class C>
 __device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int s) {
   volatile int* abort = sm.abort_flag();
   constexpr uint32_t idesc_s = make_idesc_bf16(kBlockM, C::BN, 0, 0);
+  constexpr uint32_t idesc_h = make_idesc_bf16(kBlockM, C::BN / 2, 0, 0);
   constexpr uint32_t idesc_o = make_idesc_bf16(kBlockM, C::D, 0, 1);
   constexpr uint32_t SBO = 8 * C::PANEL_BYTES;
   const uint64_t qdesc0 = make_smem_desc(sm.q(0), 16, SBO, C::LAYOUT);
@@ -655,6 +676,63 @@ __device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
     return true;
   };
 
+  // S = Q K^T into the slot's columns: all BN keys (h < 0), or half h (keys
+  // [h BN/2, (h+1) BN/2) into columns [h BN/2, (h+1) BN/2))
+  auto issue_s = [&](int qst, int st, int h) {
+    const int h0 = h < 0 ? 0 : h;
+    const uint64_t qd = qdesc0 + (uint64_t)((qst * C::Q_BYTES) >> 4);
+    const uint64_t kd =
+        kdesc0 + (uint64_t)((st * C::KV_BYTES + h0 * (C::BN / 2) * C::PANEL_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::D / 16; ++kk) {
+      const int pnl = kk * 16 / C::PANEL_ELEMS;
+      const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
+      mma_bf16_ss(tslot + h0 * (C::BN / 2),
+                  desc_add(qd, (pnl * kBlockM * C::PANEL_BYTES + within) >> 4),
+                  desc_add(kd, (pnl * C::BN * C::PANEL_BYTES + within) >> 4),
+                  h < 0 ? idesc_s : idesc_h, kk > 0 ? 1u : 0u);
+    }
+  };
+  // the block whose PV is still to be issued
+  struct PendPV {
+    bool valid, first, last, resident;
+    int st, podd;  // its K/V stage; its P over the upper half of the S columns
+    uint32_t use;  // its K/V ring index
+  } pend{};
+  // O += P V of that block (its P complete), then its releases
+  auto issue_pv = [&](const PendPV& b) -> bool {
+    if (b.first && !mbar_wait(sm.bar(C::B_OEMPTY + s), (tq & 1) ^ 1, abort, a.status,
+                              a.timeout_ns, 0x100 + C::B_OEMPTY + s))
+      return false;
+    tc_fence_after();
+    const uint64_t vd = vdesc0 + (uint64_t)((b.st * C::KV_BYTES) >> 4);
+    const uint32_t pcol = tslot + (b.podd ? C::BN / 2 : 0);
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk)
+      mma_bf16_ts(tslot + C::TMEM_O, pcol + kk * 8,
+                  desc_add(vd, (kk * 16 * C::PANEL_BYTES) >> 4), idesc_o,
+                  (!b.first || kk > 0) ? 1u : 0u);
+    mma_commit(sm.bar(C::B_PVDONE + s));
+    if (!b.resident || --kv_left[b.st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + 2 * b.st + s));
+    if (b.last) {
+      mma_commit(sm.bar(C::B_OFULL + s));
+      ++tq;
+    }
+    return true;
+  };
+  // Waiting for K/V ring index u while the pending PV holds its stage: the
+  // producer loads indices in order and cannot reach u past a reuse of that
+  // stage (an index at least NKV beyond the pending one) before the PV has
+  // released it, so issue the PV first.
+  auto clear_for = [&](uint32_t u) -> bool {
+    if (!pend.valid || (int)(u - pend.use) < C::NKV) return true;
+    if (!mbar_wait(sm.bar(C::B_PFULL + s), (pc - 1) & 1, abort, a.status, a.timeout_ns,
+                   0x100 + C::B_PFULL + s))
+      return false;
+    pend.valid = false;
+    return issue_pv(pend);
+  };
+
   TileRing<C, false> ring(0, 1);
   FTile x{};
   while (ring.next(a, sm, x)) {
@@ -668,6 +746,8 @@ __device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
       const int n_mine = x.resident ? (x.ntile + (x.slot == s ? 1 : 0)) / 2 : (mine ? 1 : 0);
       for (int j = 0; j < nb && (x.resident || !mine); ++j) {
         const int st = (int)((x.kv0 + (uint32_t)j) % C::NKV);
+        // the pending PV's count or release of this stage comes first
+        if (!clear_for(x.kv0 + (uint32_t)j)) return;
         if (n_mine == 0) {
           // not before the producer has taken the stage for this use: a
           // release ahead of its wait would complete the phase it waits on
@@ -684,43 +764,54 @@ __device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
     for (int idx = 0; idx < nb; ++idx) {
       const uint32_t ring_i = x.kv0 + (uint32_t)idx;
       const int st = (int)(ring_i % C::NKV);
-      // ---- S = Q K^T
       if (idx == 0) {
         if (!wait_tag(sm.q_tag() + qst, (int)x.qi, 0x180 + qst)) return;
         MMA_WAIT(C::B_QFULL + qst, (x.qi / C::NQ) & 1, 0x100 + C::B_QFULL + qst);
       }
+      if (!clear_for(ring_i)) return;
       if (!wait_tag(sm.kv_tag() + st, (int)ring_i, 0x190 + st)) return;
       MMA_WAIT(C::B_KVFULL + st, (ring_i / C::NKV) & 1, 0x100 + C::B_KVFULL + st);
-      if (pc > 0) MMA_WAIT(C::B_PVDONE + s, (pc - 1) & 1, 0x100 + C::B_PVDONE + s);
-      tc_fence_after();
-      const uint64_t qd = qdesc0 + (uint64_t)((qst * C::Q_BYTES) >> 4);
-      const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
-#pragma unroll
-      for (int kk = 0; kk < C::D / 16; ++kk) {
-        const int pnl = kk * 16 / C::PANEL_ELEMS;
-        const int within = (kk * 16 % C::PANEL_ELEMS) * 2;
-        mma_bf16_ss(tslot, desc_add(qd, (pnl * kBlockM * C::PANEL_BYTES + within) >> 4),
-                    desc_add(kd, (pnl * C::BN * C::PANEL_BYTES + within) >> 4), idesc_s,
-                    kk > 0 ? 1u : 0u);
+      if constexpr (!C::SPLIT) {
+        // ---- S whole, once the previous PV has read P; then PV once phi is done
+        if (pc > 0) MMA_WAIT(C::B_PVDONE + s, (pc - 1) & 1, 0x100 + C::B_PVDONE + s);
+        tc_fence_after();
+        issue_s(qst, st, -1);
+        mma_commit(sm.bar(C::B_SFULL + s));
+        if (idx == nb - 1) mma_commit(sm.bar(C::B_QEMPTY + qst));
+        MMA_WAIT(C::B_PFULL + s, pc & 1, 0x100 + C::B_PFULL + s);
+        PendPV b{true, idx == 0, idx == nb - 1, x.resident != 0, st, 0, ring_i};
+        if (!issue_pv(b)) return;
+        ++pc;
+        continue;
       }
-      mma_commit(sm.bar(C::B_SFULL + s));
-      if (idx == nb - 1) mma_commit(sm.bar(C::B_QEMPTY + qst));
-      // ---- O += P V
-      MMA_WAIT(C::B_PFULL + s, pc & 1, 0x100 + C::B_PFULL + s);
-      if (idx == 0) MMA_WAIT(C::B_OEMPTY + s, (tq & 1) ^ 1, 0x100 + C::B_OEMPTY + s);
+      // ---- S of block pc, the half phi takes first: into the columns the
+      // previous block's phi has read and not written (its P is over the
+      // other half)
+      if (pend.valid) MMA_WAIT(C::B_PFULL + s, (pc - 1) & 1, 0x100 + C::B_PFULL + s);
       tc_fence_after();
-      const uint64_t vd = vdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
-#pragma unroll
-      for (int kk = 0; kk < C::BN / 16; ++kk)
-        mma_bf16_ts(tslot + C::TMEM_O, tslot + kk * 8,
-                    desc_add(vd, (kk * 16 * C::PANEL_BYTES) >> 4), idesc_o,
-                    (idx > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(sm.bar(C::B_PVDONE + s));
-      if (!x.resident || --kv_left[st] == 0) mma_commit(sm.bar(C::B_KVEMPTY + 2 * st + s));
+      const int first_half = (int)(pc & 1);  // odd blocks take the upper keys first
+      issue_s(qst, st, first_half);
+      mma_commit(sm.bar(C::B_SFULL + s));
+      // ---- O += P V of the previous block
+      if (pend.valid && !issue_pv(pend)) return;
+      // ---- the other half of S, over the previous block's P: issued after
+      // that block's PV, and one thread's tcgen05.mma execute in issue order
+      issue_s(qst, st, first_half ^ 1);
+      mma_commit(sm.bar(C::B_SFULLB + s));
+      if (idx == nb - 1) mma_commit(sm.bar(C::B_QEMPTY + qst));
+      pend.valid = true;
+      pend.st = st;
+      pend.first = idx == 0;
+      pend.last = idx == nb - 1;
+      pend.resident = x.resident != 0;
+      pend.podd = (int)(pc & 1);
+      pend.use = ring_i;
       ++pc;
     }
-    mma_commit(sm.bar(C::B_OFULL + s));
-    ++tq;
+  }
+  if (pend.valid) {
+    MMA_WAIT(C::B_PFULL + s, (pc - 1) & 1, 0x100 + C::B_PFULL + s);
+    issue_pv(pend);
   }
 #undef MMA_WAIT
 }
@@ -965,11 +1056,25 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
       float factor = 1.f;
       const uint64_t half2 = f2_pack(0.5f, 0.5f);
       uint64_t ps2[2] = {0ull, 0ull};  // packed partial sums (softmax)
-      // P = phi(x), 32 columns at a time, written back as bf16 pairs over the
-      // S columns: chunk c0 lands in columns [c0/2, c0/2 + 16), which only
-      // hold S columns of chunks already read
+      // P = phi(x), 32 columns at a time, written back as bf16 pairs over one
+      // half of the S columns.  Blocks take the chunks in ascending order and
+      // write chunk ci's pairs to columns [16 ci, 16 ci + 16), except odd
+      // blocks of the slot with 64-key blocks (ALT), which take them in
+      // descending order and write them to BN/2 + [16 ci, 16 ci + 16).  Either
+      // way a chunk's pairs land on S columns of chunks already read.  With a
+      // split S (per-slot issuers, 64-key blocks) S comes in two halves: the
+      // one read first, then (SFULLB) the other.
+      constexpr int NCH = C::BN / 32;
+      const bool odd = C::ALT && (nsb & 1) != 0;
+      const int pbase = odd ? C::BN / 2 : 0;
 #pragma unroll 1
-      for (int c0 = 0; c0 < C::BN; c0 += 32) {
+      for (int k = 0; k < NCH; ++k) {
+        const int ci = odd ? NCH - 1 - k : k;
+        const int c0 = ci * 32;
+        if (C::SPLIT && k == NCH / 2) {
+          PHI_WAIT(C::B_SFULLB + s, nsb & 1, 0x400 + C::B_SFULLB + s);
+          tc_fence_after();
+        }
         uint32_t v[32];
         scores(c0, v);
         if (SOFTMAX) {
@@ -992,10 +1097,12 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
               ps2[0] = f2_mul(ps2[0], f2);
               ps2[1] = f2_mul(ps2[1], f2);
             }
-            // the block's P pairs already written: columns [0, c0 / 2)
+            // the block's P pairs already written (k chunks)
             tmem_wait_st();
+            const int wlo = odd ? C::BN / 2 + 16 * (NCH - k) : 0;
+            const int whi = odd ? C::BN : 16 * k;
 #pragma unroll 1
-            for (int c = 0; c < c0 / 2; c += 16) {
+            for (int c = wlo; c < whi; c += 16) {
               uint32_t pr[16];
               tmem_ld16(tslot + c, pr);
               tmem_wait_ld();
@@ -1045,7 +1152,7 @@ __device__ void role_phi(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem, int
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-        tmem_st16(tslot + c0 / 2, pk);
+        tmem_st16(tslot + pbase + ci * 16, pk);
       }
       if (has_bias) {
         mbar_arrive(sm.bar(C::B_BEMPTY + 2 * s + bb));
@@ -1219,6 +1326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(sm.bar(C::B_SFULL + s), 1);
+      mbar_init(sm.bar(C::B_SFULLB + s), 1);
       mbar_init(sm.bar(C::B_PFULL + s), 128);
       mbar_init(sm.bar(C::B_PVDONE + s), 1);
       mbar_init(sm.bar(C::B_OFULL + s), 1);
