@@ -300,6 +300,44 @@ typedef struct {
   float* lse;                   /* [H][total_q] fp32 or NULL (softmax heads only) */
 } gdpa_forward_problem_t;
 
+/* One problem of a grouped backward: the arguments of gdpa_backward. */
+typedef struct {
+  gdpa_params_t params;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  const int32_t* q_offsets;
+  const int32_t* kv_offsets;
+  const float* bias;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dbias;                 /* optional, as in gdpa_backward */
+} gdpa_backward_problem_t;
+
+/* Workspace bytes of gdpa_backward_grouped: a status block, an offsets table
+ * and one gdpa_backward workspace per problem; 0 when a problem is invalid or
+ * n_problems is outside [1, 4096]. */
+GDPA_API size_t gdpa_backward_grouped_workspace_size(const gdpa_backward_problem_t* problems,
+                                                     int n_problems);
+
+/* Grouped backward for per-event training (Kunlun paper review §2.5,
+ * "Event-level Personalization"): the gradients of several independent GDPA
+ * problems in one call, each problem's outputs equal to those of
+ * gdpa_backward on it alone.  Every problem is validated as by gdpa_backward
+ * before anything is launched.  The problems' launches go onto the stream one
+ * problem after another (schedule, delta, backward kernels of each), each
+ * with its own part of the workspace; a last kernel gathers their device
+ * status into the status block at the workspace start, which
+ * gdpa_get_device_status reads (the first error of the first problem that
+ * reported one).  Asynchronous on stream. */
+GDPA_API gdpa_status_t gdpa_backward_grouped(const gdpa_backward_problem_t* problems,
+                                             int n_problems, void* workspace,
+                                             size_t workspace_bytes, gdpa_stream_t stream);
+
 /* Workspace bytes of gdpa_forward_grouped for these problems; 0 when they are
  * invalid or exceed the limits above. */
 GDPA_API size_t gdpa_forward_grouped_workspace_size(const gdpa_forward_problem_t* problems,

@@ -196,6 +196,54 @@ bool make_map_3d(CUtensorMap* m, const void* base, const cuuint64_t (&dims)[3],
   return r == CUDA_SUCCESS;
 }
 
+// Everything gdpa_backward checks about one problem's arguments (the
+// workspace aside) before any launch.
+gdpa_status_t check_backward_args(const gdpa_params_t* p, const void* q, const void* k,
+                                  const void* v, const void* o, const void* dout,
+                                  const float* lse, const int32_t* q_offsets,
+                                  const int32_t* kv_offsets, const float* bias, const void* dq,
+                                  const void* dk, const void* dv, const float* dbias) {
+  gdpa_status_t st = check_params(p);
+  if (st != GDPA_OK) return st;
+  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
+  // a bias gradient needs a bias; it is fp32 [H][total_kv]
+  if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
+  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  const bool softmax = any_softmax(p);
+  if (p->total_q > 0 && (!q || !dout || !dq || (softmax && (!o || !lse))))
+    return GDPA_ERR_INVALID_ARG;
+  if (p->total_kv > 0 && (!k || !v || !dk || !dv)) return GDPA_ERR_INVALID_ARG;
+  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return GDPA_ERR_INVALID_ARG;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
+  return GDPA_OK;
+}
+
+// The grouped backward's status: the first error (in problem order) of the
+// problems' own status blocks at base + table[i].
+__global__ void gdpa_gather_status_kernel(DeviceStatus* dst, const uint8_t* base,
+                                          const uint64_t* table, int n) {
+  int count = 0;
+  for (int i = 0; i < n; ++i) {
+    const DeviceStatus* src = reinterpret_cast<const DeviceStatus*>(base + table[i]);
+    if (src->code != 0 && dst->code == 0) {
+      dst->code = src->code;
+      dst->where = src->where;
+    }
+    count += src->count;
+  }
+  dst->count = count;
+}
+
+cudaError_t launch_gather_status(DeviceStatus* dst, const uint8_t* base, const uint64_t* table,
+                                 int n, cudaStream_t s) {
+  gdpa_gather_status_kernel<<<1, 1, 0, s>>>(dst, base, table, n);
+  return cudaGetLastError();
+}
+
 gdpa_status_t check_sumkron(const gdpa_sumkron_params_t* p) {
   if (!p) return GDPA_ERR_INVALID_ARG;
   if (p->B < 0 || p->S <= 0 || p->T <= 0 || p->D <= 0 || p->k <= 0 || p->wait_timeout_us < 0)
@@ -505,27 +553,72 @@ gdpa_status_t gdpa_forward(const gdpa_params_t* p, const void* q, const void* k,
   return GDPA_OK;
 }
 
+size_t gdpa_backward_grouped_workspace_size(const gdpa_backward_problem_t* problems,
+                                            int n_problems) {
+  if (!problems || n_problems <= 0 || n_problems > 4096) return 0;
+  size_t off = align256(sizeof(DeviceStatus)) + align256((size_t)n_problems * 8);
+  for (int i = 0; i < n_problems; ++i) {
+    const size_t w = gdpa_workspace_size(&problems[i].params, 1);
+    if (w == 0) return 0;
+    off += align256(w);
+  }
+  return off;
+}
+
+gdpa_status_t gdpa_backward_grouped(const gdpa_backward_problem_t* problems, int n_problems,
+                                    void* workspace, size_t workspace_bytes,
+                                    gdpa_stream_t stream) {
+  if (!problems || n_problems <= 0 || n_problems > 4096) return GDPA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_problems; ++i) {
+    const gdpa_backward_problem_t& b = problems[i];
+    const gdpa_status_t st =
+        check_backward_args(&b.params, b.q, b.k, b.v, b.o, b.dout, b.lse, b.q_offsets,
+                            b.kv_offsets, b.bias, b.dq, b.dk, b.dv, b.dbias);
+    if (st != GDPA_OK) return st;
+  }
+  if (!workspace || !aligned16(workspace)) return workspace ? GDPA_ERR_INVALID_ARG
+                                                           : GDPA_ERR_WORKSPACE;
+  const size_t need = gdpa_backward_grouped_workspace_size(problems, n_problems);
+  if (need == 0) return GDPA_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return GDPA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<uint64_t> offs(n_problems);
+  size_t off = align256(sizeof(DeviceStatus)) + align256((size_t)n_problems * 8);
+  for (int i = 0; i < n_problems; ++i) {
+    offs[i] = off;
+    off += align256(gdpa_workspace_size(&problems[i].params, 1));
+  }
+  // the table is staged before cudaMemcpyAsync returns (pageable host memory)
+  uint64_t* table = reinterpret_cast<uint64_t*>(ws + align256(sizeof(DeviceStatus)));
+  if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), s) != cudaSuccess ||
+      cudaMemcpyAsync(table, offs.data(), offs.size() * 8, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess)
+    return GDPA_ERR_CUDA;
+  for (int i = 0; i < n_problems; ++i) {
+    const gdpa_backward_problem_t& b = problems[i];
+    const size_t w = gdpa_workspace_size(&b.params, 1);
+    const gdpa_status_t st =
+        gdpa_backward(&b.params, b.q, b.k, b.v, b.o, b.dout, b.lse, b.q_offsets, b.kv_offsets,
+                      b.bias, b.dq, b.dk, b.dv, b.dbias, ws + offs[i], w, stream);
+    if (st != GDPA_OK) return st;
+  }
+  return launch_gather_status(reinterpret_cast<DeviceStatus*>(ws), ws, table, n_problems, s) ==
+                 cudaSuccess
+             ? GDPA_OK
+             : GDPA_ERR_CUDA;
+}
+
 gdpa_status_t gdpa_backward(const gdpa_params_t* p, const void* q, const void* k, const void* v,
                             const void* o, const void* dout, const float* lse,
                             const int32_t* q_offsets, const int32_t* kv_offsets,
                             const float* bias, void* dq, void* dk, void* dv, float* dbias,
                             void* workspace, size_t workspace_bytes, gdpa_stream_t stream) {
-  gdpa_status_t st = check_params(p);
+  gdpa_status_t st = check_backward_args(p, q, k, v, o, dout, lse, q_offsets, kv_offsets, bias,
+                                         dq, dk, dv, dbias);
   if (st != GDPA_OK) return st;
-  if (!q_offsets || !kv_offsets) return GDPA_ERR_INVALID_ARG;
-  // a bias gradient needs a bias; it is fp32 [H][total_kv]
-  if (dbias && p->bias_kind == GDPA_BIAS_NONE) return GDPA_ERR_INVALID_ARG;
-  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 3u)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return GDPA_ERR_INVALID_ARG;
   const bool softmax = any_softmax(p);
-  if (p->total_q > 0 && (!q || !dout || !dq || (softmax && (!o || !lse))))
-    return GDPA_ERR_INVALID_ARG;
-  if (p->total_kv > 0 && (!k || !v || !dk || !dv)) return GDPA_ERR_INVALID_ARG;
-  if ((p->bias_kind != GDPA_BIAS_NONE) != (bias != nullptr)) return GDPA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
-    return GDPA_ERR_INVALID_ARG;
-  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GDPA_ERR_INVALID_ARG;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return GDPA_ERR_INVALID_ARG;
   int sms = 0;
   if (!device_info(&sms)) return GDPA_ERR_UNSUPPORTED;
   const WorkspaceLayout L = make_layout(p, 1, sms);

@@ -28,7 +28,8 @@ EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_s
             "gdpa_version", "gdpa_forward_no_alloc", "gdpa_forward_grouped_workspace_size",
             "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table",
             "gdpa_rotary_apply", "gdpa_sumkron_workspace_size", "gdpa_sumkron_forward",
-            "gdpa_sumkron_backward_workspace_size", "gdpa_sumkron_backward")
+            "gdpa_sumkron_backward_workspace_size", "gdpa_sumkron_backward",
+            "gdpa_backward_grouped_workspace_size", "gdpa_backward_grouped")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -59,6 +60,12 @@ class gdpa_forward_problem_t(ctypes.Structure):
                 ("v", ctypes.c_void_p), ("q_offsets", ctypes.c_void_p),
                 ("kv_offsets", ctypes.c_void_p), ("bias", ctypes.c_void_p),
                 ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+
+
+class gdpa_backward_problem_t(ctypes.Structure):
+    _fields_ = [("params", gdpa_params_t)] + [
+        (n, ctypes.c_void_p) for n in ("q", "k", "v", "o", "dout", "lse", "q_offsets",
+                                       "kv_offsets", "bias", "dq", "dk", "dv", "dbias")]
 
 
 class GdpaError(RuntimeError):
@@ -105,6 +112,11 @@ def load(path: str = LIB_PATH):
     lib.gdpa_forward_grouped_workspace_size.restype = sz
     lib.gdpa_forward_grouped.argtypes = [FP, ctypes.c_int, vp, sz, st]
     lib.gdpa_forward_grouped.restype = ctypes.c_int
+    BP = ctypes.POINTER(gdpa_backward_problem_t)
+    lib.gdpa_backward_grouped_workspace_size.argtypes = [BP, ctypes.c_int]
+    lib.gdpa_backward_grouped_workspace_size.restype = sz
+    lib.gdpa_backward_grouped.argtypes = [BP, ctypes.c_int, vp, sz, st]
+    lib.gdpa_backward_grouped.restype = ctypes.c_int
     lib.gdpa_rotary_table_bytes.argtypes = [ctypes.c_int, ctypes.c_int64]
     lib.gdpa_rotary_table_bytes.restype = sz
     lib.gdpa_rotary_table.argtypes = [ctypes.POINTER(gdpa_rotary_params_t), ctypes.c_int,
@@ -408,6 +420,53 @@ def forward_grouped(problems, *, workspace=None, stream=None):
         workspace = torch.empty(n, dtype=torch.uint8, device=problems[0]["q"].device)
     rc = gdpa_forward_grouped(arr, _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "gdpa_forward_grouped")
+    return outs, workspace
+
+
+def gdpa_backward_grouped_workspace_size(problems) -> int:
+    """problems: a ctypes array of gdpa_backward_problem_t (or None)."""
+    n = 0 if problems is None else len(problems)
+    return int(load().gdpa_backward_grouped_workspace_size(problems, n))
+
+
+def gdpa_backward_grouped(problems, workspace, workspace_bytes, stream) -> int:
+    n = 0 if problems is None else len(problems)
+    return int(load().gdpa_backward_grouped(problems, n, workspace, workspace_bytes, stream))
+
+
+def backward_grouped(problems, *, workspace=None, stream=None):
+    """Gradients of several GDPA problems in one call.  problems: a list of
+    dicts with q, k, v, o, dout, lse, q_offsets, kv_offsets (optional bias,
+    dbias) and the keyword arguments of backward().  Returns
+    ([(dq, dk, dv), ...], workspace)."""
+    import torch
+    arr = (gdpa_backward_problem_t * len(problems))()
+    outs, keep = [], []
+    for i, d in enumerate(problems):
+        q, k, v = d["q"], d["k"], d["v"]
+        total_q, H, D = q.shape
+        p = make_params(d["q_offsets"].numel() - 1, H, D, total_q, k.shape[0],
+                        phi=d.get("phi", "silu"), scale=d.get("scale", 1.0),
+                        window=d.get("window", (-1, -1)), bias_kind=d.get("bias_kind", "none"),
+                        max_seqlen_q=d.get("max_seqlen_q", 0),
+                        max_seqlen_kv=d.get("max_seqlen_kv", 0), head_phi=d.get("head_phi"),
+                        rope=d.get("rope"))
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        keep.append(p)
+        arr[i].params = p
+        for name, t in (("q", q), ("k", k), ("v", v), ("o", d.get("o")), ("dout", d["dout"]),
+                        ("lse", d.get("lse")), ("q_offsets", d["q_offsets"]),
+                        ("kv_offsets", d["kv_offsets"]), ("bias", d.get("bias")), ("dq", dq),
+                        ("dk", dk), ("dv", dv), ("dbias", d.get("dbias"))):
+            setattr(arr[i], name, _ptr(t))
+        outs.append((dq, dk, dv))
+    if workspace is None:
+        n = gdpa_backward_grouped_workspace_size(arr)
+        if n == 0:
+            raise GdpaError(1, "gdpa_backward_grouped_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=problems[0]["q"].device)
+    rc = gdpa_backward_grouped(arr, _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "gdpa_backward_grouped")
     return outs, workspace
 
 

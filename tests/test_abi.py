@@ -132,6 +132,32 @@ def test_grouped_forward_validation(lib):
     assert gdpa.gdpa_forward_grouped(good, FAKE + 16, 1 << 20, None) == 1
 
 
+def test_grouped_backward_validation(lib):
+    """The grouped backward checks every problem as gdpa_backward would before
+    any launch; its workspace is the status block, the offsets table and one
+    backward workspace per problem."""
+    def arr(*params):
+        a = (gdpa.gdpa_backward_problem_t * len(params))()
+        for i, p in enumerate(params):
+            a[i].params = p
+            for name in ("q", "k", "v", "o", "dout", "lse", "q_offsets", "kv_offsets", "dq",
+                         "dk", "dv"):
+                setattr(a[i], name, FAKE)
+        return a
+    assert gdpa.gdpa_backward_grouped_workspace_size(None) == 0
+    p1, p2 = _params(), _params(H=3, D=128, phi=1)
+    good = arr(p1, p2)
+    n = gdpa.gdpa_backward_grouped_workspace_size(good)
+    each = gdpa.gdpa_workspace_size(p1, 1) + gdpa.gdpa_workspace_size(p2, 1)
+    assert n >= each + 256 + 256
+    assert gdpa.gdpa_backward_grouped_workspace_size(arr(_params(), _params(D=48))) == 0
+    nobias = arr(_params(bias_kind=2))  # a gate without its tensor
+    assert gdpa.gdpa_backward_grouped(nobias, FAKE, 1 << 30, None) == 1
+    assert gdpa.gdpa_backward_grouped(None, FAKE, 1 << 30, None) == 1
+    assert gdpa.gdpa_backward_grouped(good, FAKE + 8, 1 << 30, None) == 1  # unaligned
+    assert gdpa.gdpa_backward_grouped(good, FAKE, n - 1, None) == 3        # workspace short
+
+
 def test_rotary_validation(lib):
     """Rotary tables: D, time scale, jagged sizes and alignment are checked on
     the host; the tables must come as a pair; the streamed turn adds the

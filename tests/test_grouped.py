@@ -177,3 +177,38 @@ def test_grouped_at_the_entry_limit(cuda_lib):
     for (w, _), (o, _) in zip(probs, outs):
         ro, _ = oracle.forward_workload(w)
         compare("O", o, ro)
+
+
+def _kw(d):
+    return {k: d[k] for k in ("phi", "scale", "window", "bias", "bias_kind", "max_seqlen_q",
+                              "max_seqlen_kv")}
+
+
+def test_backward_grouped_equals_separate_calls_and_oracle(cuda_lib):
+    """The grouped backward gives each problem exactly gdpa_backward's
+    gradients (bit for bit) and matches the oracle."""
+    items = []
+    for i, (w, hp) in enumerate(_problems()):
+        if hp is not None:
+            continue
+        d = _to_dev(w, None)
+        o, lse, ws0 = cuda_lib.forward(d["q"], d["k"], d["v"], d["q_offsets"], d["kv_offsets"],
+                                       **_kw(d))
+        assert cuda_lib.device_status(ws0) == 0
+        g = torch.Generator().manual_seed(600 + i)
+        dout = (torch.randn(w.q.shape, generator=g) * 0.25).to(torch.bfloat16)
+        d.update(o=o, lse=lse, dout=dout.cuda())
+        items.append((w, d, dout))
+    outs, ws = cuda_lib.backward_grouped([d for _, d, _ in items])
+    assert cuda_lib.device_status(ws) == 0
+    torch.cuda.synchronize()
+    for (w, d, dout), (dq, dk, dv) in zip(items, outs):
+        dq1, dk1, dv1, ws1 = cuda_lib.backward(d["q"], d["k"], d["v"], d["o"], d["dout"],
+                                               d["lse"], d["q_offsets"], d["kv_offsets"],
+                                               **_kw(d))
+        assert cuda_lib.device_status(ws1) == 0
+        assert torch.equal(dq, dq1) and torch.equal(dk, dk1) and torch.equal(dv, dv1)
+        rdq, rdk, rdv, _ = oracle.backward_workload(w, dout=dout)
+        compare("dQ", dq, rdq)
+        compare("dK", dk, rdk)
+        compare("dV", dv, rdv)
