@@ -225,7 +225,7 @@ GDPA_API size_t gdpa_sumkron_backward_workspace_size(const gdpa_sumkron_params_t
  * All bf16 row-major device arrays, 16-byte aligned, the caller's; fp32
  * accumulation (the sums over samples are split into fp32 partials in the
  * workspace and added in fp32).  x, a, w are the forward's inputs.  Same
- * parameter limits as the forward, and B <= 65535; B = 0 gives zero da and
+ * parameter limits as the forward; B = 0 gives zero da and
  * dw.  The workspace's status is cleared on the stream first (read it with
  * gdpa_get_device_status; GDPA_ERR_TIMEOUT if a bounded wait ran out).
  * Asynchronous on stream.  Errors (before any launch): as

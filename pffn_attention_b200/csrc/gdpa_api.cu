@@ -974,7 +974,6 @@ gdpa_status_t gdpa_sumkron_backward(const gdpa_sumkron_params_t* p, const void* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), s) != cudaSuccess) return GDPA_ERR_CUDA;
   const int B = p->B, S = p->S, T = p->T, D = p->D, k = p->k, kT = k * T;
-  if (B > 65535) return GDPA_ERR_UNSUPPORTED;  // samples are a grid dimension
   if (B == 0) {  // no sample: the parameter gradients are zero
     if (cudaMemsetAsync(da, 0, (size_t)kT * S * 2, s) != cudaSuccess ||
         cudaMemsetAsync(dw, 0, (size_t)k * D * D * 2, s) != cudaSuccess)
@@ -1002,7 +1001,7 @@ gdpa_status_t gdpa_sumkron_backward(const gdpa_sumkron_params_t* p, const void* 
   g.status = reinterpret_cast<DeviceStatus*>(ws);
   g.timeout_ns = (uint64_t)(p->wait_timeout_us > 0 ? p->wait_timeout_us : 2000000) * 1000ull;
   auto run = [&](const CUtensorMap& ta, const CUtensorMap& tb) {
-    return launch_gemm(g, ta, tb, s) == cudaSuccess;
+    return launch_gemm(g, ta, tb, sms, s) == cudaSuccess;
   };
   // Z_b = A X_b: M = kT, N = D, K = S; per sample
   g.M = kT; g.N = D; g.Z = B; g.n_rb = 1; g.nkc = S / 64; g.kc = 64; g.splits = 1;

@@ -2,13 +2,15 @@
 // backward (Kunlun paper review §2.4: its gradients are plain contractions;
 // see gdpa_api.cu for which products they are).
 //
-// One CTA per (output tile 128 x 128, split of the reduction batches, grid
-// batch).  The K loop runs over the CTA's reduction batches and, within each,
-// over the batch's K chunks; A and B chunks come through a ring of shared
-// memory stages by TMA, the MMAs accumulate in TMEM (128 columns), and the
-// epilogue writes the tile as fp32 partial sums or as bf16 at the caller's
-// layout.  Rows or columns past the operands' extents load as zeros, and
-// output rows or columns past M, N are not written.
+// Persistent CTAs walk work units (output tile 128 x 128, split of the
+// reduction batches, grid batch).  Per unit the K loop runs over the unit's
+// reduction batches and, within each, over the batch's K chunks; A and B
+// chunks come through a ring of shared memory stages by TMA (the ring runs on
+// across units), the MMAs accumulate into one of two TMEM accumulators (128
+// columns each), and the epilogue writes a unit's tile, as fp32 partial sums
+// or as bf16 at the caller's layout, while the MMAs of the next unit go into
+// the other accumulator.  Rows or columns past the operands' extents load as
+// zeros, and output rows or columns past M, N are not written.
 //
 // Warp roles (256 threads): warp 0 TMA producer (one thread); warp 1 MMA
 // issuer (one thread); warp 2 TMEM allocator; warps 4-7 epilogue, one TMEM
@@ -32,8 +34,10 @@ struct GemmCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kGemmStages * OP_BYTES;
   static constexpr int OFF_BAR = OFF_B + kGemmStages * OP_BYTES;
-  static constexpr int B_FULL = 0, B_EMPTY = kGemmStages, B_DONE = 2 * kGemmStages;
-  static constexpr int NBARS = 2 * kGemmStages + 1;
+  // ring stages; accumulator a full (MMAs done) / empty (epilogue read it)
+  static constexpr int B_FULL = 0, B_EMPTY = kGemmStages, B_ACCFULL = 2 * kGemmStages,
+                       B_ACCEMPTY = 2 * kGemmStages + 2;
+  static constexpr int NBARS = 2 * kGemmStages + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem addr, abort flag
   static constexpr int SMEM = OFF_MISC + 16;
   static_assert(OP_BYTES % 1024 == 0, "swizzle atoms");
@@ -70,18 +74,30 @@ __global__ void __launch_bounds__(kGemmThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int mtiles = (g.M + kGemmTile - 1) / kGemmTile;
-  const int tm = blockIdx.x % mtiles, tn = blockIdx.x / mtiles;
-  const int split = blockIdx.y, z = blockIdx.z;
-  const int rb0 = (int)((int64_t)g.n_rb * split / g.splits);
-  const int rb1 = (int)((int64_t)g.n_rb * (split + 1) / g.splits);
-  const int steps = (rb1 - rb0) * g.nkc;
+  const int ntiles = (g.N + kGemmTile - 1) / kGemmTile;
+  const int tiles = mtiles * ntiles;
+  const int64_t units = (int64_t)tiles * g.splits * g.Z;
+  // unit u: tile u % tiles, split (u / tiles) % splits, grid batch u / (tiles splits)
+  auto unit_of = [&](int64_t u, int& tm, int& tn, int& split, int& z, int& rb0, int& steps) {
+    const int t = (int)(u % tiles);
+    tm = t % mtiles;
+    tn = t / mtiles;
+    split = (int)((u / tiles) % g.splits);
+    z = (int)(u / ((int64_t)tiles * g.splits));
+    rb0 = (int)((int64_t)g.n_rb * split / g.splits);
+    const int rb1 = (int)((int64_t)g.n_rb * (split + 1) / g.splits);
+    steps = (rb1 - rb0) * g.nkc;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGemmStages; ++i) {
       mbar_init(bar(C::B_FULL + i), 1);
       mbar_init(bar(C::B_EMPTY + i), 1);
     }
-    mbar_init(bar(C::B_DONE), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_ACCFULL + i), 1);
+      mbar_init(bar(C::B_ACCEMPTY + i), 128);
+    }
     *abort = 0;
     fence_mbar_init();
   }
@@ -90,7 +106,7 @@ __global__ void __launch_bounds__(kGemmThreads)
     tma_prefetch_desc(&tb);
   }
   if (warp == 2) {
-    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -100,31 +116,37 @@ __global__ void __launch_bounds__(kGemmThreads)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---- producer: A and B chunks of every step into the ring
+      // ---- producer: A and B chunks of every step of every unit into the ring
       const uint64_t pol = l2_policy_evict_last();
-      for (int i = 0; i < steps; ++i) {
-        const int st = i % kGemmStages;
-        if (!mbar_wait(bar(C::B_EMPTY + st), ((i / kGemmStages) & 1) ^ 1, abort, g.status,
-                       g.timeout_ns, 0x7000 + st))
-          break;
-        mbar_arrive_expect_tx(bar(C::B_FULL + st), 2 * C::OP_BYTES);
-        const int rb = rb0 + i / g.nkc, j = i % g.nkc;
-        const uint32_t sa = base + C::OFF_A + st * C::OP_BYTES;
-        const uint32_t sb = base + C::OFF_B + st * C::OP_BYTES;
-        int c0, c1, c2;
-        for (int p = 0; p < (g.a.mn_major ? 2 : 1); ++p) {
-          operand_coords(g.a, KC, tm, p, j, rb, z, c0, c1, c2);
-          tma_load_3d(sa + p * (C::OP_BYTES / 2), &ta, bar(C::B_FULL + st), c0, c1, c2, pol);
-        }
-        for (int p = 0; p < (g.b.mn_major ? 2 : 1); ++p) {
-          operand_coords(g.b, KC, tn, p, j, rb, z, c0, c1, c2);
-          tma_load_3d(sb + p * (C::OP_BYTES / 2), &tb, bar(C::B_FULL + st), c0, c1, c2, pol);
+      uint32_t i = 0;  // ring steps so far
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, split, z, rb0, steps;
+        unit_of(u, tm, tn, split, z, rb0, steps);
+        for (int j = 0; j < steps; ++j, ++i) {
+          const int st = (int)(i % kGemmStages);
+          ok = mbar_wait(bar(C::B_EMPTY + st), ((i / kGemmStages) & 1) ^ 1, abort, g.status,
+                         g.timeout_ns, 0x7000 + st);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(C::B_FULL + st), 2 * C::OP_BYTES);
+          const int rb = rb0 + j / g.nkc, kc = j % g.nkc;
+          const uint32_t sa = base + C::OFF_A + st * C::OP_BYTES;
+          const uint32_t sb = base + C::OFF_B + st * C::OP_BYTES;
+          int c0, c1, c2;
+          for (int p = 0; p < (g.a.mn_major ? 2 : 1); ++p) {
+            operand_coords(g.a, KC, tm, p, kc, rb, z, c0, c1, c2);
+            tma_load_3d(sa + p * (C::OP_BYTES / 2), &ta, bar(C::B_FULL + st), c0, c1, c2, pol);
+          }
+          for (int p = 0; p < (g.b.mn_major ? 2 : 1); ++p) {
+            operand_coords(g.b, KC, tn, p, kc, rb, z, c0, c1, c2);
+            tma_load_3d(sb + p * (C::OP_BYTES / 2), &tb, bar(C::B_FULL + st), c0, c1, c2, pol);
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---- MMA issuer: KC / 16 MMAs of K = 16 per step into the TMEM tile
+      // ---- MMA issuer: KC / 16 MMAs of K = 16 per step into the unit's accumulator
       const uint32_t idesc = make_idesc_bf16(kGemmTile, kGemmTile, g.a.mn_major, g.b.mn_major);
       // K-major tile: 128 rows x 128 bytes (one swizzle panel), 16 elements =
       // 32 bytes per K step; MN-major tile: two panels of 64 M (or N) x KC
@@ -133,37 +155,58 @@ __global__ void __launch_bounds__(kGemmThreads)
       const uint32_t lbo_b = g.b.mn_major ? KC * 128 : 16;
       const uint32_t ka = g.a.mn_major ? (16 * 128) >> 4 : 32 >> 4;
       const uint32_t kb = g.b.mn_major ? (16 * 128) >> 4 : 32 >> 4;
+      uint32_t i = 0, n = 0;  // ring steps; units with steps (accumulator uses)
       bool ok = true;
-      for (int i = 0; i < steps && ok; ++i) {
-        const int st = i % kGemmStages;
-        ok = mbar_wait(bar(C::B_FULL + st), (i / kGemmStages) & 1, abort, g.status, g.timeout_ns,
-                       0x7100 + st);
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, split, z, rb0, steps;
+        unit_of(u, tm, tn, split, z, rb0, steps);
+        if (steps == 0) continue;
+        const int acc = (int)(n & 1);
+        // the epilogue has read this accumulator's previous unit
+        ok = mbar_wait(bar(C::B_ACCEMPTY + acc), ((n >> 1) & 1) ^ 1, abort, g.status,
+                       g.timeout_ns, 0x7140 + acc);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t da = make_smem_desc(base + C::OFF_A + st * C::OP_BYTES, lbo, 1024,
-                                           LAYOUT_SW128);
-        const uint64_t db = make_smem_desc(base + C::OFF_B + st * C::OP_BYTES, lbo_b, 1024,
-                                           LAYOUT_SW128);
+        const uint32_t tacc = tmem + acc * kGemmTile;
+        for (int j = 0; j < steps; ++j, ++i) {
+          const int st = (int)(i % kGemmStages);
+          ok = mbar_wait(bar(C::B_FULL + st), (i / kGemmStages) & 1, abort, g.status,
+                         g.timeout_ns, 0x7100 + st);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t da = make_smem_desc(base + C::OFF_A + st * C::OP_BYTES, lbo, 1024,
+                                             LAYOUT_SW128);
+          const uint64_t db = make_smem_desc(base + C::OFF_B + st * C::OP_BYTES, lbo_b, 1024,
+                                             LAYOUT_SW128);
 #pragma unroll
-        for (int kk = 0; kk < KC / 16; ++kk)
-          mma_bf16_ss(tmem, desc_add(da, kk * ka), desc_add(db, kk * kb), idesc,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(C::B_EMPTY + st));
+          for (int kk = 0; kk < KC / 16; ++kk)
+            mma_bf16_ss(tacc, desc_add(da, kk * ka), desc_add(db, kk * kb), idesc,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(C::B_EMPTY + st));
+        }
+        if (!ok) break;
+        mma_commit(bar(C::B_ACCFULL + acc));  // after every MMA of the unit
+        ++n;
       }
-      if (ok) mma_commit(bar(C::B_DONE));  // after every MMA of the tile
     }
   } else if (warp >= 4) {
-    // ---- epilogue: thread = output row
+    // ---- epilogue: thread = output row of each unit
     const int wq = warp & 3;
-    const int m = tm * kGemmTile + wq * 32 + lane;
+    uint32_t n = 0;
     bool ok = true;
-    if (steps > 0) {
-      ok = mbar_wait(bar(C::B_DONE), 0, abort, g.status, g.timeout_ns, 0x7180);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-    }
-    if (ok) {
-      const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int tm, tn, split, z, rb0, steps;
+      unit_of(u, tm, tn, split, z, rb0, steps);
+      const int m = tm * kGemmTile + wq * 32 + lane;
+      const int acc = (int)(n & 1);
+      if (steps > 0) {
+        ok = mbar_wait(bar(C::B_ACCFULL + acc), (n >> 1) & 1, abort, g.status, g.timeout_ns,
+                       0x7180 + acc);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16) + acc * kGemmTile;
 #pragma unroll 1
       for (int c0 = 0; c0 < kGemmTile; c0 += 32) {
         const int n0 = tn * kGemmTile + c0;
@@ -194,6 +237,11 @@ __global__ void __launch_bounds__(kGemmThreads)
                            pack_bf16x2(v[e + 4], v[e + 5]), pack_bf16x2(v[e + 6], v[e + 7]));
         }
       }
+      if (steps > 0) {  // the accumulator may take a later unit
+        tc_fence_before();
+        mbar_arrive(bar(C::B_ACCEMPTY + acc));
+        ++n;
+      }
     }
   }
   __syncwarp();
@@ -209,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads)
   }
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -234,14 +282,18 @@ __global__ void __launch_bounds__(256)
 
 template <int KC>
 cudaError_t launch_kc(const GemmLaunch& g, const CUtensorMap& ta, const CUtensorMap& tb,
-                      cudaStream_t s) {
+                      int sms, cudaStream_t s) {
   using C = GemmCfg<KC>;
   auto kern = gdpa_gemm_kernel<KC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const int mtiles = (g.M + kGemmTile - 1) / kGemmTile;
-  const int ntiles = (g.N + kGemmTile - 1) / kGemmTile;
-  dim3 grid(mtiles * ntiles, g.splits, g.Z);
+  const int64_t units = (int64_t)((g.M + kGemmTile - 1) / kGemmTile) *
+                       ((g.N + kGemmTile - 1) / kGemmTile) * g.splits * g.Z;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemmThreads, C::SMEM);
+  if (e != cudaSuccess) return e;
+  per_sm = std::max(1, std::min(per_sm, 2));  // two 256-column TMEM allocations per SM
+  const int grid = (int)std::min<int64_t>(units, (int64_t)sms * per_sm);
   kern<<<grid, kGemmThreads, C::SMEM, s>>>(g, ta, tb);
   return cudaGetLastError();
 }
@@ -249,12 +301,12 @@ cudaError_t launch_kc(const GemmLaunch& g, const CUtensorMap& ta, const CUtensor
 }  // namespace
 
 cudaError_t launch_gemm(const GemmLaunch& g, const CUtensorMap& ta, const CUtensorMap& tb,
-                        cudaStream_t s) {
+                        int sms, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || g.Z <= 0 || g.splits <= 0 || g.n_rb < 0 || g.nkc <= 0)
     return cudaErrorInvalidValue;
-  if (g.Z > 65535 || g.splits > 65535) return cudaErrorInvalidValue;
-  if (g.kc == 64) return launch_kc<64>(g, ta, tb, s);
-  if (g.kc == 32 && g.a.mn_major && g.b.mn_major) return launch_kc<32>(g, ta, tb, s);
+  if (sms <= 0) return cudaErrorInvalidValue;
+  if (g.kc == 64) return launch_kc<64>(g, ta, tb, sms, s);
+  if (g.kc == 32 && g.a.mn_major && g.b.mn_major) return launch_kc<32>(g, ta, tb, sms, s);
   return cudaErrorInvalidValue;
 }
 

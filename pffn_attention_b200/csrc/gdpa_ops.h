@@ -86,7 +86,7 @@ struct GemmLaunch {
   uint64_t timeout_ns;
 };
 cudaError_t launch_gemm(const GemmLaunch& g, const CUtensorMap& ta, const CUtensorMap& tb,
-                        cudaStream_t s);
+                        int sms, cudaStream_t s);
 // out[i] = bf16(sum over s < splits of part[s * count + i]), i < count (count % 8 == 0).
 cudaError_t launch_sum_splits(const float* part, int splits, int64_t count, __nv_bfloat16* out,
                               int sms, cudaStream_t s);
