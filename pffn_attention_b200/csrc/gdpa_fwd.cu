@@ -772,8 +772,9 @@ __device__ void role_mma_slot(const FwdArgs& a, const Smem<C>& sm, uint32_t tmem
       if (!wait_tag(sm.kv_tag() + st, (int)ring_i, 0x190 + st)) return;
       MMA_WAIT(C::B_KVFULL + st, (ring_i / C::NKV) & 1, 0x100 + C::B_KVFULL + st);
       if constexpr (!C::SPLIT) {
-        // ---- S whole, once the previous PV has read P; then PV once phi is done
-        if (pc > 0) MMA_WAIT(C::B_PVDONE + s, (pc - 1) & 1, 0x100 + C::B_PVDONE + s);
+        // ---- S whole over the previous block's P: issued after that block's
+        // PV by this thread, so it executes after the PV has read P (no wait
+        // for the PV's completion); then PV once phi is done
         tc_fence_after();
         issue_s(qst, st, -1);
         mma_commit(sm.bar(C::B_SFULL + s));
