@@ -39,6 +39,7 @@
 // workspace status, all roles leave their loops, TMEM is freed and the kernel
 // returns.
 #include <algorithm>
+#include <atomic>
 #include <cfloat>
 #include <climits>
 
@@ -70,6 +71,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kInvSqrt2 = 0.7071067811865476f;  // Phi(x) = (1 + erf(x / sqrt 2)) / 2
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8
 
+#ifndef GDPA_FWD_NQ
+#define GDPA_FWD_NQ 8
+#endif
+
 template <int D_, int BN_, bool GROUPED_, bool ROPE_ = false>
 struct FwdCfg {
   static constexpr int D = D_;
@@ -99,9 +104,10 @@ struct FwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;  // one K (or V) block
   // Q tiles come through a ring of NQ stages, so the producer loads a few tiles
   // ahead of the MMAs (one load's latency no longer sits in every tile's
-  // chain): 4 stages for D <= 64, 2 (one per slot) for D = 128, where shared
-  // memory is full.
-  static constexpr int NQ = D >= 128 ? 2 : 4;
+  // chain): 8 stages for D <= 64, 2 (one per slot) for D = 128, where shared
+  // memory is full.  (With short K/V, Q is nearly all a tile reads; 4, 6 and
+  // 8 stages measured within 1% of each other on the PFFN workload.)
+  static constexpr int NQ = D >= 128 ? 2 : GDPA_FWD_NQ;
   // K/V ring: 128 KB of stages for D = 128 (2 of 128 keys or 4 of 64), 64 KB
   // for smaller D, at most 8
   static constexpr int KV_RING = (D >= 128 ? 64 : 32) * 1024;
@@ -1315,6 +1321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm.base = smem_u32(smem_raw);
   sm.ptr = smem_raw;
   if (sm.base & 1023u) {  // swizzled TMA tiles need 1024-byte alignment
+    griddep_wait();
     if (threadIdx.x == 0) record_error(a.status, 2, 0x7000);
     return;
   }
@@ -1370,6 +1377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
+  // The set-up above touches only this CTA's own state, so it may overlap the
+  // schedule kernel before it; everything below reads that kernel's results.
+  griddep_wait();
 
   // Registers: the phi warpgroups take the most, the epilogue warpgroups the
   // fewest; each budget is set inside its own branch.
@@ -1420,25 +1430,47 @@ cudaError_t launch_one(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMa
                        cudaStream_t stream) {
   using C = FwdCfg<D, BN, GROUPED, ROPE>;
   auto kern = gdpa_fwd_kernel<D, BN, SOFTMAX, GROUPED, ROPE>;
-  // when the roles' register budgets differ, the raising side's setmaxnreg
-  // waits until the block's launch registers cover it: never launch a build
-  // whose per-thread count would leave that wait unsatisfiable
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  // The per-build checks and the shared-memory attribute, once per device.
+  static std::atomic<uint64_t> ready{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  constexpr bool kSplit =
-      kRegsControl != kRegsLaunch || kRegsPhi != kRegsLaunch || kRegsEpi != kRegsLaunch;
-  if (kSplit && fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsPhi + 256 * kRegsEpi)
-    return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, C::SMEM_ALLOC);
-  if (e != cudaSuccess) return e;
-  // the kernel allocates all 512 TMEM columns: exactly one CTA per SM
-  if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  const uint64_t dev_bit = dev >= 0 && dev < 64 ? 1ull << dev : 0;
+  if (!(ready.load(std::memory_order_acquire) & dev_bit)) {
+    // when the roles' register budgets differ, the raising side's setmaxnreg
+    // waits until the block's launch registers cover it: never launch a build
+    // whose per-thread count would leave that wait unsatisfiable
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    constexpr bool kSplit =
+        kRegsControl != kRegsLaunch || kRegsPhi != kRegsLaunch || kRegsEpi != kRegsLaunch;
+    if (kSplit && fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsPhi + 256 * kRegsEpi)
+      return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    // the kernel allocates all 512 TMEM columns: exactly one CTA per SM
+    if (per_sm != 1) return cudaErrorInvalidConfiguration;
+    ready.fetch_or(dev_bit, std::memory_order_acq_rel);
+  }
   const int grid = std::max(1, std::min(a.n_units, sms));
-  kern<<<grid, kThreads, C::SMEM_ALLOC, stream>>>(a, tq, tk, tv, to);
+  // programmatic stream serialization: the CTAs start their set-up while the
+  // schedule kernel before them finishes (the kernel waits before reading it)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a, tq, tk, tv, to);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -10,7 +10,14 @@
 //   tile_start[p] = query tiles of order[0..p).
 // One CTA: costs into shared memory as 64-bit keys (inverted cost, index) so
 // an ascending bitonic sort yields the order with unique keys, then a block
-// scan of the tile counts.  The kernel also clears the workspace status.
+// scan of the tile counts (kept in shared memory by sample from the first
+// pass).  Compare-exchange stages whose partners lie within one warp run on
+// shuffles in registers, so only the wider stages pass through shared memory
+// with a block barrier.  The kernel also clears the workspace status, and lets
+// the attention kernel that follows it start its set-up at once (that kernel
+// waits for this one's results before it reads them).
+#include <atomic>
+
 #include "gdpa_internal.h"
 
 namespace gdpa {
@@ -63,44 +70,38 @@ __device__ __forceinline__ bool sample_lengths(const int32_t* __restrict__ q_off
   return bad;
 }
 
-__global__ void __launch_bounds__(kSchedThreads)
-    gdpa_schedule_kernel(const int32_t* __restrict__ q_offsets,
-                         const int32_t* __restrict__ kv_offsets, int B, int BM, int BN, int wl,
-                         int wr, int32_t* __restrict__ tile_start, int32_t* __restrict__ order,
-                         int4* __restrict__ info, int max_q, int max_kv, int64_t total_q,
-                         int64_t total_kv, DeviceStatus* status) {
-  extern __shared__ unsigned long long keys[];
-  __shared__ long long warp_tot[kSchedThreads / 32];
+// One compare-exchange of element i with element i ^ j (j < 32: the partner
+// is lane ^ j of the same warp) in the bitonic merge of width k: the lower
+// index keeps the smaller key where the merge ascends ((i & k) == 0).
+__device__ __forceinline__ unsigned long long shfl_cmpx(unsigned long long x, int i, int j,
+                                                        int k) {
+  const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+  const bool keep_min = ((i & j) == 0) == ((i & k) == 0);
+  return keep_min ? (x < y ? x : y) : (x < y ? y : x);
+}
+
+// Ascending bitonic sort of keys[0, n) (n a power of two) by the whole block;
+// element i = r * kSchedThreads + tid belongs to thread tid (lane i % 32).
+// Returns after a block barrier.
+__device__ void block_bitonic_sort(unsigned long long* keys, int n) {
   const int tid = threadIdx.x;
-  if (status && tid == 0) {
-    status->code = 0;
-    status->where = 0;
-    status->count = 0;
+  const int per = (n + kSchedThreads - 1) / kSchedThreads;
+  // merges of width <= 32 stay inside a warp
+  for (int r = 0; r < per; ++r) {
+    const int i = r * kSchedThreads + tid;
+    unsigned long long x = i < n ? keys[i] : ~0ull;
+    for (int k = 2; k <= 32 && k <= n; k <<= 1)
+      for (int j = k >> 1; j > 0; j >>= 1) x = shfl_cmpx(x, i, j, k);
+    if (i < n) keys[i] = x;
   }
   __syncthreads();
-  int n = 1;
-  while (n < B) n <<= 1;
-  for (int i = tid; i < n; i += kSchedThreads) {
-    unsigned long long key = ~0ull;
-    if (i < B) {
-      int q0, Lq, k0, Lk;
-      sample_lengths(q_offsets, kv_offsets, i, info != nullptr, max_q, max_kv, total_q, total_kv,
-                     q0, Lq, k0, Lk);
-      unsigned long long c = sample_cost(Lq, Lk, BM, BN, wl, wr);
-      if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
-      key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
-    }
-    keys[i] = key;
-  }
-  __syncthreads();
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
+  for (int k = 64; k <= n; k <<= 1) {
+    for (int j = k >> 1; j >= 32; j >>= 1) {
       for (int i = tid; i < n; i += kSchedThreads) {
         const int ixj = i ^ j;
         if (ixj > i) {
           const unsigned long long x = keys[i], y = keys[ixj];
-          const bool ascending = (i & k) == 0;
-          if ((x > y) == ascending) {
+          if ((x > y) == ((i & k) == 0)) {
             keys[i] = y;
             keys[ixj] = x;
           }
@@ -108,25 +109,69 @@ __global__ void __launch_bounds__(kSchedThreads)
       }
       __syncthreads();
     }
+    for (int r = 0; r < per; ++r) {
+      const int i = r * kSchedThreads + tid;
+      unsigned long long x = i < n ? keys[i] : ~0ull;
+      for (int j = 16; j > 0; j >>= 1) x = shfl_cmpx(x, i, j, k);
+      if (i < n) keys[i] = x;
+    }
+    __syncthreads();
   }
-  // order, then an exclusive scan of the tile counts in that order
-  const int chunk = (B + kSchedThreads - 1) / kSchedThreads;
-  const int beg = min(B, tid * chunk), end = min(B, beg + chunk);
-  long long local = 0;
-  for (int p = beg; p < end; ++p) {
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+    gdpa_schedule_kernel(const int32_t* __restrict__ q_offsets,
+                         const int32_t* __restrict__ kv_offsets, int B, int BM, int BN, int wl,
+                         int wr, int32_t* __restrict__ tile_start, int32_t* __restrict__ order,
+                         int4* __restrict__ info, int max_q, int max_kv, int64_t total_q,
+                         int64_t total_kv, DeviceStatus* status) {
+  extern __shared__ unsigned long long keys[];  // n keys, then tiles[B]
+  __shared__ long long warp_tot[kSchedThreads / 32];
+  const int tid = threadIdx.x;
+  griddep_launch_dependents();
+  if (status && tid == 0) {
+    status->code = 0;
+    status->where = 0;
+    status->count = 0;
+  }
+  int n = 1;
+  while (n < B) n <<= 1;
+  int32_t* tiles = reinterpret_cast<int32_t*>(keys + n);  // query tiles by sample index
+  const bool check = info != nullptr;
+  for (int i = tid; i < n; i += kSchedThreads) {
+    unsigned long long key = ~0ull;
+    if (i < B) {
+      int q0, Lq, k0, Lk;
+      sample_lengths(q_offsets, kv_offsets, i, check, max_q, max_kv, total_q, total_kv, q0, Lq,
+                     k0, Lk);
+      unsigned long long c = sample_cost(Lq, Lk, BM, BN, wl, wr);
+      if (c > 0xFFFFFFFFull) c = 0xFFFFFFFFull;
+      key = ((0xFFFFFFFFull - c) << 32) | (unsigned long long)(unsigned)i;
+      tiles[i] = (Lq + BM - 1) / BM;
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  block_bitonic_sort(keys, n);
+  // the order and each sorted sample's descriptor (independent loads per thread)
+#pragma unroll 4
+  for (int p = tid; p < B; p += kSchedThreads) {
     const int b = (int)(keys[p] & 0xFFFFFFFFull);
     order[p] = b;
-    int q0, Lq, k0, Lk;
-    const bool bad = sample_lengths(q_offsets, kv_offsets, b, info != nullptr, max_q, max_kv,
-                                    total_q, total_kv, q0, Lq, k0, Lk);
-    local += (Lq + BM - 1) / BM;
     if (info) {
+      int q0, Lq, k0, Lk;
+      const bool bad = sample_lengths(q_offsets, kv_offsets, b, true, max_q, max_kv, total_q,
+                                      total_kv, q0, Lq, k0, Lk);
       // a sample outside the declared bounds is reported and skipped
       if (bad && status) record_error(status, 6, b);
       info[p] = make_int4(q0, Lq, k0, Lk);
     }
   }
-  // block-wide exclusive scan of `local`
+  // exclusive scan of the tile counts in sorted order, contiguous chunks
+  const int chunk = (B + kSchedThreads - 1) / kSchedThreads;
+  const int beg = min(B, tid * chunk), end = min(B, beg + chunk);
+  long long local = 0;
+  for (int p = beg; p < end; ++p) local += tiles[keys[p] & 0xFFFFFFFFull];
   const int lane = tid & 31, warp = tid >> 5;
   long long incl = local;
   for (int off = 1; off < 32; off <<= 1) {
@@ -148,10 +193,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   long long run = warp_tot[warp] + incl - local;
   for (int p = beg; p < end; ++p) {
     tile_start[p] = (int32_t)run;
-    int q0, Lq, k0, Lk;
-    sample_lengths(q_offsets, kv_offsets, order[p], info != nullptr, max_q, max_kv, total_q,
-                   total_kv, q0, Lq, k0, Lk);
-    run += (Lq + BM - 1) / BM;
+    run += tiles[keys[p] & 0xFFFFFFFFull];
   }
   if (end == B && beg < end) tile_start[B] = (int32_t)run;
   if (B == 0 && tid == 0) tile_start[0] = 0;
@@ -168,6 +210,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   extern __shared__ unsigned long long keys[];
   __shared__ GroupSchedProblem sp[kMaxGroupProblems];
   const int tid = threadIdx.x;
+  griddep_launch_dependents();
   const GroupSchedJob job = jobs[blockIdx.x];
   const GroupSchedProblem* __restrict__ probs = job.probs;
   const int n_probs = job.n_probs, n_entries = job.n_entries, BN = job.block_n;
@@ -200,22 +243,7 @@ __global__ void __launch_bounds__(kSchedThreads)
     keys[i] = key;
   }
   __syncthreads();
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < n; i += kSchedThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long x = keys[i], y = keys[ixj];
-          const bool ascending = (i & k) == 0;
-          if ((x > y) == ascending) {
-            keys[i] = y;
-            keys[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  block_bitonic_sort(keys, n);
   for (int pos = tid; pos < n_entries; pos += kSchedThreads) {
     const int e = (int)(keys[pos] & 0xFFFFFFFFull);
     const int p = problem_of(e);
@@ -251,13 +279,22 @@ cudaError_t launch_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                             int block_m, int block_n, int wl, int wr, int32_t* tile_start,
                             int32_t* order, int4* info, int max_q, int max_kv, int64_t total_q,
                             int64_t total_kv, DeviceStatus* status, cudaStream_t stream) {
+  if (B < 0 || B > kMaxSortBatch) return cudaErrorInvalidValue;
   int n = 1;
   while (n < B) n <<= 1;
-  const size_t smem = (size_t)n * sizeof(unsigned long long);
-  cudaError_t e = cudaFuncSetAttribute(gdpa_schedule_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(kMaxSortBatch * sizeof(unsigned long long)));
+  const size_t smem = (size_t)n * sizeof(unsigned long long) + (size_t)B * sizeof(int32_t);
+  // the shared-memory attribute, once per device
+  static std::atomic<uint64_t> ready{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t dev_bit = dev >= 0 && dev < 64 ? 1ull << dev : 0;
+  if (!(ready.load(std::memory_order_acquire) & dev_bit)) {
+    e = cudaFuncSetAttribute(gdpa_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kMaxSortBatch * (sizeof(unsigned long long) + sizeof(int32_t))));
+    if (e != cudaSuccess) return e;
+    ready.fetch_or(dev_bit, std::memory_order_acq_rel);
+  }
   gdpa_schedule_kernel<<<1, kSchedThreads, smem, stream>>>(q_offsets, kv_offsets, B, block_m,
                                                            block_n, wl, wr, tile_start, order,
                                                            info, max_q, max_kv, total_q, total_kv,
