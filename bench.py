@@ -81,9 +81,11 @@ def algorithmic_bytes(w, backward: bool) -> tuple[float, float]:
     return fwd, bwd
 
 
+# per entry of profiles/traffic.json: the sources of the kernels whose DRAM
+# bytes it records (the schedule kernel's few bytes are not in those figures)
 KERNEL_SOURCES = {
-    "gdpa_backward": ["gdpa_bwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
-    "gdpa_forward": ["gdpa_fwd.cu", "gdpa_schedule.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_backward": ["gdpa_bwd.cu", "gdpa_internal.h", "sm100.cuh"],
+    "gdpa_forward": ["gdpa_fwd.cu", "gdpa_internal.h", "sm100.cuh", "gdpa_pdl.cuh"],
     "gdpa_sumkron_forward": ["gdpa_sumkron.cu", "gdpa_ops.h", "gdpa_internal.h", "sm100.cuh"],
     "gdpa_rotary_apply": ["gdpa_rotary.cu", "gdpa_ops.h", "gdpa_internal.h", "sm100.cuh"],
 }

@@ -46,6 +46,7 @@
 #include <cuda_fp16.h>
 
 #include "gdpa_internal.h"
+#include "gdpa_pdl.cuh"
 
 namespace gdpa {
 namespace {

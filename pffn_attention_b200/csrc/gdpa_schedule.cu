@@ -19,6 +19,7 @@
 #include <atomic>
 
 #include "gdpa_internal.h"
+#include "gdpa_pdl.cuh"
 
 namespace gdpa {
 namespace {

@@ -30,18 +30,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
-// serialization may start while the kernel before it in the stream still
-// runs; griddep_wait() returns once that kernel has completed and its memory
-// writes are visible (a no-op for a kernel launched the ordinary way).
-// griddep_launch_dependents() lets the next such kernel start early.
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
