@@ -33,7 +33,8 @@
  *
  * Ownership: the caller allocates and frees everything (inputs, outputs and
  * the workspace).  The library never allocates, frees or synchronises,
- * except gdpa_get_device_status, which synchronises the stream it is given.
+ * except gdpa_get_device_status and gdpa_forward_no_alloc_status, which
+ * synchronise the stream they are given.
  * All launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  * default stream).  Calls that share one workspace must not overlap.
  *
@@ -364,13 +365,11 @@ GDPA_API gdpa_status_t gdpa_forward_grouped(const gdpa_forward_problem_t* proble
  * stream capture.  All calls on a device share the one array: calls that
  * overlap on the GPU (on different streams, or from different host threads)
  * race and must be serialised by the caller.  Each call overwrites what it
- * needs, so nothing from an earlier call leaks in.  Device-side status of
- * these calls is not readable through gdpa_get_device_status: a bounded wait
- * that runs out, or a sample that fails the device checks (see
- * GDPA_ERR_DEVICE_CHECK), leaves the affected O and LSE rows unwritten while
- * the call still returns GDPA_OK.  A caller that must detect this can fill O
- * with a sentinel (NaN) before the call, or check the offsets on the host
- * against max_seqlen_q / _kv and the totals.  With rotary
+ * needs, so nothing from an earlier call leaks in.  A bounded wait that runs
+ * out, or a sample that fails the device checks (see GDPA_ERR_DEVICE_CHECK),
+ * leaves the affected O and LSE rows unwritten while the call still returns
+ * GDPA_OK: read the call's device status with gdpa_forward_no_alloc_status.
+ * With rotary
  * tables (rope_q / rope_kv) the attention kernel turns Q and K itself (as
  * debug_flags bit 2 selects for gdpa_forward): no turned copies, the same
  * results bit for bit. */
@@ -379,6 +378,15 @@ GDPA_API gdpa_status_t gdpa_forward_no_alloc(const gdpa_params_t* p, const void*
                                              const int32_t* q_offsets,
                                              const int32_t* kv_offsets, const float* bias,
                                              void* o, float* lse, gdpa_stream_t stream);
+
+/* Device status of the last gdpa_forward_no_alloc call on the current device
+ * (the status block at the start of the built-in array): GDPA_OK,
+ * GDPA_ERR_TIMEOUT or GDPA_ERR_DEVICE_CHECK, as gdpa_get_device_status gives
+ * for a workspace.  Synchronises `stream` (the stream of that call) first,
+ * then copies the block to the host.  Every no-alloc call on a device clears
+ * and rewrites the one block, so read it before the next call.  GDPA_ERR_CUDA
+ * if the array's address cannot be looked up or the copy fails. */
+GDPA_API gdpa_status_t gdpa_forward_no_alloc_status(gdpa_stream_t stream);
 
 /* The jagged tile schedule the kernels use, exported so it can be checked:
  * query tiles of block_m rows, key blocks of block_n keys (both multiples of

@@ -74,3 +74,10 @@ extern "C" GDPA_API gdpa_status_t gdpa_forward_no_alloc(
   return gdpa_forward(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, scratch, kNoAllocBytes,
                       stream);
 }
+
+extern "C" GDPA_API gdpa_status_t gdpa_forward_no_alloc_status(gdpa_stream_t stream) {
+  void* scratch = scratch_for_current_device();
+  if (!scratch) return GDPA_ERR_CUDA;
+  // the status block is the array's first 256 bytes, as in a workspace
+  return gdpa_get_device_status(scratch, stream);
+}

@@ -29,7 +29,8 @@ EXPORTED = ("gdpa_workspace_size", "gdpa_forward", "gdpa_backward", "gdpa_tile_s
             "gdpa_forward_grouped", "gdpa_rotary_table_bytes", "gdpa_rotary_table",
             "gdpa_rotary_apply", "gdpa_sumkron_workspace_size", "gdpa_sumkron_forward",
             "gdpa_sumkron_backward_workspace_size", "gdpa_sumkron_backward",
-            "gdpa_backward_grouped_workspace_size", "gdpa_backward_grouped")
+            "gdpa_backward_grouped_workspace_size", "gdpa_backward_grouped",
+            "gdpa_forward_no_alloc_status")
 
 
 class gdpa_params_t(ctypes.Structure):
@@ -105,6 +106,8 @@ def load(path: str = LIB_PATH):
     lib.gdpa_status_string.restype = ctypes.c_char_p
     lib.gdpa_forward_no_alloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, st]
     lib.gdpa_forward_no_alloc.restype = ctypes.c_int
+    lib.gdpa_forward_no_alloc_status.argtypes = [st]
+    lib.gdpa_forward_no_alloc_status.restype = ctypes.c_int
     lib.gdpa_version.argtypes = []
     lib.gdpa_version.restype = ctypes.c_int
     FP = ctypes.POINTER(gdpa_forward_problem_t)
@@ -196,6 +199,12 @@ def gdpa_forward_no_alloc(p, q, k, v, q_offsets, kv_offsets, bias, o, lse, strea
     """Forward with the library's built-in scratch (no caller workspace)."""
     return int(load().gdpa_forward_no_alloc(ctypes.byref(p), q, k, v, q_offsets, kv_offsets,
                                             bias, o, lse, stream))
+
+
+def gdpa_forward_no_alloc_status(stream) -> int:
+    """Device status of the last no-alloc forward on the current device
+    (synchronises the stream)."""
+    return int(load().gdpa_forward_no_alloc_status(stream))
 
 
 def gdpa_backward(p, q, k, v, o, dout, lse, q_offsets, kv_offsets, bias, dq, dk, dv, dbias,

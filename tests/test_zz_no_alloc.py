@@ -32,6 +32,7 @@ def _run_both(gdpa, w):
                                     ko.data_ptr(), None if bias is None else bias.data_ptr(),
                                     o.data_ptr(), lse.data_ptr(), stream.cuda_stream)
     assert rc == 0, gdpa.gdpa_status_string(rc)
+    assert gdpa.gdpa_forward_no_alloc_status(stream.cuda_stream) == 0
     torch.cuda.synchronize()
     return ref_o, ref_lse, o, lse
 
@@ -54,6 +55,29 @@ def test_no_alloc_forward_matches_forward_on_consecutive_calls(cuda_lib):
         compare("O", o, ro)
         if w.phi == 1:
             np.testing.assert_allclose(lse.cpu().numpy(), rlse, atol=2e-3, rtol=0)
+
+
+def test_no_alloc_status_reports_malformed_offsets(cuda_lib):
+    """A sample whose offsets decrease is skipped and reported: the call
+    returns GDPA_OK, the built-in status block holds GDPA_ERR_DEVICE_CHECK, and
+    the next (well-formed) call clears it."""
+    w = make_workload(2, B=4, seed=503)
+    dev = torch.device("cuda")
+    q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+    ko = torch.tensor(w.kv_offsets, dtype=torch.int32, device=dev)
+    good = list(w.q_offsets)
+    bad = list(good)
+    bad[2] = bad[1] - 5  # sample 1 gets a negative length
+    stream = torch.cuda.current_stream().cuda_stream
+    p = cuda_lib.make_params(w.B, w.H, w.D, w.total_q, w.total_kv, phi=w.phi, scale=w.scale)
+    o = torch.full_like(q, float("nan"))
+    for offsets, expect in ((bad, 6), (good, 0)):  # 6: GDPA_ERR_DEVICE_CHECK
+        qo = torch.tensor(offsets, dtype=torch.int32, device=dev)
+        rc = cuda_lib.gdpa_forward_no_alloc(p, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            qo.data_ptr(), ko.data_ptr(), None, o.data_ptr(),
+                                            None, stream)
+        assert rc == 0, cuda_lib.gdpa_status_string(rc)
+        assert cuda_lib.gdpa_forward_no_alloc_status(stream) == expect
 
 
 def test_no_alloc_rejects_batches_beyond_its_scratch(cuda_lib):
